@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the megakernel engine.
+
+A step is one autoregressive decode step (every instruction class of the
+decode path: RMSNorm + QKV + RoPE + KV append, split-KV GQA attention,
+O projection, RMSNorm + gate/up + SiLU, down projection, final norm + LM head +
+argmax) of the Llama-3.2-1B-shaped model at batch 1, KV cache pre-filled to
+1024 positions, on seeded synthetic weights (bf16 ~N(0, 0.02)).  Prints one
+JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mk|reference]
+
+N > 1 runs under torchrun: batch-1 decode does not shard, so every rank runs
+an independent replica ("replicas only"); value = all ranks' steps / max time.
+--impl reference times the CPU oracle (the only reference this build has).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode steps/sec & µs/step (Llama-1B shape, batch 1); HBM GB/s as % of roofline"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=128)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    ap.add_argument("--workload", default="llama1b")
+    ap.add_argument("--exec-mode", default="megakernel", choices=["megakernel", "per_op", "per_op_graph"])
+    ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
+    ap.add_argument("--kv-splits", type=int, default=0)
+    ap.add_argument("--l2-prefetch-kb", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--breakdown", action="store_true", help="add a per-instruction-class time breakdown")
+    ap.add_argument("--no-logits", action="store_true", help="do not write logits_out")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def src_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_megakernel_interpreter_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("src_hash") == src_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.reasons = set()
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = None
+            try:
+                import torch
+                pr = torch.cuda.get_device_properties(index)
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                f = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = f(self.h)
+                for n, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def step_bytes(shape, weight_bytes: int, positions, logits: bool) -> float:
+    """Algorithmic HBM bytes of one step: weights streamed once (+ norm
+    vectors and one embedding row per sequence), the KV cache read over
+    positions 0..pos, the new K/V row written, fp32 logits written."""
+    L, H, d, nkv = shape.n_layers, shape.hidden, shape.head_dim, shape.n_kv_heads
+    norms = (2 * L + 1) * H * 2
+    per_pos = L * nkv * d * 2 * 2
+    tot = 0.0
+    for p in positions:
+        tot += weight_bytes + norms + H * 2 + per_pos * (p + 1) + per_pos + (shape.vocab * 4 if logits else 0)
+    return tot / len(positions)
+
+
+def dist_setup(n):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if n > 1 and world != n:
+        raise SystemExit(f"--gpus {n} needs torchrun with {n} ranks (WORLD_SIZE={world})")
+    return world, rank, local
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle (fp64) on this host's cores: the workload's decode steps,
+    a bounded sample of them."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    s = w.shape
+    model = synth.make_model(s)
+    k, v = synth.alloc_kv(s, 1, w.context + args.steps + args.warmup + 2)
+    synth.fill_kv_prefix(s, k, v, [w.context])
+    orc = oracle.Oracle(s, model, "f64")
+    tok = int(synth.first_tokens(w)[0])
+    pos = w.context
+    t0 = time.perf_counter()
+    lg = orc.decode_step(k, v, 0, tok, pos)
+    t_step = time.perf_counter() - t0
+    tok, pos = int(np.argmax(lg)), pos + 1
+    budget = 150.0
+    n = max(1, min(args.steps, int(budget / max(t_step, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        lg = orc.decode_step(k, v, 0, tok, pos)
+        tok, pos = int(np.argmax(lg)), pos + 1
+    el = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    val = n / el
+    sample = f"{n} of the {args.steps} requested decode steps of {args.workload} (1 untimed warm-up), fp64 oracle"
+    out = {"metric": METRIC, "value": val, "unit": "steps/s", "n_gpus": world, "steps": n, "warmup": 1,
+           "ms_per_step": 1e3 * el / n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic (seeded bf16 weights ~N(0,0.02), KV ~N(0,1))",
+           "config": {"workload": args.workload, "batch": 1, "context": w.context},
+           "impl": "reference",
+           "cpu_baseline": {"value": val, "unit": "steps/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": val, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def cpu_baseline(model, w, s, seconds=15.0):
+    import numpy as np
+    import oracle
+    import synth
+    k, v = synth.alloc_kv(s, 1, w.context + 64)
+    synth.fill_kv_prefix(s, k, v, [w.context])
+    orc = oracle.Oracle(s, model, "f64")
+    tok, pos = int(synth.first_tokens(w)[0]), w.context
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        lg = orc.decode_step(k, v, 0, tok, pos)
+        tok, pos, n = int(np.argmax(lg)), pos + 1, n + 1
+        el = time.perf_counter() - t0
+        if el >= seconds or n >= 60:
+            break
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": n / el, "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} consecutive decode steps of {w.name} (context {w.context}+), fp64 oracle, "
+                      f"{el:.1f} s of host time"}
+
+
+def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
+    import numpy as np
+    import torch
+    eng.plan(**{**eng.plan_kw, "trace": True})
+    pos = torch.tensor([pos0], dtype=torch.int32, device="cuda")
+    eng.decode_step(tokens, pos, logits, nxt)
+    torch.cuda.synchronize()
+    tr = eng.trace().astype(np.int64)
+    eng.plan(**eng.plan_kw)
+    ops = tr[:, 4] & 0xFF
+    t_start = tr[:, 0].min()
+    total = tr[:, 3].max() - t_start
+    out = {"step_us_traced": total / 1e3}
+    for op in sorted(set(ops.tolist())):
+        m = ops == op
+        wait = (tr[m, 1] - tr[m, 0]) / 1e3
+        body = (tr[m, 2] - tr[m, 1]) / 1e3
+        out[mk.OP_NAMES[int(op)]] = {"count": int(m.sum()), "mean_wait_us": float(wait.mean()),
+                                     "mean_body_us": float(body.mean()),
+                                     "sum_body_us_per_cta": float(body.sum() / info.num_ctas)}
+    return out
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    import numpy as np
+    import torch
+    import decode_megakernel_interpreter_b200 as mk
+    from decode_megakernel_interpreter_b200 import harness
+    import synth
+
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    w = synth.WORKLOADS[args.workload]
+    s = w.shape
+    B = w.batch
+    K, W = args.steps, args.warmup
+    ctx = int(w.lengths()[0])
+    max_seq = ctx + K + W + 2
+    model = synth.make_model(s)
+    dev = harness.upload_model(model, s.tied)
+    k, v = synth.alloc_kv(s, B, max_seq)
+    synth.fill_kv_prefix(s, k, v, w.lengths())
+    kc, vc = harness.upload_kv(k, v)
+    del k, v
+    eng = harness.make_engine(s, dev, kc, vc, B, max_seq)
+    plan_kw = dict(batch=B, kv_splits=args.kv_splits, sched=args.sched, exec_mode=args.exec_mode,
+                   l2_prefetch_kb=args.l2_prefetch_kb)
+    eng.plan_kw = plan_kw
+    info = eng.plan(**plan_kw)
+    stream = torch.cuda.current_stream()
+    first = torch.tensor(synth.first_tokens(w), dtype=torch.int32, device="cuda")
+    tokens = first.clone()  # next_tokens_out aliases tokens: device-to-device feedback
+    pos_all = torch.arange(ctx, ctx + max(K, W) + 1, dtype=torch.int32, device="cuda")
+    logits = None if args.no_logits else torch.empty(B, s.vocab, dtype=torch.float32, device="cuda")
+    lptr = logits.data_ptr() if logits is not None else None
+
+    def step(i):
+        rc = mk.mk_decode_step(eng.h, tokens.data_ptr(), pos_all.data_ptr() + 4 * i, lptr, tokens.data_ptr(),
+                               stream.cuda_stream)
+        if rc != mk.MK_OK:
+            raise mk.MkError(rc, "mk_decode_step")
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    rc = eng.status()
+    if rc != mk.MK_OK:
+        raise mk.MkError(rc, "warm-up")
+    tokens.copy_(first)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(stream)
+        for i in range(K):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    ms = ev0.elapsed_time(ev1)
+    rc = eng.status()
+    if rc != mk.MK_OK:
+        raise mk.MkError(rc, "timed steps")
+    if pg:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    us_step = 1e3 * ms / K
+    value = world * K / (ms / 1e3)
+    launches_per_step = 1 if args.exec_mode == "megakernel" else s.n_layers * 5 + 1
+
+    # end to end through the C ABI with host buffers: per step copy the token
+    # and position in from pinned memory, run, read the next token back
+    e2e = None
+    if not args.no_e2e:
+        h_tok = torch.empty(B, dtype=torch.int32, pin_memory=True)
+        h_pos = torch.empty(B, dtype=torch.int32, pin_memory=True)
+        h_next = torch.empty(B, dtype=torch.int32, pin_memory=True)
+        d_tok = torch.empty(B, dtype=torch.int32, device="cuda")
+        d_pos = torch.empty(B, dtype=torch.int32, device="cuda")
+        d_next = torch.empty(B, dtype=torch.int32, device="cuda")
+        h_tok.copy_(first.cpu())
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(K):
+            h_pos.fill_(ctx + i)
+            d_tok.copy_(h_tok, non_blocking=True)
+            d_pos.copy_(h_pos, non_blocking=True)
+            rc = mk.mk_decode_step(eng.h, d_tok.data_ptr(), d_pos.data_ptr(), lptr, d_next.data_ptr(),
+                                   stream.cuda_stream)
+            if rc != mk.MK_OK:
+                raise mk.MkError(rc, "e2e step")
+            h_next.copy_(d_next, non_blocking=True)
+            stream.synchronize()
+            h_tok.copy_(h_next)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if pg:
+            t = torch.tensor([ems], dtype=torch.float64, device="cuda")
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * K / (ems / 1e3), "unit": "steps/s", "h2d_bytes_per_step": 8 * B,
+               "d2h_bytes_per_step": 4 * B, "us_per_step": 1e3 * ems / K}
+
+    bd = breakdown(eng, mk, info, tokens, ctx, logits, torch.empty_like(tokens)) if args.breakdown else None
+    eng.close()
+
+    if rank == 0:
+        peak, peak_kind = peaks()
+        positions = [ctx + i for i in range(K)]
+        bytes_step = step_bytes(s, info.weight_bytes_per_step, positions, logits is not None) * B
+        achieved = bytes_step / (us_step * 1e-6) / 1e9
+        out = {
+            "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": us_step / 1e3, "us_per_step": us_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 weights, fp32 arithmetic", "data": "synthetic",
+            "config": {"workload": f"{w.name}: Llama-3.2-1B shape (16 layers, hidden 2048, 32/8 heads, head_dim 64, "
+                                   f"ffn 8192, vocab 128256, tied), batch {B}, KV pre-filled to {ctx}, "
+                                   f"{K} greedy steps" if w.name == "llama1b" else w.name,
+                       "batch": B, "context": ctx, "exec_mode": args.exec_mode, "sched": args.sched,
+                       "kv_splits": info.kv_splits, "ctas": info.num_ctas, "smem_pages": info.num_pages,
+                       "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (weights streamed once per step, 2.5 GB)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "peak_kind": peak_kind, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                         "traffic": ncu_traffic(args.workload), "algorithmic_bytes_per_step": bytes_step,
+                         "kernel": "mk::interp_kernel<1>"},
+            "clocks": clk.summary(),
+            "gpu_launches": K * launches_per_step,
+        }
+        if e2e:
+            out["e2e"] = e2e
+        if bd:
+            out["breakdown"] = bd
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(model, w, s)
+        print(json.dumps(out), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,697 @@
+// C ABI of the decode megakernel engine (declared in include/mk.h and
+// include/mk_host.h).  Host code: validation, device buffers, weight
+// repacking, the RoPE table, plan upload and launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "../../include/mk_host.h"
+#include "mk_internal.h"
+#include "planner.h"
+
+namespace mk {
+cudaError_t launch_interp(const KParams &p, int nb, int grid, int smem, cudaStream_t st, bool cooperative);
+cudaError_t occupancy_interp(int nb, int smem, int *blocks_per_sm);
+int shared_bytes_fixed(int num_pages, size_t act_floats);
+}  // namespace mk
+
+using namespace mk;
+
+static_assert(sizeof(mk_instr_desc) == sizeof(Instr), "mk_instr_desc mirrors Instr");
+
+struct mk_handle {
+  mk_config cfg;
+  Shape shape;
+  int device = 0, sm_count = 0, smem_optin = 0;
+  // borrowed
+  const uint16_t *embed = nullptr, *lm_head = nullptr, *final_norm = nullptr;
+  uint16_t *kc = nullptr, *vc = nullptr;
+  std::vector<mk_layer_weights> lw;
+  // owned for the handle's lifetime
+  std::vector<void *> allocs;
+  uint16_t *wqkv = nullptr, *wgu = nullptr, *wd = nullptr;
+  LayerDev *d_layers = nullptr;
+  float2 *d_rope = nullptr;
+  float *qbuf = nullptr, *obuf = nullptr, *xres = nullptr, *actb = nullptr, *dpart = nullptr;
+  unsigned *ctr_epoch = nullptr;  // [0] = epoch
+  int *status = nullptr;
+  // owned per plan
+  std::vector<void *> plan_allocs;
+  bool planned = false;
+  Plan plan;
+  mk_plan_opts opts;
+  KParams kp;
+  int smem = 0, grid = 0, nb = 1;
+  // per-op graph mode
+  cudaGraphExec_t gexec = nullptr;
+  const void *g_tokens = nullptr, *g_pos = nullptr, *g_logits = nullptr, *g_next = nullptr;
+};
+
+namespace {
+
+int cuda_code(cudaError_t e) {
+  if (e == cudaSuccess) return MK_OK;
+  if (e == cudaErrorMemoryAllocation) return MK_ERR_OUT_OF_MEMORY;
+  if (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorLaunchOutOfResources) return MK_ERR_LAUNCH;
+  return MK_ERR_CUDA;
+}
+
+#define MK_CUDA(call)                  \
+  do {                                 \
+    cudaError_t e_ = (call);           \
+    if (e_ != cudaSuccess) {           \
+      cudaGetLastError();              \
+      return cuda_code(e_);            \
+    }                                  \
+  } while (0)
+
+template <class T>
+int dalloc(std::vector<void *> &list, T **out, size_t count, bool zero = true) {
+  void *p = nullptr;
+  size_t bytes = std::max<size_t>(count * sizeof(T), 16);
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_OUT_OF_MEMORY;
+  }
+  list.push_back(p);
+  if (zero) {
+    e = cudaMemset(p, 0, bytes);
+    if (e != cudaSuccess) return MK_ERR_CUDA;
+  }
+  *out = static_cast<T *>(p);
+  return MK_OK;
+}
+
+void free_list(std::vector<void *> &list) {
+  for (void *p : list) cudaFree(p);
+  list.clear();
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+Shape shape_of(const mk_config &c) {
+  return Shape{c.n_layers, c.hidden, c.n_q_heads, c.n_kv_heads, c.head_dim, c.ffn, c.vocab};
+}
+
+// Copy rows of `row_elems` bf16 from src_ptrs[r] to dst + r * row_elems.
+__global__ void gather_rows_kernel(uint16_t *dst, const unsigned long long *src_ptrs, int row_elems,
+                                   long long n_rows) {
+  const int n16 = row_elems / 8;
+  for (long long r = blockIdx.x; r < n_rows; r += gridDim.x) {
+    const uint4 *s = reinterpret_cast<const uint4 *>(src_ptrs[r]);
+    uint4 *d = reinterpret_cast<uint4 *>(dst + r * (long long)row_elems);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) d[i] = s[i];
+  }
+}
+
+int gather_rows(uint16_t *dst, const std::vector<unsigned long long> &src, int row_elems) {
+  if (src.empty()) return MK_OK;
+  unsigned long long *d_src = nullptr;
+  MK_CUDA(cudaMalloc(&d_src, src.size() * sizeof(unsigned long long)));
+  cudaError_t e = cudaMemcpy(d_src, src.data(), src.size() * sizeof(unsigned long long), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) {
+    int blocks = (int)std::min<size_t>(src.size(), 65535);
+    gather_rows_kernel<<<blocks, 256>>>(dst, d_src, row_elems, (long long)src.size());
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  }
+  cudaFree(d_src);
+  return cuda_code(e);
+}
+
+// Repack the weights so that every 16 KiB page an instruction streams is
+// contiguous: QKV rows in rotation-pair order, gate/up rows interleaved per
+// page, down projection split into K pieces.
+int repack(mk_handle *h, const Plan &p) {
+  const Shape &s = h->shape;
+  const int H = s.H, d = s.d;
+  const size_t per_qkv = (size_t)p.P_qkv * kPageElems, per_gu = (size_t)p.P_gu * kPageElems,
+               per_dn = (size_t)p.ndp * p.P_dp * kPageElems;
+  int rc;
+  if ((rc = dalloc(h->allocs, &h->wqkv, per_qkv * s.L, false))) return rc;
+  if ((rc = dalloc(h->allocs, &h->wgu, per_gu * s.L, false))) return rc;
+  if ((rc = dalloc(h->allocs, &h->wd, per_dn * s.L, false))) return rc;
+  const int Rh = p.Rh, half = Rh / 2, pph = d / Rh;
+  std::vector<unsigned long long> src;
+  for (int l = 0; l < s.L; ++l) {
+    const mk_layer_weights &W = h->lw[l];
+    const uint16_t *wq = (const uint16_t *)W.wq, *wk = (const uint16_t *)W.wk, *wv = (const uint16_t *)W.wv;
+    src.clear();
+    for (int j = 0; j < p.P_qkv; ++j) {
+      const int head = j / pph, jj = j % pph;
+      for (int t = 0; t < Rh; ++t) {
+        const int rin = t < half ? jj * half + t : d / 2 + jj * half + (t - half);
+        const uint16_t *base;
+        int hh;
+        if (head < s.nq) {
+          base = wq;
+          hh = head;
+        } else if (head < s.nq + s.nkv) {
+          base = wk;
+          hh = head - s.nq;
+        } else {
+          base = wv;
+          hh = head - s.nq - s.nkv;
+        }
+        src.push_back((unsigned long long)(base + ((size_t)hh * d + rin) * H));
+      }
+    }
+    if ((rc = gather_rows(h->wqkv + per_qkv * l, src, H))) return rc;
+    src.clear();
+    const uint16_t *wg = (const uint16_t *)W.w_gate, *wu = (const uint16_t *)W.w_up;
+    for (int j = 0; j < p.P_gu; ++j)
+      for (int t = 0; t < Rh; ++t) {
+        const uint16_t *base = t < half ? wg : wu;
+        const int row = j * half + (t < half ? t : t - half);
+        src.push_back((unsigned long long)(base + (size_t)row * H));
+      }
+    if ((rc = gather_rows(h->wgu + per_gu * l, src, H))) return rc;
+    src.clear();
+    const uint16_t *wdn = (const uint16_t *)W.w_down;
+    for (int k = 0; k < p.ndp; ++k)
+      for (int r = 0; r < H; ++r) src.push_back((unsigned long long)(wdn + (size_t)r * s.F + (size_t)k * p.KCd));
+    if ((rc = gather_rows(h->wd + per_dn * l, src, p.KCd))) return rc;
+  }
+  std::vector<LayerDev> ld(s.L);
+  for (int l = 0; l < s.L; ++l) {
+    ld[l].wqkv = h->wqkv + per_qkv * l;
+    ld[l].wo = (const uint16_t *)h->lw[l].wo;
+    ld[l].wgu = h->wgu + per_gu * l;
+    ld[l].wd = h->wd + per_dn * l;
+    ld[l].attn_norm = (const uint16_t *)h->lw[l].attn_norm;
+    ld[l].ffn_norm = (const uint16_t *)h->lw[l].ffn_norm;
+  }
+  if ((rc = dalloc(h->allocs, &h->d_layers, s.L, false))) return rc;
+  MK_CUDA(cudaMemcpy(h->d_layers, ld.data(), sizeof(LayerDev) * s.L, cudaMemcpyHostToDevice));
+  return MK_OK;
+}
+
+// RoPE table: angle pos * theta^(-2i/d) in double, stored as float (cos, sin).
+int build_rope(mk_handle *h) {
+  const int d = h->cfg.head_dim, hd = d / 2, S = h->cfg.max_seq;
+  std::vector<float2> t((size_t)S * hd);
+  for (int i = 0; i < hd; ++i) {
+    const double w = std::pow(h->cfg.rope_theta, -2.0 * i / d);
+    for (int pos = 0; pos < S; ++pos) {
+      const double a = (double)pos * w;
+      t[(size_t)pos * hd + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+    }
+  }
+  int rc = dalloc(h->allocs, &h->d_rope, t.size(), false);
+  if (rc) return rc;
+  MK_CUDA(cudaMemcpy(h->d_rope, t.data(), t.size() * sizeof(float2), cudaMemcpyHostToDevice));
+  return MK_OK;
+}
+
+mk_plan_opts default_opts(const mk_config &c) {
+  mk_plan_opts o;
+  memset(&o, 0, sizeof o);
+  o.batch = c.max_batch;
+  return o;
+}
+
+PlanRequest make_request(const mk_config &c, const mk_plan_opts &o, int num_ctas) {
+  PlanRequest r;
+  r.s = shape_of(c);
+  r.B = o.batch;
+  r.S = o.kv_splits;
+  r.num_ctas = num_ctas;
+  r.dynamic = o.sched_mode == MK_SCHED_DYNAMIC;
+  r.assumed_context = std::max(1, c.max_seq);
+  r.drop_producer = o.debug_drop_producer != 0;
+  return r;
+}
+
+void set_err(char *err, size_t n, const std::string &m) {
+  if (err && n) {
+    snprintf(err, n, "%s", m.c_str());
+  }
+}
+
+int check_cfg(const mk_config *c, std::string *why) {
+  if (!c) return MK_ERR_INVALID_ARG;
+  if (c->max_batch < 1 || c->max_seq < 1 || c->n_layers < 1 || !(c->rms_eps >= 0.f) ||
+      !(c->rope_theta > 0.0)) {
+    *why = "non-positive capacity or parameter";
+    return MK_ERR_INVALID_ARG;
+  }
+  std::string e = check_shape(shape_of(*c), c->max_batch);
+  if (!e.empty()) {
+    *why = e;
+    return MK_ERR_UNSUPPORTED_SHAPE;
+  }
+  return MK_OK;
+}
+
+size_t act_floats_for(const mk_config &c, const Plan &p, int nb) {
+  const int G = c.n_q_heads / c.n_kv_heads;
+  size_t vec = (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim, p.KCd});
+  size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim;  // + cur K/V rows (bf16)
+  size_t f = std::max(vec, attn);
+  return (f + 31) / 32 * 32;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+
+extern "C" const char *mk_status_string(int code) {
+  switch (code) {
+    case MK_OK: return "ok";
+    case MK_ERR_INVALID_ARG: return "invalid argument";
+    case MK_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MK_ERR_NOT_PLANNED: return "mk_plan has not been called";
+    case MK_ERR_CUDA: return "CUDA runtime error";
+    case MK_ERR_LAUNCH: return "persistent launch refused (CTAs not co-resident)";
+    case MK_ERR_TIMEOUT: return "a device-side wait timed out";
+    case MK_ERR_DEVICE_INPUT: return "token id or position out of range on the device";
+    case MK_ERR_OUT_OF_MEMORY: return "device allocation failed";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv, mk_handle **out) {
+  if (out) *out = nullptr;
+  if (!cfg || !w || !kv || !out) return MK_ERR_INVALID_ARG;
+  std::string why;
+  int rc = check_cfg(cfg, &why);
+  if (rc) return rc;
+  if (!w->embed || !w->final_norm || !w->layers || (!cfg->tied_lm_head && !w->lm_head) || !kv->k || !kv->v)
+    return MK_ERR_INVALID_ARG;
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const mk_layer_weights &L = w->layers[l];
+    const void *ps[] = {L.attn_norm, L.wq, L.wk, L.wv, L.wo, L.ffn_norm, L.w_gate, L.w_up, L.w_down};
+    for (const void *p : ps)
+      if (!p || !aligned16(p)) return MK_ERR_INVALID_ARG;
+  }
+  const void *lm = cfg->tied_lm_head ? w->embed : w->lm_head;
+  if (!aligned16(w->embed) || !aligned16(lm) || !aligned16(w->final_norm) || !aligned16(kv->k) ||
+      !aligned16(kv->v))
+    return MK_ERR_INVALID_ARG;
+
+  mk_handle *h = new (std::nothrow) mk_handle();
+  if (!h) return MK_ERR_OUT_OF_MEMORY;
+  h->cfg = *cfg;
+  h->shape = shape_of(*cfg);
+  h->embed = (const uint16_t *)w->embed;
+  h->lm_head = (const uint16_t *)lm;
+  h->final_norm = (const uint16_t *)w->final_norm;
+  h->kc = (uint16_t *)kv->k;
+  h->vc = (uint16_t *)kv->v;
+  h->lw.assign(w->layers, w->layers + cfg->n_layers);
+  auto fail = [&](int code) {
+    cudaDeviceSynchronize();
+    free_list(h->allocs);
+    delete h;
+    return code;
+  };
+  cudaError_t e = cudaGetDevice(&h->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&h->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->device);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MK_ERR_CUDA);
+  }
+  // geometry (independent of batch and CTA count)
+  PlanRequest req = make_request(*cfg, default_opts(*cfg), 1);
+  req.B = 1;
+  Plan geo;
+  std::string err = build_plan(req, &geo);
+  if (!err.empty()) return fail(MK_ERR_UNSUPPORTED_SHAPE);
+  if ((rc = repack(h, geo))) return fail(rc);
+  if ((rc = build_rope(h))) return fail(rc);
+  const Shape &s = h->shape;
+  const size_t Bm = cfg->max_batch;
+  if ((rc = dalloc(h->allocs, &h->qbuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
+  if ((rc = dalloc(h->allocs, &h->obuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
+  if ((rc = dalloc(h->allocs, &h->xres, (size_t)s.L * Bm * s.H))) return fail(rc);
+  if ((rc = dalloc(h->allocs, &h->actb, (size_t)s.L * Bm * s.F))) return fail(rc);
+  if ((rc = dalloc(h->allocs, &h->dpart, (size_t)s.L * geo.ndp * Bm * s.H))) return fail(rc);
+  if ((rc = dalloc(h->allocs, &h->ctr_epoch, 4))) return fail(rc);
+  if ((rc = dalloc(h->allocs, &h->status, kStatusWords))) return fail(rc);
+  e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MK_ERR_CUDA);
+  }
+  *out = h;
+  return MK_OK;
+}
+
+static void drop_plan(mk_handle *h) {
+  if (h->gexec) {
+    cudaGraphExecDestroy(h->gexec);
+    h->gexec = nullptr;
+  }
+  free_list(h->plan_allocs);
+  h->planned = false;
+}
+
+extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  mk_plan_opts o = opts_in ? *opts_in : default_opts(h->cfg);
+  if (o.batch < 1 || o.batch > h->cfg.max_batch) return MK_ERR_INVALID_ARG;
+  if (o.sched_mode != MK_SCHED_STATIC && o.sched_mode != MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
+  if (o.exec_mode < MK_EXEC_MEGAKERNEL || o.exec_mode > MK_EXEC_PER_OP_GRAPH) return MK_ERR_INVALID_ARG;
+  if (o.exec_mode != MK_EXEC_MEGAKERNEL && o.sched_mode == MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
+  if (o.kv_splits < 0 || o.num_sms < 0 || o.wait_timeout_ns < 0) return MK_ERR_INVALID_ARG;
+  if (o.batch > 1) return MK_ERR_UNSUPPORTED_SHAPE;  // batched instructions: not in this build yet
+  cudaError_t ce = cudaDeviceSynchronize();
+  if (ce != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  drop_plan(h);
+  const int num_ctas = o.num_sms > 0 ? std::min(o.num_sms, h->sm_count) : h->sm_count;
+  PlanRequest req = make_request(h->cfg, o, num_ctas);
+  Plan p;
+  std::string err = build_plan(req, &p);
+  if (err.empty()) err = validate_plan(req, p);
+  if (!err.empty()) {
+    fprintf(stderr, "mk_plan: %s\n", err.c_str());
+    return MK_ERR_UNSUPPORTED_SHAPE;
+  }
+  const int nb = 1;
+  const size_t act_floats = act_floats_for(h->cfg, p, nb);
+  const int fixed = shared_bytes_fixed(0, act_floats);
+  int num_pages = (h->smem_optin - fixed) / (kPageBytes + 16);
+  num_pages = std::min(num_pages, 16);
+  if (num_pages < 2) return MK_ERR_UNSUPPORTED_SHAPE;
+  const int smem = shared_bytes_fixed(num_pages, act_floats);
+  int per_sm = 0;
+  cudaError_t e = occupancy_interp(nb, smem, &per_sm);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (per_sm < 1) return MK_ERR_LAUNCH;
+
+  const Shape &s = h->shape;
+  const int B = o.batch;
+  KParams &k = h->kp;
+  memset(&k, 0, sizeof k);
+  int rc;
+  float *part_o, *part_ml, *arg_val;
+  int *arg_idx, *q_off, *q_len;
+  unsigned *ctr;
+  Instr *instrs;
+  unsigned long long *trace = nullptr;
+  if ((rc = dalloc(h->plan_allocs, &part_o, (size_t)s.L * B * s.nq * p.S * s.d))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &part_ml, (size_t)s.L * B * s.nq * p.S * 2))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &arg_val, (size_t)B * p.n_lm))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &arg_idx, (size_t)B * p.n_lm))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &ctr, (size_t)p.n_counters))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &instrs, p.instrs.size(), false))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &q_off, (size_t)num_ctas, false))) return rc;
+  if ((rc = dalloc(h->plan_allocs, &q_len, (size_t)num_ctas, false))) return rc;
+  if (o.trace && (rc = dalloc(h->plan_allocs, &trace, p.instrs.size() * MK_TRACE_WORDS))) return rc;
+  e = cudaMemcpy(instrs, p.instrs.data(), p.instrs.size() * sizeof(Instr), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(q_off, p.q_off.data(), sizeof(int) * num_ctas, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(q_len, p.q_len.data(), sizeof(int) * num_ctas, cudaMemcpyHostToDevice);
+  const unsigned one = 1;
+  if (e == cudaSuccess) e = cudaMemcpy(h->ctr_epoch, &one, sizeof one, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(h->status, 0, sizeof(int) * kStatusWords);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+
+  k.L = s.L;
+  k.H = s.H;
+  k.nq = s.nq;
+  k.nkv = s.nkv;
+  k.d = s.d;
+  k.F = s.F;
+  k.V = s.V;
+  k.qdim = s.nq * s.d;
+  k.kvdim = s.nkv * s.d;
+  k.B = B;
+  k.Rh = p.Rh;
+  k.Ro = p.Ro;
+  k.Rd = p.Rd;
+  k.KCd = p.KCd;
+  k.ndp = p.ndp;
+  k.S = p.S;
+  k.max_seq = h->cfg.max_seq;
+  k.eps = h->cfg.rms_eps;
+  k.attn_scale = (float)(1.0 / std::sqrt((double)s.d));
+  k.layers = h->d_layers;
+  k.embed = h->embed;
+  k.lm_head = h->lm_head;
+  k.final_norm = h->final_norm;
+  k.kc = h->kc;
+  k.vc = h->vc;
+  k.kv_hs = (long long)h->cfg.max_seq * s.d;
+  k.kv_bs = k.kv_hs * s.nkv;
+  k.kv_ls = k.kv_bs * h->cfg.max_batch;
+  k.rope = h->d_rope;
+  k.qbuf = h->qbuf;
+  k.part_o = part_o;
+  k.part_ml = part_ml;
+  k.obuf = h->obuf;
+  k.xres = h->xres;
+  k.actb = h->actb;
+  k.dpart = h->dpart;
+  k.arg_val = arg_val;
+  k.arg_idx = arg_idx;
+  k.n_lm = p.n_lm;
+  k.ctr = ctr;
+  k.epoch = h->ctr_epoch;
+  k.status = h->status;
+  k.attn_ticket0 = p.attn_ticket0;
+  k.arg_ticket0 = p.arg_ticket0;
+  k.exit_ticket = p.exit_ticket;
+  k.dyn_head = p.dyn_head;
+  k.instrs = instrs;
+  k.q_off = q_off;
+  k.q_len = q_len;
+  k.n_instr = (int)p.instrs.size();
+  k.num_pages = num_pages;
+  k.act_floats = (long long)act_floats;
+  int pf_kb = o.l2_prefetch_kb;
+  if (pf_kb == 0) pf_kb = -1;  // automatic: off until measured otherwise
+  k.pf_pages = pf_kb > 0 ? (pf_kb * 1024) / kPageBytes : 0;
+  k.timeout_ns = o.wait_timeout_ns > 0 ? o.wait_timeout_ns : 1000000000LL;
+  k.trace = trace;
+  k.mode = (o.trace ? MODE_TRACE : 0u) | (o.sched_mode == MK_SCHED_DYNAMIC ? MODE_DYNAMIC : 0u);
+  k.stage_filter = -1;
+  h->plan = std::move(p);
+  h->opts = o;
+  h->smem = smem;
+  h->grid = num_ctas;
+  h->nb = nb;
+  h->planned = true;
+  return MK_OK;
+}
+
+static int launch_per_op(mk_handle *h, KParams k, cudaStream_t st) {
+  const int n_stage = h->shape.L * kStagesPerLayer + 1;
+  for (int sidx = 0; sidx < n_stage; ++sidx) {
+    // skip the empty per-layer stage slot of the LM head
+    k.stage_filter = sidx;
+    k.mode = (h->kp.mode & MODE_TRACE) | MODE_NO_WAIT | (sidx == n_stage - 1 ? MODE_FINAL_LAUNCH : 0u);
+    cudaError_t e = launch_interp(k, h->nb, h->grid, h->smem, st, false);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_code(e);
+    }
+  }
+  return MK_OK;
+}
+
+extern "C" int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions, float *logits_out,
+                              int32_t *next_tokens_out, void *stream) {
+  if (!h || !tokens || !positions || !next_tokens_out) return MK_ERR_INVALID_ARG;
+  if (!h->planned) return MK_ERR_NOT_PLANNED;
+  cudaStream_t st = (cudaStream_t)stream;
+  KParams k = h->kp;
+  k.tokens = tokens;
+  k.positions = positions;
+  k.logits = logits_out;
+  k.next_tokens = next_tokens_out;
+  if (h->opts.exec_mode == MK_EXEC_MEGAKERNEL) {
+    k.mode |= MODE_FINAL_LAUNCH;
+    cudaError_t e = launch_interp(k, h->nb, h->grid, h->smem, st, true);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_code(e);
+    }
+    return MK_OK;
+  }
+  if (h->opts.exec_mode == MK_EXEC_PER_OP) return launch_per_op(h, k, st);
+  // per-op launches replayed as one CUDA graph (re-captured if the I/O pointers change)
+  if (!h->gexec || h->g_tokens != tokens || h->g_pos != positions || h->g_logits != logits_out ||
+      h->g_next != next_tokens_out) {
+    if (h->gexec) {
+      cudaGraphExecDestroy(h->gexec);
+      h->gexec = nullptr;
+    }
+    cudaStream_t cap;
+    MK_CUDA(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal);
+    int rc = MK_OK;
+    if (e == cudaSuccess) {
+      rc = launch_per_op(h, k, cap);
+      e = cudaStreamEndCapture(cap, &graph);
+    }
+    if (e == cudaSuccess && rc == MK_OK) e = cudaGraphInstantiate(&h->gexec, graph, 0);
+    if (graph) cudaGraphDestroy(graph);
+    cudaStreamDestroy(cap);
+    if (rc != MK_OK) return rc;
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_code(e);
+    }
+    h->g_tokens = tokens;
+    h->g_pos = positions;
+    h->g_logits = logits_out;
+    h->g_next = next_tokens_out;
+  }
+  MK_CUDA(cudaGraphLaunch(h->gexec, st));
+  return MK_OK;
+}
+
+extern "C" int mk_get_status(mk_handle *h, void *stream) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  int st[kStatusWords];
+  e = cudaMemcpy(st, h->status, sizeof st, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (st[0] == 0) return MK_OK;
+  const int code = st[0];
+  // the step that failed left the counters inconsistent: start the step
+  // numbering again
+  e = cudaMemset(h->status, 0, sizeof(int) * kStatusWords);
+  if (e == cudaSuccess && h->planned) {
+    const unsigned one = 1;
+    e = cudaMemset(h->kp.ctr, 0, sizeof(unsigned) * h->plan.n_counters);
+    if (e == cudaSuccess) e = cudaMemcpy(h->ctr_epoch, &one, sizeof one, cudaMemcpyHostToDevice);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  return code;
+}
+
+extern "C" void mk_destroy(mk_handle *h) {
+  if (!h) return;
+  cudaDeviceSynchronize();
+  drop_plan(h);
+  free_list(h->allocs);
+  delete h;
+}
+
+extern "C" int mk_get_plan_info(const mk_handle *h, mk_plan_info *info) {
+  if (!h || !info) return MK_ERR_INVALID_ARG;
+  if (!h->planned) return MK_ERR_NOT_PLANNED;
+  info->num_ctas = h->grid;
+  info->threads_per_cta = kThreads;
+  info->smem_bytes = h->smem;
+  info->num_pages = h->kp.num_pages;
+  info->num_instructions = (int)h->plan.instrs.size();
+  info->num_counters = h->plan.n_counters;
+  info->kv_splits = h->plan.S;
+  int mx = 0;
+  for (int l : h->plan.q_len) mx = std::max(mx, l);
+  info->max_queue_len = mx;
+  info->weight_bytes_per_step = h->plan.weight_bytes;
+  return MK_OK;
+}
+
+extern "C" int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words) {
+  if (!h || !out) return MK_ERR_INVALID_ARG;
+  if (!h->planned) return MK_ERR_NOT_PLANNED;
+  if (!h->kp.trace) return MK_ERR_INVALID_ARG;
+  const size_t need = h->plan.instrs.size() * MK_TRACE_WORDS;
+  if (n_words < need) return MK_ERR_INVALID_ARG;
+  MK_CUDA(cudaDeviceSynchronize());
+  MK_CUDA(cudaMemcpy(out, h->kp.trace, need * sizeof(uint64_t), cudaMemcpyDeviceToHost));
+  return MK_OK;
+}
+
+// ====================================================================== host-only planner
+
+extern "C" int mk_host_plan(const mk_config *cfg, const mk_plan_opts *opts, int32_t num_ctas,
+                            mk_instr_desc *instrs_out, int32_t max_instrs, int32_t *n_instrs, int32_t *queue_off,
+                            int32_t *queue_len, mk_plan_info *info, char *err, size_t err_len) {
+  std::string why;
+  int rc = check_cfg(cfg, &why);
+  if (rc) {
+    set_err(err, err_len, why);
+    return rc;
+  }
+  if (num_ctas < 1) return MK_ERR_INVALID_ARG;
+  mk_plan_opts o = opts ? *opts : default_opts(*cfg);
+  if (o.batch < 1 || o.batch > cfg->max_batch) return MK_ERR_INVALID_ARG;
+  PlanRequest req = make_request(*cfg, o, num_ctas);
+  Plan p;
+  std::string e = build_plan(req, &p);
+  if (e.empty()) e = validate_plan(req, p);
+  if (!e.empty()) {
+    set_err(err, err_len, e);
+    return MK_ERR_UNSUPPORTED_SHAPE;
+  }
+  if (n_instrs) *n_instrs = (int32_t)p.instrs.size();
+  if (instrs_out) {
+    if (max_instrs < (int32_t)p.instrs.size()) return MK_ERR_INVALID_ARG;
+    memcpy(instrs_out, p.instrs.data(), p.instrs.size() * sizeof(Instr));
+  }
+  if (queue_off)
+    for (int c = 0; c < num_ctas; ++c) queue_off[c] = p.q_off[c];
+  if (queue_len)
+    for (int c = 0; c < num_ctas; ++c) queue_len[c] = p.q_len[c];
+  if (info) {
+    memset(info, 0, sizeof *info);
+    info->num_ctas = num_ctas;
+    info->threads_per_cta = kThreads;
+    info->num_instructions = (int)p.instrs.size();
+    info->num_counters = p.n_counters;
+    info->kv_splits = p.S;
+    int mx = 0;
+    for (int l : p.q_len) mx = std::max(mx, l);
+    info->max_queue_len = mx;
+    info->weight_bytes_per_step = p.weight_bytes;
+  }
+  return MK_OK;
+}
+
+extern "C" int mk_host_plan_simulate(const mk_config *cfg, const mk_plan_opts *opts, int32_t num_ctas, int32_t steps,
+                                     uint64_t seed, int32_t timeout_ms, char *err, size_t err_len) {
+  std::string why;
+  int rc = check_cfg(cfg, &why);
+  if (rc) {
+    set_err(err, err_len, why);
+    return rc;
+  }
+  if (num_ctas < 1 || steps < 1 || timeout_ms < 1) return MK_ERR_INVALID_ARG;
+  mk_plan_opts o = opts ? *opts : default_opts(*cfg);
+  if (o.batch < 1 || o.batch > cfg->max_batch) return MK_ERR_INVALID_ARG;
+  PlanRequest req = make_request(*cfg, o, num_ctas);
+  Plan p;
+  std::string e = build_plan(req, &p);
+  if (e.empty()) e = validate_plan(req, p);
+  if (e.empty()) e = simulate_plan(req, p, steps, seed, timeout_ms);
+  if (!e.empty()) {
+    set_err(err, err_len, e);
+    return MK_ERR_INVALID_ARG;
+  }
+  return MK_OK;
+}

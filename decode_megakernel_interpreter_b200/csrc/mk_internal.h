@@ -1,0 +1,133 @@
+// Internal types shared by the host planner, the C ABI and the interpreter
+// kernel.  Not part of the public ABI (include/mk.h is).
+#pragma once
+#include <stdint.h>
+#include <vector_types.h>  // float2
+
+namespace mk {
+
+// ---------------------------------------------------------------- geometry
+// Every weight byte the interpreter streams moves in 16 KiB shared-memory
+// pages (the paged shared memory of the "Hazy megakernel summary" page,
+// section 四(二), re-sized for Blackwell's 227 KB per CTA).  A matrix-vector
+// page holds R rows x KC columns of bf16 with R * KC = 8192.
+constexpr int kPageBytes = 16384;
+constexpr int kPageElems = kPageBytes / 2;
+constexpr int kComputeWarps = 8;              // warps 1..8
+constexpr int kThreads = 32 * (1 + kComputeWarps);
+constexpr int kComputeThreads = 32 * kComputeWarps;
+constexpr int kMaxKc = 4096;                  // largest K staged in one page row
+constexpr int kMaxBatch = 16;
+
+// ---------------------------------------------------------------- opcodes
+// The instruction set of the decode step (the fused instructions the
+// "Hazy megakernel summary" page lists: RMSNorm + QKV + RoPE, attention, ...).
+enum Op : uint8_t {
+  OP_NOP = 0,
+  OP_QKV = 1,    // rms(x)*g1 -> fused QKV rows -> RoPE -> q (fp32) / K,V cache (bf16)
+  OP_ATTN = 2,   // one (sequence, kv head, split) of split-KV GQA decode attention;
+                 // the last split to finish merges the splits (log-sum-exp)
+  OP_OPROJ = 3,  // x_mid = x_in + Wo * attn
+  OP_GATEUP = 4, // rms(x_mid)*g2 -> gate/up rows -> silu(gate)*up
+  OP_DOWN = 5,   // partial_k = Wd[:, K-piece k] * act[K-piece k]
+  OP_LMHEAD = 6, // rms(x_out)*gf -> logits rows -> per-instruction argmax; last merges
+};
+
+// Instruction classes double as the "stage" used by the per-op comparison path
+// (one launch per stage per layer).
+enum Stage : uint8_t { ST_QKV = 0, ST_ATTN = 1, ST_OPROJ = 2, ST_GATEUP = 3, ST_DOWN = 4, ST_LMHEAD = 5 };
+constexpr int kStagesPerLayer = 5;
+
+constexpr uint32_t kNoCounter = 0xFFFFFFFFu;
+
+// One interpreter instruction (32 bytes).
+struct Instr {
+  uint8_t op;
+  uint8_t pad0;
+  uint16_t layer;
+  uint32_t a;        // matvec: first page | attn: kv head g | lmhead: first page
+  uint32_t b;        // matvec: page count | attn: split index s
+  uint32_t c;        // down: K piece | attn: sequence | lmhead: argmax slot
+  uint32_t wait_ctr; // counter to wait on (kNoCounter: none)
+  uint32_t wait_cnt; // producers per step: wait until ctr >= epoch * wait_cnt
+  uint32_t sig_ctr;  // first counter to signal (kNoCounter: none)
+  uint16_t sig_n;    // number of consecutive counters to signal
+  uint16_t seq;      // global position of the instruction in the topological order
+};
+static_assert(sizeof(Instr) == 32, "Instr must be 32 bytes");
+
+// Per-layer weight pointers the kernel reads.
+struct LayerDev {
+  const uint16_t *wqkv;     // packed [(nq+2nkv)*d / R pages][R][H]
+  const uint16_t *wo;       // caller's [H][q_dim]
+  const uint16_t *wgu;      // packed [F/(R/2) pages][R][H] (R/2 gate rows, R/2 up rows)
+  const uint16_t *wd;       // packed [F/KCd pieces][H/Rd pages][Rd][KCd]
+  const uint16_t *attn_norm;
+  const uint16_t *ffn_norm;
+};
+
+// Mode bits.
+enum : uint32_t {
+  MODE_NO_WAIT = 1u,      // per-op path: kernel boundaries order the stages
+  MODE_TRACE = 2u,
+  MODE_DYNAMIC = 4u,      // one global queue claimed with an atomic
+  MODE_FINAL_LAUNCH = 8u, // this launch ends the step (advances the epoch)
+};
+
+// Status words (device): [0] first error code, [1] abort flag, [2..7] detail.
+constexpr int kStatusWords = 8;
+
+struct KParams {
+  // shape
+  int L, H, nq, nkv, d, F, V, qdim, kvdim, B;
+  int Rh;       // rows per page of the H-input matrices (QKV, gate/up, LM head) = 8192 / H
+  int Ro;       // rows per page of O projection = 8192 / q_dim
+  int Rd, KCd;  // rows per page / K piece width of the down projection
+  int ndp;      // number of down K pieces = F / KCd
+  int S;        // kv splits
+  int max_seq;
+  float eps, attn_scale;
+  // weights
+  const LayerDev *layers;
+  const uint16_t *embed, *lm_head, *final_norm;
+  // kv cache
+  uint16_t *kc, *vc;
+  long long kv_ls, kv_bs, kv_hs;   // element strides: layer, batch, head (position stride = d)
+  const float2 *rope;              // [max_seq][d/2] (cos, sin)
+  // activations (fp32)
+  float *qbuf;     // [L][B][q_dim]
+  float *part_o;   // [L][B][nq][S][d]
+  float *part_ml;  // [L][B][nq][S][2]
+  float *obuf;     // [L][B][q_dim]
+  float *xres;     // [L][B][H]
+  float *actb;     // [L][B][F]
+  float *dpart;    // [L][ndp][B][H]
+  float *arg_val;  // [B][n_lm]
+  int *arg_idx;    // [B][n_lm]
+  int n_lm;        // LM-head instructions (argmax slots) per step
+  // sync
+  unsigned *ctr;      // counters + tickets
+  unsigned *epoch;    // current step number (>= 1), advanced by the last CTA
+  int *status;        // kStatusWords
+  unsigned attn_ticket0;  // index of the first attention merge ticket [L][B][nkv]
+  unsigned arg_ticket0;   // index of the first argmax ticket [B]
+  unsigned exit_ticket;   // index of the exit ticket
+  unsigned dyn_head;      // index of the dynamic-queue head counter
+  // plan
+  const Instr *instrs;    // all instructions; static: per-CTA contiguous queues
+  const int *q_off, *q_len;
+  int n_instr;
+  int num_pages;          // ring pages per CTA
+  long long act_floats;   // floats of the staging region (input vectors, attention scratch)
+  int pf_pages;           // L2 prefetch distance in pages (0 = off)
+  long long timeout_ns;
+  unsigned long long *trace;  // [n_instr][5]
+  uint32_t mode;
+  int stage_filter;       // per-op path: run only this (layer*5 + stage), -1 = all
+  // io
+  const int *tokens, *positions;
+  float *logits;
+  int *next_tokens;
+};
+
+}  // namespace mk

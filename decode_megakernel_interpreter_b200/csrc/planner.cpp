@@ -1,0 +1,607 @@
+// Host planner for the decode interpreter.
+//
+// The schedule is built on the host ahead of time and reused for every step
+// ("Hazy megakernel summary" page, section 四(二): each SM's instruction
+// sequence is laid out in Python ahead of time and one schedule serves
+// hundreds of forward passes).  Two placements are offered, after the
+// "MegaKernel 日志" page's section on static and dynamic scheduling: static
+// per-CTA queues (default), or one global queue in topological order that the
+// CTAs claim with an atomic.  Work of a stage is split by bytes into at most
+// one chunk per CTA and placed largest-first on the least-loaded CTA (a
+// load-balancing refinement of the round-robin placement the "Mirage
+// Persistent Kernel" article describes as its current policy).
+#include "planner.h"
+
+#include <algorithm>
+#include <atomic>
+#include <chrono>
+#include <cstdio>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <numeric>
+#include <random>
+#include <thread>
+
+namespace mk {
+
+static bool pow2_in(int x, int lo, int hi) {
+  return x >= lo && x <= hi && (x & (x - 1)) == 0;
+}
+
+static int down_kc(int F) { return F <= 2048 ? F : 2048; }
+
+std::string check_shape(const Shape &s, int B) {
+  char buf[256];
+  if (s.L < 1 || s.H < 1 || s.nq < 1 || s.nkv < 1 || s.d < 1 || s.F < 1 || s.V < 1)
+    return "non-positive dimension";
+  if (s.d != 64 && s.d != 128) return "head_dim must be 64 or 128";
+  if (!pow2_in(s.H, 256, 4096)) return "hidden must be a power of two in [256, 4096]";
+  if (!pow2_in(s.nq * s.d, 256, 4096)) return "n_q_heads*head_dim must be a power of two in [256, 4096]";
+  if (s.nq % s.nkv) return "n_q_heads must be a multiple of n_kv_heads";
+  if (s.nq / s.nkv > 8) return "more than 8 query heads per KV head";
+  int Rh = kPageElems / s.H;
+  if (s.d % Rh) return "head_dim must be a multiple of the rows per page";
+  int kc = down_kc(s.F);
+  if (s.F % 256 || (s.F > 2048 && s.F % 2048) || kPageElems % kc) {
+    snprintf(buf, sizeof buf, "ffn=%d must be a multiple of 256 (and of 2048 above 2048)", s.F);
+    return buf;
+  }
+  if (s.F % (Rh / 2)) return "ffn must be a multiple of half the rows per page";
+  if (B < 1 || B > kMaxBatch) return "batch must be in [1, 16]";
+  return "";
+}
+
+namespace {
+
+struct Chunk {
+  int first, count;
+};
+
+std::vector<Chunk> split_even(int n, int parts) {
+  std::vector<Chunk> v;
+  if (n <= 0) return v;
+  parts = std::max(1, std::min(parts, n));
+  int base = n / parts, rem = n % parts, at = 0;
+  for (int i = 0; i < parts; ++i) {
+    int c = base + (i < rem ? 1 : 0);
+    v.push_back({at, c});
+    at += c;
+  }
+  return v;
+}
+
+struct Pending {
+  Instr ins;
+  int64_t bytes;
+  int stage_key;  // layer * 8 + stage (global order key)
+  int order;      // order inside the stage
+};
+
+}  // namespace
+
+std::string build_plan(const PlanRequest &req, Plan *out) {
+  const Shape &s = req.s;
+  std::string err = check_shape(s, req.B);
+  if (!err.empty()) return err;
+  if (req.num_ctas < 1) return "num_ctas must be >= 1";
+  Plan p;
+  p.num_ctas = req.num_ctas;
+  p.dynamic = req.dynamic;
+  p.Rh = kPageElems / s.H;
+  p.Ro = kPageElems / (s.nq * s.d);
+  p.KCd = down_kc(s.F);
+  p.Rd = kPageElems / p.KCd;
+  p.ndp = s.F / p.KCd;
+  const int G = s.nq / s.nkv;
+  if (req.S > 0) {
+    p.S = std::min(req.S, 256);
+  } else {
+    // one attention item per CTA, but keep at least ~32 positions per split
+    int items = req.B * s.nkv;
+    int S = std::max(1, req.num_ctas / items);
+    S = std::min(S, std::max(1, req.assumed_context / 32));
+    p.S = std::min(S, 64);
+  }
+  p.P_qkv = (s.nq + 2 * s.nkv) * s.d / p.Rh;
+  p.P_o = s.H / p.Ro;
+  p.P_gu = s.F / (p.Rh / 2);
+  p.P_dp = s.H / p.Rd;
+  p.P_lm = (s.V + p.Rh - 1) / p.Rh;
+  p.ctr_per_layer = 4 + p.ndp;
+  unsigned next = (unsigned)(s.L * p.ctr_per_layer);
+  p.attn_ticket0 = next;
+  next += (unsigned)(s.L * req.B * s.nkv);
+  p.arg_ticket0 = next;
+  next += (unsigned)req.B;
+  p.exit_ticket = next++;
+  p.dyn_head = next++;
+  p.n_counters = (int)next;
+
+  const int n = req.num_ctas;
+  const int parts = req.dynamic ? n * std::max(1, req.dyn_chunks_per_cta) : n;
+  std::vector<Pending> all;
+  auto mk_instr = [](Op op, int layer) {
+    Instr I;
+    memset(&I, 0, sizeof I);
+    I.op = op;
+    I.layer = (uint16_t)layer;
+    I.wait_ctr = kNoCounter;
+    I.sig_ctr = kNoCounter;
+    return I;
+  };
+  std::vector<int> n_down(s.L, 0), n_qkv(s.L, 0), n_o(s.L, 0);
+  for (int l = 0; l < s.L; ++l) {
+    // fused RMSNorm + QKV + RoPE
+    auto cq = split_even(p.P_qkv, parts);
+    n_qkv[l] = (int)cq.size();
+    for (size_t i = 0; i < cq.size(); ++i) {
+      Instr I = mk_instr(OP_QKV, l);
+      I.a = cq[i].first;
+      I.b = cq[i].count;
+      if (l > 0) {
+        I.wait_ctr = p.ctr_dn(l - 1);
+        I.wait_cnt = n_down[l - 1];
+      }
+      I.sig_ctr = p.ctr_qkv(l);
+      I.sig_n = 1;
+      all.push_back({I, (int64_t)cq[i].count * kPageBytes, l * 8 + ST_QKV, (int)i});
+    }
+    // split-KV attention
+    int ord = 0;
+    for (int b = 0; b < req.B; ++b)
+      for (int g = 0; g < s.nkv; ++g)
+        for (int sp = 0; sp < p.S; ++sp) {
+          Instr I = mk_instr(OP_ATTN, l);
+          I.a = g;
+          I.b = sp;
+          I.c = b;
+          I.wait_ctr = p.ctr_qkv(l);
+          I.wait_cnt = n_qkv[l];
+          I.sig_ctr = p.ctr_attn(l);  // signalled by the split that merges
+          I.sig_n = 1;
+          int64_t bytes = (int64_t)req.assumed_context / p.S * s.d * 4 + 4096;
+          all.push_back({I, bytes, l * 8 + ST_ATTN, ord++});
+        }
+    // O projection + residual
+    auto co = split_even(p.P_o, parts);
+    n_o[l] = (int)co.size();
+    for (size_t i = 0; i < co.size(); ++i) {
+      Instr I = mk_instr(OP_OPROJ, l);
+      I.a = co[i].first;
+      I.b = co[i].count;
+      I.wait_ctr = p.ctr_attn(l);
+      I.wait_cnt = req.B * s.nkv;
+      I.sig_ctr = p.ctr_o(l);
+      I.sig_n = 1;
+      all.push_back({I, (int64_t)co[i].count * kPageBytes, l * 8 + ST_OPROJ, (int)i});
+    }
+    // RMSNorm + gate/up + SiLU; signals the down-projection K pieces it feeds
+    auto cg = split_even(p.P_gu, parts);
+    std::vector<int> gu_per_piece(p.ndp, 0);
+    const int half = p.Rh / 2;
+    for (size_t i = 0; i < cg.size(); ++i) {
+      Instr I = mk_instr(OP_GATEUP, l);
+      I.a = cg[i].first;
+      I.b = cg[i].count;
+      I.wait_ctr = p.ctr_o(l);
+      I.wait_cnt = n_o[l];
+      int row0 = cg[i].first * half, row1 = (cg[i].first + cg[i].count) * half;  // act rows
+      int k0 = row0 / p.KCd, k1 = (row1 - 1) / p.KCd;
+      I.sig_ctr = p.ctr_gu(l, k0);
+      I.sig_n = (uint16_t)(k1 - k0 + 1);
+      for (int k = k0; k <= k1; ++k) gu_per_piece[k]++;
+      all.push_back({I, (int64_t)cg[i].count * kPageBytes, l * 8 + ST_GATEUP, (int)i});
+    }
+    // down projection, K-split into pieces; each piece waits only for the
+    // gate/up instructions that produce its K range
+    int total = p.ndp * p.P_dp;
+    int ord2 = 0;
+    for (int k = 0; k < p.ndp; ++k) {
+      int ck = (int)((int64_t)parts * (k + 1) / p.ndp - (int64_t)parts * k / p.ndp);
+      auto cd = split_even(p.P_dp, std::max(1, ck));
+      for (auto &c : cd) {
+        Instr I = mk_instr(OP_DOWN, l);
+        I.a = c.first;
+        I.b = c.count;
+        I.c = k;
+        I.wait_ctr = p.ctr_gu(l, k);
+        I.wait_cnt = gu_per_piece[k];
+        I.sig_ctr = p.ctr_dn(l);
+        I.sig_n = 1;
+        n_down[l]++;
+        all.push_back({I, (int64_t)c.count * kPageBytes, l * 8 + ST_DOWN, ord2++});
+      }
+    }
+    (void)total;
+  }
+  // final RMSNorm + LM head + argmax
+  auto cl = split_even(p.P_lm, parts);
+  p.n_lm = (int)cl.size();
+  for (size_t i = 0; i < cl.size(); ++i) {
+    Instr I = mk_instr(OP_LMHEAD, s.L);
+    I.a = cl[i].first;
+    I.b = cl[i].count;
+    I.c = (uint32_t)i;
+    I.wait_ctr = p.ctr_dn(s.L - 1);
+    I.wait_cnt = n_down[s.L - 1];
+    all.push_back({I, (int64_t)cl[i].count * kPageBytes, s.L * 8 + ST_QKV + 0, (int)i});
+  }
+  // the LM head sorts after every layer
+  for (auto &x : all)
+    if (x.ins.op == OP_LMHEAD) x.stage_key = s.L * 8;
+
+  std::stable_sort(all.begin(), all.end(), [](const Pending &a, const Pending &b) {
+    if (a.stage_key != b.stage_key) return a.stage_key < b.stage_key;
+    return a.order < b.order;
+  });
+  if (all.size() > 65535) return "too many instructions for one step";
+  for (size_t i = 0; i < all.size(); ++i) all[i].ins.seq = (uint16_t)i;
+  for (auto &x : all) {
+    if (x.ins.op >= OP_QKV && x.ins.op <= OP_LMHEAD && x.ins.op != OP_ATTN)
+      p.weight_bytes += (int64_t)x.ins.b * kPageBytes;
+  }
+  // the last LM page may be partial
+  {
+    int64_t full = (int64_t)p.P_lm * kPageBytes, real = (int64_t)s.V * s.H * 2;
+    p.weight_bytes -= full - real;
+  }
+
+  if (req.drop_producer) {
+    // test hook: remove the first QKV instruction of layer 0 but keep the
+    // counter targets, so attention in layer 0 can never start
+    for (size_t i = 0; i < all.size(); ++i)
+      if (all[i].ins.op == OP_QKV && all[i].ins.layer == 0) {
+        all[i].ins.op = OP_NOP;
+        all[i].ins.sig_ctr = kNoCounter;
+        all[i].ins.sig_n = 0;
+        all[i].ins.wait_ctr = kNoCounter;
+        break;
+      }
+  }
+
+  if (req.dynamic) {
+    for (auto &x : all) p.instrs.push_back(x.ins);
+    p.q_off.assign(n, 0);
+    p.q_len.assign(n, 0);
+  } else {
+    std::vector<std::vector<Instr>> q(n);
+    std::vector<int64_t> load(n, 0);
+    std::vector<int> idx(n);
+    size_t i = 0;
+    while (i < all.size()) {
+      size_t j = i;
+      while (j < all.size() && all[j].stage_key == all[i].stage_key) ++j;
+      // this stage: largest chunk onto the least-loaded CTA, one chunk per CTA per round
+      std::vector<size_t> items(j - i);
+      std::iota(items.begin(), items.end(), i);
+      std::stable_sort(items.begin(), items.end(),
+                       [&](size_t a, size_t b) { return all[a].bytes > all[b].bytes; });
+      size_t at = 0;
+      while (at < items.size()) {
+        std::iota(idx.begin(), idx.end(), 0);
+        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return load[a] < load[b]; });
+        for (int c = 0; c < n && at < items.size(); ++c, ++at) {
+          const Pending &pp = all[items[at]];
+          q[idx[c]].push_back(pp.ins);
+          load[idx[c]] += pp.bytes;
+        }
+      }
+      i = j;
+    }
+    for (int c = 0; c < n; ++c) {
+      std::sort(q[c].begin(), q[c].end(), [](const Instr &a, const Instr &b) { return a.seq < b.seq; });
+      p.q_off.push_back((int)p.instrs.size());
+      p.q_len.push_back((int)q[c].size());
+      for (auto &I : q[c]) p.instrs.push_back(I);
+    }
+  }
+  *out = std::move(p);
+  return "";
+}
+
+// ------------------------------------------------------------------ validation
+
+namespace {
+
+// Element sets read and written by one instruction, as (buffer id, begin,
+// end) ranges over flattened per-step buffers.
+enum Buf { B_QKV, B_PART, B_O, B_XRES, B_ACT, B_DPART, B_ARG, B_NBUF };
+
+struct Range {
+  int buf;
+  int64_t lo, hi;
+};
+
+struct Layout {
+  int64_t base[B_NBUF];
+  int64_t size[B_NBUF];
+};
+
+Layout make_layout(const PlanRequest &req, const Plan &p) {
+  const Shape &s = req.s;
+  Layout L;
+  L.size[B_QKV] = (int64_t)s.L * p.P_qkv;
+  L.size[B_PART] = (int64_t)s.L * req.B * s.nkv * p.S;
+  L.size[B_O] = (int64_t)s.L * req.B * s.nkv;
+  L.size[B_XRES] = (int64_t)s.L * s.H;
+  L.size[B_ACT] = (int64_t)s.L * s.F;
+  L.size[B_DPART] = (int64_t)s.L * p.ndp * s.H;
+  L.size[B_ARG] = p.n_lm;
+  int64_t at = 0;
+  for (int b = 0; b < B_NBUF; ++b) {
+    L.base[b] = at;
+    at += L.size[b];
+  }
+  return L;
+}
+
+void layer_input_reads(const PlanRequest &req, const Plan &p, int l, int64_t r0, int64_t r1,
+                       std::vector<Range> &rd) {
+  if (l <= 0) return;  // embedding rows
+  const Shape &s = req.s;
+  rd.push_back({B_XRES, (int64_t)(l - 1) * s.H + r0, (int64_t)(l - 1) * s.H + r1});
+  for (int k = 0; k < p.ndp; ++k)
+    rd.push_back({B_DPART, ((int64_t)(l - 1) * p.ndp + k) * s.H + r0,
+                  ((int64_t)(l - 1) * p.ndp + k) * s.H + r1});
+}
+
+// reads before the instruction's own work, the writes, and (attention/LM)
+// the reads of the merging instance
+void rw_sets(const PlanRequest &req, const Plan &p, const Instr &I, std::vector<Range> &rd,
+             std::vector<Range> &wr, std::vector<Range> &merge_rd, std::vector<Range> &merge_wr) {
+  const Shape &s = req.s;
+  const int G = s.nq / s.nkv;
+  const int l = I.layer;
+  switch (I.op) {
+    case OP_QKV:
+      layer_input_reads(req, p, l, 0, s.H, rd);
+      wr.push_back({B_QKV, (int64_t)l * p.P_qkv + I.a, (int64_t)l * p.P_qkv + I.a + I.b});
+      break;
+    case OP_ATTN: {
+      const int pph = s.d / p.Rh;  // pages per head
+      int g = I.a;
+      int64_t q0 = (int64_t)l * p.P_qkv;
+      rd.push_back({B_QKV, q0 + (int64_t)g * G * pph, q0 + (int64_t)(g + 1) * G * pph});
+      rd.push_back({B_QKV, q0 + (int64_t)(s.nq + g) * pph, q0 + (int64_t)(s.nq + g + 1) * pph});
+      rd.push_back({B_QKV, q0 + (int64_t)(s.nq + s.nkv + g) * pph,
+                    q0 + (int64_t)(s.nq + s.nkv + g + 1) * pph});
+      int64_t part0 = (((int64_t)l * req.B + I.c) * s.nkv + g) * p.S;
+      wr.push_back({B_PART, part0 + I.b, part0 + I.b + 1});
+      merge_rd.push_back({B_PART, part0, part0 + p.S});
+      int64_t o = ((int64_t)l * req.B + I.c) * s.nkv + g;
+      merge_wr.push_back({B_O, o, o + 1});
+      break;
+    }
+    case OP_OPROJ: {
+      rd.push_back({B_O, (int64_t)l * req.B * s.nkv, (int64_t)(l + 1) * req.B * s.nkv});
+      int64_t r0 = (int64_t)I.a * p.Ro, r1 = (int64_t)(I.a + I.b) * p.Ro;
+      layer_input_reads(req, p, l, r0, r1, rd);
+      wr.push_back({B_XRES, (int64_t)l * s.H + r0, (int64_t)l * s.H + r1});
+      break;
+    }
+    case OP_GATEUP: {
+      rd.push_back({B_XRES, (int64_t)l * s.H, (int64_t)(l + 1) * s.H});
+      int half = p.Rh / 2;
+      wr.push_back({B_ACT, (int64_t)l * s.F + (int64_t)I.a * half,
+                    (int64_t)l * s.F + (int64_t)(I.a + I.b) * half});
+      break;
+    }
+    case OP_DOWN: {
+      rd.push_back({B_ACT, (int64_t)l * s.F + (int64_t)I.c * p.KCd,
+                    (int64_t)l * s.F + (int64_t)(I.c + 1) * p.KCd});
+      int64_t base = ((int64_t)l * p.ndp + I.c) * s.H;
+      wr.push_back({B_DPART, base + (int64_t)I.a * p.Rd, base + (int64_t)(I.a + I.b) * p.Rd});
+      break;
+    }
+    case OP_LMHEAD:
+      layer_input_reads(req, p, s.L, 0, s.H, rd);
+      wr.push_back({B_ARG, I.c, I.c + 1});
+      merge_rd.push_back({B_ARG, 0, p.n_lm});
+      break;
+    default:
+      break;
+  }
+}
+
+std::vector<const Instr *> global_order(const Plan &p) {
+  std::vector<const Instr *> v;
+  for (auto &I : p.instrs) v.push_back(&I);
+  std::sort(v.begin(), v.end(), [](const Instr *a, const Instr *b) { return a->seq < b->seq; });
+  return v;
+}
+
+}  // namespace
+
+std::string validate_plan(const PlanRequest &req, const Plan &p) {
+  char buf[512];
+  const Shape &s = req.s;
+  auto order = global_order(p);
+  for (size_t i = 0; i < order.size(); ++i)
+    if (order[i]->seq != i) return "instruction sequence numbers are not 0..n-1";
+  // queues follow the global order
+  if (!p.dynamic) {
+    if ((int)p.q_off.size() != p.num_ctas) return "queue table size";
+    size_t total = 0;
+    for (int c = 0; c < p.num_ctas; ++c) {
+      for (int i = 1; i < p.q_len[c]; ++i)
+        if (p.instrs[p.q_off[c] + i].seq <= p.instrs[p.q_off[c] + i - 1].seq) {
+          snprintf(buf, sizeof buf, "queue of CTA %d is not a subsequence of the global order", c);
+          return buf;
+        }
+      total += p.q_len[c];
+    }
+    if (total != p.instrs.size()) return "queues do not cover every instruction exactly once";
+  }
+  // producers of every counter
+  std::vector<int> n_prod(p.n_counters, 0), last_prod(p.n_counters, -1);
+  for (auto *I : order) {
+    if (I->sig_ctr == kNoCounter) continue;
+    for (int k = 0; k < I->sig_n; ++k) {
+      unsigned c = I->sig_ctr + k;
+      if (c >= (unsigned)p.n_counters) return "signal counter out of range";
+      if (I->op == OP_ATTN) {
+        // one signal per (sequence, kv head): counted once, by split 0's slot
+        if (I->b == 0) n_prod[c]++;
+      } else {
+        n_prod[c]++;
+      }
+      last_prod[c] = std::max(last_prod[c], (int)I->seq);
+    }
+  }
+  for (auto *I : order) {
+    if (I->wait_ctr == kNoCounter) continue;
+    unsigned c = I->wait_ctr;
+    if (c >= (unsigned)p.n_counters) return "wait counter out of range";
+    if (n_prod[c] != (int)I->wait_cnt && !req.drop_producer) {
+      snprintf(buf, sizeof buf, "instruction %d (op %d layer %d) waits for %u signals of counter %u but %d producers exist",
+               I->seq, I->op, I->layer, I->wait_cnt, c, n_prod[c]);
+      return buf;
+    }
+    if (last_prod[c] >= (int)I->seq) {
+      snprintf(buf, sizeof buf, "instruction %d waits on a producer that comes later (%d)", I->seq, last_prod[c]);
+      return buf;
+    }
+  }
+  // every element written exactly once per step; every read covered by a
+  // producer that the reader (transitively) waits for is checked by the
+  // simulation, here we check coverage
+  Layout L = make_layout(req, p);
+  std::vector<int> wcount(L.base[B_NBUF - 1] + L.size[B_NBUF - 1], 0);
+  for (auto *I : order) {
+    std::vector<Range> rd, wr, mrd, mwr;
+    rw_sets(req, p, *I, rd, wr, mrd, mwr);
+    if (I->op == OP_ATTN && I->b == 0) wr.insert(wr.end(), mwr.begin(), mwr.end());
+    for (auto &r : wr)
+      for (int64_t e = r.lo; e < r.hi; ++e) wcount[L.base[r.buf] + e]++;
+  }
+  if (!req.drop_producer)
+    for (int b = 0; b < B_NBUF; ++b)
+      for (int64_t e = 0; e < L.size[b]; ++e)
+        if (wcount[L.base[b] + e] != 1) {
+          snprintf(buf, sizeof buf, "buffer %d element %lld written %d times per step", b, (long long)e,
+                   wcount[L.base[b] + e]);
+          return buf;
+        }
+  (void)s;
+  return "";
+}
+
+// ------------------------------------------------------------------ simulation
+
+std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint64_t seed,
+                          int timeout_ms) {
+  Layout L = make_layout(req, p);
+  const int64_t n_el = L.base[B_NBUF - 1] + L.size[B_NBUF - 1];
+  std::unique_ptr<std::atomic<uint32_t>[]> stamp(new std::atomic<uint32_t>[n_el]);
+  for (int64_t i = 0; i < n_el; ++i) stamp[i].store(0);
+  std::unique_ptr<std::atomic<uint32_t>[]> ctr(new std::atomic<uint32_t>[p.n_counters]);
+  for (int i = 0; i < p.n_counters; ++i) ctr[i].store(0);
+  std::atomic<bool> failed{false};
+  std::mutex err_mu;
+  std::string err;
+  auto fail = [&](const std::string &m) {
+    std::lock_guard<std::mutex> g(err_mu);
+    if (!failed.exchange(true)) err = m;
+  };
+
+  for (uint32_t epoch = 1; epoch <= (uint32_t)steps && !failed; ++epoch) {
+    std::atomic<uint32_t> dyn_next{0};
+    auto run_cta = [&](int cta) {
+      std::mt19937_64 rng(seed * 1000003ull + cta * 7919ull + epoch);
+      std::uniform_int_distribution<int> jitter(0, 9);
+      auto pause = [&]() {
+        int j = jitter(rng);
+        if (j < 5) std::this_thread::yield();
+        else if (j == 9) std::this_thread::sleep_for(std::chrono::microseconds(50));
+      };
+      auto check_reads = [&](const std::vector<Range> &rd, const Instr &I) {
+        for (auto &r : rd)
+          for (int64_t e = r.lo; e < r.hi; ++e)
+            if (stamp[L.base[r.buf] + e].load(std::memory_order_relaxed) != epoch) {
+              char b[256];
+              snprintf(b, sizeof b, "step %u: instruction %d (op %d layer %d) read a stale element of buffer %d",
+                       epoch, I.seq, I.op, I.layer, r.buf);
+              fail(b);
+              return false;
+            }
+        return true;
+      };
+      auto do_writes = [&](const std::vector<Range> &wr, const Instr &I) {
+        for (auto &r : wr)
+          for (int64_t e = r.lo; e < r.hi; ++e) {
+            uint32_t old = stamp[L.base[r.buf] + e].exchange(epoch, std::memory_order_relaxed);
+            if (old == epoch) {
+              char b[256];
+              snprintf(b, sizeof b, "step %u: instruction %d wrote buffer %d element twice", epoch, I.seq, r.buf);
+              fail(b);
+            }
+          }
+      };
+      int qi = 0;
+      while (!failed) {
+        const Instr *I;
+        if (p.dynamic) {
+          uint32_t k = dyn_next.fetch_add(1);
+          if (k >= p.instrs.size()) break;
+          I = &p.instrs[k];
+        } else {
+          if (qi >= p.q_len[cta]) break;
+          I = &p.instrs[p.q_off[cta] + qi++];
+        }
+        if (I->op == OP_NOP) continue;
+        if (I->wait_ctr != kNoCounter) {
+          uint64_t target = (uint64_t)epoch * I->wait_cnt;
+          auto t0 = std::chrono::steady_clock::now();
+          while (ctr[I->wait_ctr].load(std::memory_order_acquire) < target) {
+            if (failed) return;
+            std::this_thread::yield();
+            if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms)) {
+              char b[256];
+              snprintf(b, sizeof b, "step %u: instruction %d (op %d layer %d) waited too long on counter %u",
+                       epoch, I->seq, I->op, I->layer, I->wait_ctr);
+              fail(b);
+              return;
+            }
+          }
+        }
+        pause();
+        std::vector<Range> rd, wr, mrd, mwr;
+        rw_sets(req, p, *I, rd, wr, mrd, mwr);
+        if (!check_reads(rd, *I)) return;
+        pause();
+        do_writes(wr, *I);
+        bool signal = true;
+        if (I->op == OP_ATTN || I->op == OP_LMHEAD) {
+          unsigned t = I->op == OP_ATTN ? p.attn_ticket0 + (I->layer * req.B + I->c) * req.s.nkv + I->a
+                                        : p.arg_ticket0;
+          uint32_t per = I->op == OP_ATTN ? (uint32_t)p.S : (uint32_t)p.n_lm;
+          uint32_t old = ctr[t].fetch_add(1, std::memory_order_acq_rel);
+          signal = false;
+          if (old == epoch * per - 1) {  // the last one merges
+            if (!check_reads(mrd, *I)) return;
+            do_writes(mwr, *I);
+            signal = I->op == OP_ATTN;
+          }
+        }
+        if (signal && I->sig_ctr != kNoCounter)
+          for (int k = 0; k < I->sig_n; ++k) ctr[I->sig_ctr + k].fetch_add(1, std::memory_order_release);
+      }
+    };
+    std::vector<std::thread> th;
+    for (int c = 0; c < p.num_ctas; ++c) th.emplace_back(run_cta, c);
+    for (auto &t : th) t.join();
+    if (failed) break;
+    for (int b = 0; b < B_NBUF; ++b)
+      for (int64_t e = 0; e < L.size[b]; ++e)
+        if (stamp[L.base[b] + e].load() != epoch) {
+          char bb[256];
+          snprintf(bb, sizeof bb, "step %u: buffer %d element %lld never written", epoch, b, (long long)e);
+          fail(bb);
+          break;
+        }
+  }
+  return failed ? err : "";
+}
+
+}  // namespace mk

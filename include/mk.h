@@ -1,0 +1,217 @@
+/*
+ * mk -- decode megakernel engine for Llama-style decoders on B200 (sm_100a).
+ *
+ * One call of mk_decode_step runs one autoregressive decode step of a batch of
+ * sequences (RMSNorm, fused QKV projection + RoPE + KV-cache append, GQA
+ * attention over the KV cache, O projection + residual, RMSNorm + gate/up +
+ * SiLU, down projection + residual, final RMSNorm + LM head + argmax) as ONE
+ * persistent kernel: every SM runs an interpreter over an instruction queue
+ * that a host planner built once (mk_plan) and that every later step reuses.
+ *
+ * Sources (web pages on decode megakernels):
+ *  - "Hazy megakernel summary" (yaoshibet.com), section 四(二): the on-GPU
+ *    interpreter, the per-SM instruction sequences scheduled ahead of time on
+ *    the host and reused across forward passes, the fused instruction set,
+ *    paged shared memory and the global counter array;
+ *  - "MegaKernel 日志" (koas-w.github.io), sections on the on-GPU interpreter
+ *    and on static (per-SM queues) versus dynamic (one global queue)
+ *    scheduling;
+ *  - "Mirage Persistent Kernel" article (m.kljzs.com), Part 2: a runtime
+ *    loop of fetch task -> run -> notify event -> repeat.
+ *
+ * Conventions for every call below:
+ *  - Pointers named *device* point to CUDA device memory of the device that
+ *    was current at mk_create; everything else is host memory.
+ *  - All tensors are row-major.  Weight matrices are [out][in] (bf16), so one
+ *    output row is contiguous.  bf16 = IEEE bfloat16 bit pattern (uint16).
+ *  - Return value: MK_OK (0) or a negative MK_ERR_* code.  No call throws.
+ *  - A handle is not thread-safe: one host thread at a time per handle.
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ errors */
+enum {
+  MK_OK = 0,
+  MK_ERR_INVALID_ARG = -1,      /* NULL/negative/inconsistent argument */
+  MK_ERR_UNSUPPORTED_SHAPE = -2,/* shape outside what the kernels implement */
+  MK_ERR_NOT_PLANNED = -3,      /* mk_decode_step before a successful mk_plan */
+  MK_ERR_CUDA = -4,             /* a CUDA runtime call failed */
+  MK_ERR_LAUNCH = -5,           /* the persistent launch was refused (co-residency) */
+  MK_ERR_TIMEOUT = -6,          /* a device-side wait gave up (reported by mk_get_status) */
+  MK_ERR_DEVICE_INPUT = -7,     /* a token id or position was out of range on the device */
+  MK_ERR_OUT_OF_MEMORY = -8     /* a device allocation failed */
+};
+
+typedef struct mk_handle mk_handle;
+
+/* ------------------------------------------------------------------ model */
+typedef struct {
+  int32_t n_layers;     /* decoder layers */
+  int32_t hidden;       /* H */
+  int32_t n_q_heads;    /* query heads */
+  int32_t n_kv_heads;   /* key/value heads; n_q_heads % n_kv_heads == 0 */
+  int32_t head_dim;     /* d */
+  int32_t ffn;          /* F, SwiGLU width */
+  int32_t vocab;        /* V */
+  float rms_eps;        /* RMSNorm epsilon */
+  double rope_theta;    /* RoPE base */
+  int32_t tied_lm_head; /* 1: lm_head == embed (the weights pointer may be either) */
+  int32_t max_batch;    /* capacity: sequences per step */
+  int32_t max_seq;      /* capacity: KV positions per sequence */
+} mk_config;
+
+typedef struct {
+  const void *attn_norm; /* device bf16 [H] */
+  const void *wq;        /* device bf16 [n_q_heads*d][H] */
+  const void *wk;        /* device bf16 [n_kv_heads*d][H] */
+  const void *wv;        /* device bf16 [n_kv_heads*d][H] */
+  const void *wo;        /* device bf16 [H][n_q_heads*d] */
+  const void *ffn_norm;  /* device bf16 [H] */
+  const void *w_gate;    /* device bf16 [F][H] */
+  const void *w_up;      /* device bf16 [F][H] */
+  const void *w_down;    /* device bf16 [H][F] */
+} mk_layer_weights;
+
+typedef struct {
+  const void *embed;      /* device bf16 [V][H] */
+  const void *lm_head;    /* device bf16 [V][H]; ignored (embed used) when tied */
+  const void *final_norm; /* device bf16 [H] */
+  const mk_layer_weights *layers; /* HOST array [n_layers]; read during mk_create only */
+} mk_weights;
+
+typedef struct {
+  void *k; /* device bf16 [n_layers][max_batch][n_kv_heads][max_seq][head_dim] */
+  void *v; /* same layout */
+} mk_kv_cache;
+
+/*
+ * mk_create: validate the shape, take the weight and KV pointers, and build the
+ * device-side state (repacked weight copies, RoPE table, activation buffers).
+ *  - Ownership: weights and the KV cache are BORROWED; they must stay valid
+ *    until mk_destroy and the library never frees them.  The library keeps its
+ *    own repacked copy of the fused QKV, gate/up and down-projection weights
+ *    (taken at mk_create: later changes to the caller's weights are not seen),
+ *    and reads embed / wo / lm_head / norm weights in place.  The KV cache is
+ *    written only at row positions[b] of sequence b by mk_decode_step.
+ *  - Shapes implemented: head_dim in {64, 128}, hidden and n_q_heads*head_dim
+ *    in {256, 512, 1024, 2048, 4096}, ffn a multiple of 256 (and of 2048 when
+ *    above 2048), vocab >= 1, max_batch in [1, 16], max_seq >= 1.  Others give
+ *    MK_ERR_UNSUPPORTED_SHAPE.
+ *  - Uses the current CUDA device.  Synchronous (returns when set-up is done).
+ *  - Errors: MK_ERR_INVALID_ARG (NULL pointer, non-positive size),
+ *    MK_ERR_UNSUPPORTED_SHAPE, MK_ERR_OUT_OF_MEMORY, MK_ERR_CUDA.
+ *    On error *out is set to NULL and nothing is leaked.
+ */
+int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv,
+              mk_handle **out);
+
+/* ------------------------------------------------------------------ plan */
+enum { MK_SCHED_STATIC = 0, MK_SCHED_DYNAMIC = 1 };
+enum { MK_EXEC_MEGAKERNEL = 0, MK_EXEC_PER_OP = 1, MK_EXEC_PER_OP_GRAPH = 2 };
+
+typedef struct {
+  int32_t batch;          /* sequences per step, 1..max_batch */
+  int32_t kv_splits;      /* split-KV factor of decode attention; 0 = automatic */
+  int32_t sched_mode;     /* MK_SCHED_STATIC (per-SM queues) or MK_SCHED_DYNAMIC
+                             (one global queue claimed with an atomic) */
+  int32_t exec_mode;      /* MK_EXEC_MEGAKERNEL, or the comparison path:
+                             one launch per instruction class (PER_OP), optionally
+                             replayed as a CUDA graph (PER_OP_GRAPH) */
+  int32_t num_sms;        /* CTAs of the persistent grid; 0 = every SM */
+  int32_t trace;          /* 1: record per-instruction timestamps (mk_trace_read) */
+  int64_t wait_timeout_ns;/* bound on every device-side wait; 0 = 1 second */
+  int32_t l2_prefetch_kb; /* per-SM L2 prefetch distance ahead of shared memory;
+                             0 = automatic, -1 = off */
+  int32_t debug_drop_producer; /* TEST HOOK: 1 drops one producer instruction so
+                             that a dependency can never be met and the bounded
+                             wait must report MK_ERR_TIMEOUT; 0 in normal use */
+} mk_plan_opts;
+
+/*
+ * mk_plan: build the instruction DAG for this batch size, partition it into
+ * per-SM queues (or one global queue), set the dependency-counter targets,
+ * check the plan (every queue follows one global topological order) and upload
+ * it.  Call once; the plan is reused by every later mk_decode_step.  Calling it
+ * again replaces the plan (and synchronises the device).  Resets the step
+ * counters, so it must not overlap a running step of this handle.
+ *  - opts may be NULL (defaults: batch = max_batch, everything else automatic).
+ *  - Errors: MK_ERR_INVALID_ARG (batch out of range, bad mode),
+ *    MK_ERR_UNSUPPORTED_SHAPE, MK_ERR_OUT_OF_MEMORY, MK_ERR_CUDA.
+ */
+int mk_plan(mk_handle *h, const mk_plan_opts *opts);
+
+/* ------------------------------------------------------------------ step */
+/*
+ * mk_decode_step: one decode step for sequences b = 0..batch-1.
+ *  - tokens          device int32 [batch]: the input token of each sequence.
+ *  - positions       device int32 [batch]: its position p_b (0 <= p_b < max_seq).
+ *                    The step writes the token's K and V at row p_b of the
+ *                    cache and attends over rows 0..p_b, so rows 0..p_b-1 must
+ *                    hold this sequence's earlier keys (post-RoPE) and values.
+ *  - logits_out      device float [batch][vocab], or NULL to skip writing logits.
+ *  - next_tokens_out device int32 [batch]: argmax of the logits (lowest index
+ *                    among equal maxima).  May alias `tokens` (feeding the next
+ *                    step without a host round trip).
+ *  - stream          cudaStream_t (as void*); NULL = legacy default stream.
+ * Asynchronous and stream-ordered: returns once the work is enqueued, with no
+ * host synchronisation.  Device-side problems (a wait timeout, a token id
+ * outside [0, vocab) or a position outside [0, max_seq) -- which are clamped)
+ * are reported by the next mk_get_status.  Errors returned here:
+ * MK_ERR_INVALID_ARG, MK_ERR_NOT_PLANNED, MK_ERR_LAUNCH, MK_ERR_CUDA.
+ */
+int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions,
+                   float *logits_out, int32_t *next_tokens_out, void *stream);
+
+/*
+ * mk_get_status: synchronise `stream` and return the first device-side error
+ * recorded since the last call (MK_ERR_TIMEOUT, MK_ERR_DEVICE_INPUT), or a CUDA
+ * error (MK_ERR_CUDA), or MK_OK.  Clears the recorded device error.
+ */
+int mk_get_status(mk_handle *h, void *stream);
+
+/* Static English text for a code (never NULL). */
+const char *mk_status_string(int code);
+
+/* Free everything the handle owns (synchronises the device first).  Borrowed
+   weights and KV are untouched.  NULL is allowed. */
+void mk_destroy(mk_handle *h);
+
+/* ------------------------------------------------------------------ introspection */
+typedef struct {
+  int32_t num_ctas;        /* persistent grid size */
+  int32_t threads_per_cta;
+  int32_t smem_bytes;      /* dynamic shared memory per CTA */
+  int32_t num_pages;       /* 16 KiB shared-memory pages per CTA */
+  int32_t num_instructions;/* per step */
+  int32_t num_counters;
+  int32_t kv_splits;
+  int32_t max_queue_len;   /* longest per-CTA queue (static mode) */
+  int64_t weight_bytes_per_step; /* weight bytes the plan streams per step */
+} mk_plan_info;
+
+/* Fill *info for the current plan.  MK_ERR_NOT_PLANNED before mk_plan. */
+int mk_get_plan_info(const mk_handle *h, mk_plan_info *info);
+
+/*
+ * mk_trace_read: copy the per-instruction timestamps of the last step into
+ * `out` (host, uint64 [num_instructions][MK_TRACE_WORDS], nanoseconds of the
+ * device global timer).  Requires a plan with trace = 1; synchronises.
+ * Word meaning: 0 = instruction fetched by the compute warps, 1 = its
+ * dependencies were met, 2 = its input vector was staged, 3 = it signalled
+ * completion; 4 = (opcode | layer << 8 | cta << 16).
+ */
+#define MK_TRACE_WORDS 5
+int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

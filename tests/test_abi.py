@@ -1,0 +1,75 @@
+"""The C-ABI library: it loads, exports every entry point the public headers
+declare, and its host-side argument checks work without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_megakernel_interpreter_b200 as mk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = set()
+    for h in ("mk.h", "mk_host.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(mk_\w+)\s*\(", src))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported():
+    lib = mk.load()
+    names = declared_functions()
+    assert {"mk_create", "mk_plan", "mk_decode_step", "mk_get_status", "mk_status_string",
+            "mk_destroy"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for code in range(-8, 1):
+        assert mk.mk_status_string(code)
+    assert mk.mk_status_string(-99) == "unknown status"
+    assert "timed out" in mk.mk_status_string(mk.MK_ERR_TIMEOUT)
+
+
+def test_null_arguments_rejected_without_gpu():
+    lib = mk.load()
+    h = ctypes.c_void_p()
+    assert lib.mk_create(None, None, None, ctypes.byref(h)) == mk.MK_ERR_INVALID_ARG
+    assert h.value is None
+    assert lib.mk_plan(None, None) == mk.MK_ERR_INVALID_ARG
+    assert lib.mk_decode_step(None, None, None, None, None, None) == mk.MK_ERR_INVALID_ARG
+    assert lib.mk_get_status(None, None) == mk.MK_ERR_INVALID_ARG
+    assert lib.mk_get_plan_info(None, None) == mk.MK_ERR_INVALID_ARG
+    assert lib.mk_trace_read(None, None, 0) == mk.MK_ERR_INVALID_ARG
+    lib.mk_destroy(None)
+
+
+def test_unsupported_shape_rejected_before_any_device_call():
+    import synth
+    lib = mk.load()
+    cfg = mk.make_config(synth.TINY, 1, 64)
+    cfg.head_dim = 96
+    w = mk.mk_weights()
+    kv = mk.mk_kv_cache()
+    h = ctypes.c_void_p()
+    # null pointers are checked after the shape, so a bad shape wins
+    assert lib.mk_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(h)) == \
+        mk.MK_ERR_UNSUPPORTED_SHAPE
+    cfg = mk.make_config(synth.TINY, 1, 64)
+    cfg.max_batch = 17
+    assert lib.mk_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(h)) == \
+        mk.MK_ERR_UNSUPPORTED_SHAPE
+    cfg = mk.make_config(synth.TINY, 1, 0)
+    assert lib.mk_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(kv), ctypes.byref(h)) == \
+        mk.MK_ERR_INVALID_ARG
+
+
+def test_struct_layouts_match_headers():
+    assert ctypes.sizeof(mk.mk_instr_desc) == 32
+    assert ctypes.sizeof(mk.mk_config) == 56
+    assert ctypes.sizeof(mk.mk_plan_opts) == 40

@@ -1,0 +1,244 @@
+"""GPU parity: the engine (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Per step: every logit within |gpu - oracle| <= 2e-2 + 1e-2 |oracle| (the
+oracle is fed the GPU's own input token, so the two never drift apart), the
+greedy id identical unless the oracle's top-2 margin is inside the tolerance,
+next_tokens_out == argmax(logits_out) exactly, and the K/V row written at the
+step's position within one bf16 ulp of the oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_megakernel_interpreter_b200 as mk
+from decode_megakernel_interpreter_b200 import harness
+import synth
+from gpu_common import HostSetup, compare_step, within_one_bf16_ulp
+
+pytestmark = pytest.mark.gpu
+
+
+def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan_kw: dict, b=0,
+               check_kv=True, engine_out=None):
+    s = hs.shape
+    dev = harness.upload_model(hs.model, s.tied)
+    kc, vc = harness.upload_kv(hs.k, hs.v)
+    eng = harness.make_engine(s, dev, kc, vc, hs.batch, hs.max_seq)
+    eng.plan(**plan_kw)
+    tokens = torch.zeros(hs.batch, dtype=torch.int32, device="cuda")
+    pos = torch.zeros(hs.batch, dtype=torch.int32, device="cuda")
+    logits = torch.empty(hs.batch, s.vocab, dtype=torch.float32, device="cuda")
+    nxt = torch.empty(hs.batch, dtype=torch.int32, device="cuda")
+    tok, p = first_token, first_pos
+    stats = {"near_ties": 0, "max_abs": 0.0, "max_rel": 0.0, "tokens": [], "logits": []}
+    try:
+        for step in range(steps):
+            tokens.fill_(tok)
+            pos.fill_(p)
+            eng.decode_step(tokens, pos, logits, nxt)
+            assert eng.status() == mk.MK_OK
+            gl = logits[b].cpu().numpy()
+            gn = int(nxt[b].item())
+            assert gn == int(np.argmax(gl)), "next token must be the first maximal logit"
+            ol = hs.orc.decode_step(hs.k, hs.v, b, tok, p)
+            ok, near, mabs, mrel = compare_step(gl, ol, gn)
+            stats["max_abs"] = max(stats["max_abs"], mabs)
+            stats["max_rel"] = max(stats["max_rel"], mrel)
+            assert ok, f"step {step}: logits off by up to {mabs}"
+            if near:
+                stats["near_ties"] += 1
+            else:
+                assert gn == int(np.argmax(ol)), f"step {step}: greedy id differs"
+            if check_kv:
+                gk = harness.kv_to_host(kc)[:, b, :, p]
+                gv = harness.kv_to_host(vc)[:, b, :, p]
+                assert within_one_bf16_ulp(gk, hs.k[:, b, :, p]), f"step {step}: K row"
+                assert within_one_bf16_ulp(gv, hs.v[:, b, :, p]), f"step {step}: V row"
+            stats["tokens"].append(gn)
+            stats["logits"].append(gl.copy())
+            tok, p = gn, p + 1
+    finally:
+        eng.close()
+    assert stats["near_ties"] <= max(1, steps // 8)
+    return stats
+
+
+# ------------------------------------------------------------------ tiny
+
+@pytest.fixture(scope="module")
+def tiny_model():
+    return synth.make_model(synth.TINY)
+
+
+def tiny_setup(model, max_seq=96):
+    w = synth.WORKLOADS["tiny"]
+    hs = HostSetup(synth.TINY, 1, max_seq, model)
+    prompt = synth.prompt_tokens(w)
+    last = hs.prefill_prompt(prompt)
+    return hs, int(np.argmax(last)), len(prompt)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),
+    dict(exec_mode="per_op"),
+    dict(exec_mode="per_op_graph"),
+    dict(sched="dynamic"),
+    dict(num_sms=3, kv_splits=7),
+    dict(num_sms=1, kv_splits=1),
+    dict(l2_prefetch_kb=256),
+], ids=["mk", "per_op", "per_op_graph", "dynamic", "3sm", "1sm", "l2pf"])
+def test_tiny_16_steps(tiny_model, kw):
+    hs, tok, pos = tiny_setup(tiny_model)
+    run_parity(hs, tok, pos, 16, kw)
+
+
+def test_schedule_independence_bitwise(tiny_model):
+    """Every row's dot product runs inside one page on one warp, so the plan's
+    placement must not change a single bit (fixed kv_splits)."""
+    outs = []
+    for kw in (dict(kv_splits=4), dict(kv_splits=4, exec_mode="per_op"), dict(kv_splits=4, sched="dynamic"),
+               dict(kv_splits=4, num_sms=5)):
+        hs, tok, pos = tiny_setup(tiny_model)
+        outs.append(run_parity(hs, tok, pos, 4, kw))
+    for o in outs[1:]:
+        assert o["tokens"] == outs[0]["tokens"]
+        for a, b in zip(o["logits"], outs[0]["logits"]):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_tiny_from_empty_cache(tiny_model):
+    """Position 0: attention over the single current key."""
+    hs = HostSetup(synth.TINY, 1, 32, tiny_model)
+    run_parity(hs, 17, 0, 8, dict(kv_splits=5))
+
+
+def test_tiny_last_position(tiny_model):
+    hs, tok, pos = tiny_setup(tiny_model, max_seq=66)
+    run_parity(hs, tok, pos, 2, dict())  # positions 64 and 65 = max_seq - 1
+
+
+def test_ragged_vocab_and_untied_head():
+    """vocab not a multiple of the rows per page: a partial last LM page."""
+    s = synth.ModelShape(2, 256, 4, 2, 64, 512, 1000, 1e-5, 1e4, False)
+    hs = HostSetup(s, 1, 48)
+    hs.fill_prefix([30])
+    run_parity(hs, 999, 30, 6, dict())
+
+
+def test_mha_and_head_dim_128():
+    s = synth.ModelShape(2, 512, 4, 4, 128, 2048, 2048, 1e-5, 5e5, True)
+    hs = HostSetup(s, 1, 200)
+    hs.fill_prefix([150])
+    run_parity(hs, 5, 150, 4, dict(kv_splits=6))
+
+
+def test_gqa_group_of_eight():
+    s = synth.ModelShape(1, 1024, 16, 2, 64, 4096, 3000, 1e-5, 1e4, True)
+    hs = HostSetup(s, 1, 300)
+    hs.fill_prefix([257])
+    run_parity(hs, 2999, 257, 3, dict())
+
+
+def test_next_tokens_may_alias_tokens(tiny_model):
+    """Feeding next_tokens_out back as tokens without a host round trip."""
+    hs, tok, pos = tiny_setup(tiny_model)
+    s = hs.shape
+    dev = harness.upload_model(hs.model, s.tied)
+    kc, vc = harness.upload_kv(hs.k, hs.v)
+    eng = harness.make_engine(s, dev, kc, vc, 1, hs.max_seq)
+    eng.plan()
+    buf = torch.tensor([tok], dtype=torch.int32, device="cuda")
+    positions = [torch.tensor([pos + i], dtype=torch.int32, device="cuda") for i in range(6)]
+    logits = torch.empty(1, s.vocab, device="cuda")
+    got = []
+    for i in range(6):
+        eng.decode_step(buf, positions[i], logits, buf)
+        got.append(buf.clone())
+    assert eng.status() == mk.MK_OK
+    eng.close()
+    want_tok = tok
+    for i in range(6):
+        ol = hs.orc.decode_step(hs.k, hs.v, 0, want_tok, pos + i)
+        want_tok = int(np.argmax(ol))
+        assert int(got[i].item()) == want_tok
+
+
+def test_bad_token_reported_and_clamped(tiny_model):
+    hs, tok, pos = tiny_setup(tiny_model)
+    s = hs.shape
+    dev = harness.upload_model(hs.model, s.tied)
+    kc, vc = harness.upload_kv(hs.k, hs.v)
+    eng = harness.make_engine(s, dev, kc, vc, 1, hs.max_seq)
+    eng.plan()
+    t = torch.tensor([s.vocab + 5], dtype=torch.int32, device="cuda")
+    p = torch.tensor([pos], dtype=torch.int32, device="cuda")
+    nxt = torch.empty(1, dtype=torch.int32, device="cuda")
+    eng.decode_step(t, p, None, nxt)
+    assert eng.status() == mk.MK_ERR_DEVICE_INPUT
+    # the engine keeps working afterwards
+    t.fill_(tok)
+    eng.decode_step(t, p, None, nxt)
+    assert eng.status() == mk.MK_OK
+    eng.close()
+
+
+def test_trace_records_every_instruction(tiny_model):
+    hs, tok, pos = tiny_setup(tiny_model)
+    s = hs.shape
+    dev = harness.upload_model(hs.model, s.tied)
+    kc, vc = harness.upload_kv(hs.k, hs.v)
+    eng = harness.make_engine(s, dev, kc, vc, 1, hs.max_seq)
+    info = eng.plan(trace=True)
+    t = torch.tensor([tok], dtype=torch.int32, device="cuda")
+    p = torch.tensor([pos], dtype=torch.int32, device="cuda")
+    nxt = torch.empty(1, dtype=torch.int32, device="cuda")
+    eng.decode_step(t, p, None, nxt)
+    assert eng.status() == mk.MK_OK
+    tr = eng.trace()
+    eng.close()
+    assert tr.shape == (info.num_instructions, mk.MK_TRACE_WORDS)
+    ops = tr[:, 4] & 0xFF
+    assert set(ops.tolist()) == {1, 2, 3, 4, 5, 6}
+    assert np.all(tr[:, 0] <= tr[:, 1]) and np.all(tr[:, 1] <= tr[:, 2]) and np.all(tr[:, 2] <= tr[:, 3])
+    assert np.all(tr[:, 3] - tr[:, 0] < 1_000_000_000)
+
+
+# ------------------------------------------------------------------ full-size shapes
+
+@pytest.fixture(scope="module")
+def llama1b_model():
+    return synth.make_model(synth.LLAMA_1B)
+
+
+def test_llama1b_1024_context(llama1b_model):
+    w = synth.WORKLOADS["llama1b"]
+    hs = HostSetup(w.shape, 1, w.context + 8, llama1b_model)
+    hs.fill_prefix(w.lengths())
+    st = run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 3, dict())
+    print("llama1b max_abs", st["max_abs"], "max_rel", st["max_rel"])
+
+
+def test_llama1b_8k_context(llama1b_model):
+    w = synth.WORKLOADS["llama1b_8k"]
+    hs = HostSetup(w.shape, 1, w.context + 4, llama1b_model)
+    hs.fill_prefix(w.lengths())
+    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 2, dict())
+
+
+def test_llama1b_per_op_matches_megakernel(llama1b_model):
+    w = synth.WORKLOADS["llama1b"]
+    outs = []
+    for kw in (dict(), dict(exec_mode="per_op")):
+        hs = HostSetup(w.shape, 1, w.context + 4, llama1b_model)
+        hs.fill_prefix(w.lengths())
+        outs.append(run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 2, kw, check_kv=False))
+    for a, b in zip(outs[0]["logits"], outs[1]["logits"]):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_llama8b_2048_context():
+    w = synth.WORKLOADS["llama8b"]
+    hs = HostSetup(w.shape, 1, w.context + 2)
+    hs.fill_prefix(w.lengths())
+    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 1, dict())

@@ -1,0 +1,150 @@
+"""The host planner (no GPU): structure of the plans it emits and a host
+simulation of the counter protocol (one CPU thread per CTA, real atomics,
+random delays, version stamps on every buffer element)."""
+import collections
+
+import pytest
+
+import decode_megakernel_interpreter_b200 as mk
+import synth
+
+OP = {v: k for k, v in mk.OP_NAMES.items()}
+NOC = 0xFFFFFFFF
+
+
+def cfg_for(name, max_batch=1, max_seq=None):
+    w = synth.WORKLOADS[name]
+    return mk.make_config(w.shape, max_batch, max_seq or (w.context + w.steps))
+
+
+def check_structure(cfg, instrs, off, ln, num_ctas, dynamic=False):
+    s = cfg
+    Rh = 8192 // s.hidden
+    Ro = 8192 // (s.n_q_heads * s.head_dim)
+    KCd = s.ffn if s.ffn <= 2048 else 2048
+    Rd = 8192 // KCd
+    ndp = s.ffn // KCd
+    P = {"qkv": (s.n_q_heads + 2 * s.n_kv_heads) * s.head_dim // Rh, "oproj": s.hidden // Ro,
+         "gateup": s.ffn // (Rh // 2), "lmhead": -(-s.vocab // Rh)}
+    by_seq = sorted(instrs, key=lambda i: i.seq)
+    assert [i.seq for i in by_seq] == list(range(len(instrs)))
+    # queues are subsequences of the global order and cover everything once
+    if not dynamic:
+        assert sum(ln) == len(instrs)
+        for c in range(num_ctas):
+            q = instrs[off[c]:off[c] + ln[c]]
+            assert all(a.seq < b.seq for a, b in zip(q, q[1:]))
+    # page coverage: every page of every stage exactly once
+    cover = collections.Counter()
+    for i in instrs:
+        name = mk.OP_NAMES[i.op]
+        if name in P or name == "down":
+            key = (name, i.layer, i.c if name == "down" else 0)
+            for pg in range(i.a, i.a + i.b):
+                cover[key + (pg,)] += 1
+    for l in range(s.n_layers):
+        for name in ("qkv", "oproj", "gateup"):
+            assert all(cover[(name, l, 0, pg)] == 1 for pg in range(P[name])), (name, l)
+        for k in range(ndp):
+            assert all(cover[("down", l, k, pg)] == 1 for pg in range(s.hidden // Rd))
+    assert all(cover[("lmhead", s.n_layers, 0, pg)] == 1 for pg in range(P["lmhead"]))
+    assert sum(cover.values()) == sum(cover[k] for k in cover)
+    # waits: count == number of producers, all producers earlier
+    prod = collections.defaultdict(list)
+    for i in instrs:
+        if i.sig_ctr != NOC:
+            for k in range(i.sig_n):
+                if i.op != OP["attn"] or i.b == 0:
+                    prod[i.sig_ctr + k].append(i.seq)
+                else:
+                    prod.setdefault(i.sig_ctr + k, prod[i.sig_ctr + k])
+    attn_last = collections.defaultdict(int)
+    for i in instrs:
+        if i.op == OP["attn"]:
+            attn_last[i.sig_ctr] = max(attn_last[i.sig_ctr], i.seq)
+    for i in instrs:
+        if i.wait_ctr == NOC:
+            continue
+        assert len(prod[i.wait_ctr]) == i.wait_cnt, (mk.OP_NAMES[i.op], i.layer)
+        assert max(prod[i.wait_ctr] + [attn_last.get(i.wait_ctr, -1)]) < i.seq
+    # dependency chain of a layer: qkv waits for the previous layer's down
+    first = {mk.OP_NAMES[i.op]: i for i in reversed(by_seq) if i.layer == 1}
+    if s.n_layers > 1:
+        assert first["qkv"].wait_ctr != NOC
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama1b", "llama1b_8k", "llama8b"])
+@pytest.mark.parametrize("num_ctas", [148, 37, 5, 1])
+def test_plan_structure(name, num_ctas):
+    cfg = cfg_for(name)
+    instrs, off, ln, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1), num_ctas)
+    check_structure(cfg, instrs, off, ln, num_ctas)
+    assert info.num_instructions == len(instrs)
+    s = synth.WORKLOADS[name].shape
+    want = 2 * (s.n_params() - s.vocab * s.hidden * (1 if s.tied else 2) - s.hidden
+                - s.n_layers * 2 * s.hidden) + 2 * s.vocab * s.hidden
+    assert info.weight_bytes_per_step == want
+
+
+@pytest.mark.parametrize("num_ctas", [148, 16])
+def test_plan_structure_dynamic(num_ctas):
+    cfg = cfg_for("llama1b")
+    instrs, off, ln, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1, sched="dynamic"), num_ctas)
+    check_structure(cfg, instrs, off, ln, num_ctas, dynamic=True)
+    assert [i.seq for i in instrs] == list(range(len(instrs)))
+
+
+def test_static_plan_balances_bytes():
+    cfg = cfg_for("llama1b")
+    instrs, off, ln, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1), 148)
+    load = []
+    for c in range(148):
+        load.append(sum(i.b for i in instrs[off[c]:off[c] + ln[c]] if i.op not in (OP["attn"], 0)))
+    assert max(load) <= min(load) * 1.03 + 8  # pages per CTA within ~3 %
+    # at most one chunk per stage per CTA
+    for c in range(148):
+        keys = [(i.op, i.layer, i.c if i.op == OP["down"] else 0) for i in instrs[off[c]:off[c] + ln[c]]
+                if i.op != OP["attn"]]
+        assert len(keys) == len(set(keys))
+
+
+def test_kv_splits_automatic_and_explicit():
+    cfg = cfg_for("llama1b")
+    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1), 148)
+    assert info.kv_splits == 148 // 8
+    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1, kv_splits=5), 148)
+    assert info.kv_splits == 5
+
+
+@pytest.mark.parametrize("sched", ["static", "dynamic"])
+@pytest.mark.parametrize("num_ctas", [8, 3, 1])
+def test_simulation_tiny(sched, num_ctas):
+    cfg = cfg_for("tiny")
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched=sched, kv_splits=3), num_ctas, steps=3,
+                                   seed=num_ctas)
+    assert err == ""
+
+
+@pytest.mark.parametrize("sched", ["static", "dynamic"])
+def test_simulation_llama1b_full_grid(sched):
+    cfg = cfg_for("llama1b")
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched=sched), 148, steps=2, seed=7,
+                                   timeout_ms=20000)
+    assert err == ""
+
+
+def test_simulation_detects_a_missing_producer():
+    """The drop-a-producer test hook makes a wait impossible: the simulation
+    must report it as a timeout instead of hanging."""
+    cfg = cfg_for("tiny")
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, debug_drop_producer=True), 4, steps=1, seed=1,
+                                   timeout_ms=300)
+    assert "waited too long" in err
+
+
+def test_plan_rejects_bad_options():
+    cfg = cfg_for("tiny")
+    with pytest.raises(mk.MkError):
+        mk.mk_host_plan(cfg, mk.plan_opts(batch=2), 8)
+    with pytest.raises(mk.MkError):
+        mk.mk_host_plan(cfg, mk.plan_opts(batch=0), 8)
