@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="add a per-instruction-class time breakdown")
     ap.add_argument("--no-logits", action="store_true", help="do not write logits_out")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: truncate the model to this many layers (not a bench number)")
     return ap.parse_args()
 
 
@@ -272,6 +274,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
         pg = dist
     w = synth.WORKLOADS[args.workload]
+    if args.layers:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}_{args.layers}layers",
+                                shape=dataclasses.replace(w.shape, n_layers=args.layers))
     s = w.shape
     B = w.batch
     K, W = args.steps, args.warmup

@@ -15,8 +15,22 @@ def bf16_ordered(bits: np.ndarray) -> np.ndarray:
     return np.where(b & 0x8000, -(b & 0x7FFF), b)
 
 
-def within_one_bf16_ulp(a: np.ndarray, b: np.ndarray) -> bool:
-    return bool(np.all(np.abs(bf16_ordered(a) - bf16_ordered(b)) <= 1))
+def kv_row_mismatch(gpu_bits: np.ndarray, ora_bits: np.ndarray, rel_floor: float = 1e-4) -> str:
+    """'' when every element of the GPU's bf16 rows is within one bf16 ulp of
+    the oracle's, or within rel_floor * max|oracle| of it: an element that
+    is small through cancellation has a bf16 ulp far below the fp32 error of
+    the value being rounded (which scales with the row's magnitude and the
+    depth of the layer), so there the two sides cannot take the same rounding
+    decision.  Else a message naming the worst element."""
+    ulps = np.abs(bf16_ordered(gpu_bits) - bf16_ordered(ora_bits))
+    g = synth.bf16_bits_to_f32(gpu_bits).astype(np.float64)
+    o = synth.bf16_bits_to_f32(ora_bits).astype(np.float64)
+    abs_floor = rel_floor * float(np.abs(o).max())
+    bad = (ulps > 1) & (np.abs(g - o) > abs_floor)
+    if not bad.any():
+        return ""
+    i = np.unravel_index(np.argmax(np.where(bad, np.abs(g - o), -1)), g.shape)
+    return f"{int(bad.sum())} elements off; worst at {i}: gpu {g[i]!r} oracle {o[i]!r} ({int(ulps[i])} ulp)"
 
 
 class HostSetup:
