@@ -113,6 +113,8 @@ def load(path: str = LIB_PATH):
     L.mk_host_plan.restype = i32
     L.mk_host_plan.argtypes = [P(mk_config), P(mk_plan_opts), i32, P(mk_instr_desc), i32, P(i32), P(i32), P(i32),
                                P(mk_plan_info), ctypes.c_char_p, sz]
+    L.mk_decode_step_noalloc.restype = i32
+    L.mk_decode_step_noalloc.argtypes = [P(mk_config), P(mk_weights), P(mk_kv_cache), vp, vp, vp, vp, vp]
     L.mk_host_plan_simulate.restype = i32
     L.mk_host_plan_simulate.argtypes = [P(mk_config), P(mk_plan_opts), i32, i32, u64, i32, ctypes.c_char_p, sz]
     _lib = L
@@ -143,6 +145,14 @@ def mk_decode_step(h: int, tokens: int, positions: int, logits_out: int | None, 
                    stream: int | None) -> int:
     """Raw pointers (ints).  Returns the status code (no exception: the step is async)."""
     return load().mk_decode_step(h, tokens, positions, logits_out, next_tokens_out, stream)
+
+
+def mk_decode_step_noalloc(cfg: mk_config, weights: mk_weights, kv: mk_kv_cache, tokens: int, positions: int,
+                           logits_out: int | None, next_tokens_out: int, stream: int | None) -> int:
+    """The allocation-free step (scratch in a fixed device array; see mk.h).
+    Raw pointers (ints); returns the status code."""
+    return load().mk_decode_step_noalloc(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(kv), tokens,
+                                         positions, logits_out, next_tokens_out, stream)
 
 
 def mk_get_status(h: int, stream: int | None) -> int:

@@ -284,6 +284,66 @@ __device__ __forceinline__ uint32_t issue_page(const KParams &p, const Instr &I,
   return bytes;
 }
 
+// Same pages as issue_page, gathered from the caller's weights in their own
+// layout (several smaller bulk copies per page instead of one): the QKV page
+// of rotation pairs is two row runs, a gate/up page is a run of gate rows and
+// a run of up rows, a down page is Rd row segments of one K piece.  The page
+// contents are identical, so the compute side is unchanged.
+__device__ __forceinline__ void issue_page_raw(const KParams &p, const Instr &I, int t, uint8_t *dst,
+                                               uint64_t *bar, uint64_t pol_w, uint64_t pol_kv, bool prefetch_only) {
+  if (I.op != OP_QKV && I.op != OP_GATEUP && I.op != OP_DOWN) {
+    if (I.op == OP_OPROJ) {
+      const uint16_t *src = p.layers_raw[I.layer].wo + (size_t)(I.a + t) * kPageElems;
+      if (prefetch_only) {
+        px::bulk_prefetch_l2(src, kPageBytes);
+        return;
+      }
+      px::mbar_expect_tx(bar, kPageBytes);
+      px::bulk_g2s(dst, src, kPageBytes, bar, pol_w);
+      return;
+    }
+    issue_page(p, I, t, dst, bar, pol_w, pol_kv, prefetch_only);  // LM head, attention: caller's layout already
+    return;
+  }
+  const LayerRaw &W = p.layers_raw[I.layer];
+  const int j = I.a + t;
+  if (!prefetch_only) px::mbar_expect_tx(bar, kPageBytes);
+  auto copy = [&](const uint16_t *src, uint32_t off, uint32_t bytes) {
+    if (prefetch_only)
+      px::bulk_prefetch_l2(src, bytes);
+    else
+      px::bulk_g2s(dst + off, src, bytes, bar, pol_w);
+  };
+  if (I.op == OP_QKV) {
+    const int half = p.Rh / 2, pph = p.d / p.Rh;
+    const int head = j / pph, jj = j % pph;
+    const uint16_t *base;
+    int hh;
+    if (head < p.nq) {
+      base = W.wq;
+      hh = head;
+    } else if (head < p.nq + p.nkv) {
+      base = W.wk;
+      hh = head - p.nq;
+    } else {
+      base = W.wv;
+      hh = head - p.nq - p.nkv;
+    }
+    const uint32_t run = (uint32_t)half * p.H * 2;
+    copy(base + ((size_t)hh * p.d + jj * half) * p.H, 0, run);
+    copy(base + ((size_t)hh * p.d + p.d / 2 + jj * half) * p.H, run, run);
+  } else if (I.op == OP_GATEUP) {
+    const int half = p.Rh / 2;
+    const uint32_t run = (uint32_t)half * p.H * 2;
+    copy(W.wg + (size_t)j * half * p.H, 0, run);
+    copy(W.wu + (size_t)j * half * p.H, run, run);
+  } else {
+    const uint32_t seg = (uint32_t)p.KCd * 2;
+    for (int r = 0; r < p.Rd; ++r)
+      copy(W.wd + (size_t)(j * p.Rd + r) * p.F + (size_t)I.c * p.KCd, r * seg, seg);
+  }
+}
+
 // Instruction iterator shared by the loader and the compute warps.  Static
 // mode: the CTA's own queue.  (The dynamic mode hands instructions from the
 // loader to the compute warps through a small shared-memory FIFO.)
@@ -293,6 +353,7 @@ struct Queue {
 };
 
 // ============================================================== loader
+template <bool RAW>
 __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_t *full, uint64_t *empty,
                            Queue q, volatile int *dyn_fifo, volatile int *dyn_tail, volatile int *dyn_head,
                            unsigned epoch) {
@@ -349,7 +410,12 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
             pf_t = 0;
             continue;
           }
-          if (pf_g >= g + (uint32_t)NP) issue_page(p, J, pf_t, nullptr, nullptr, 0, 0, true);
+          if (pf_g >= g + (uint32_t)NP) {
+            if constexpr (RAW)
+              issue_page_raw(p, J, pf_t, nullptr, nullptr, 0, 0, true);
+            else
+              issue_page(p, J, pf_t, nullptr, nullptr, 0, 0, true);
+          }
           ++pf_t;
           ++pf_g;
         }
@@ -360,7 +426,10 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
         ok = false;
         break;
       }
-      issue_page(p, I, t, pages + (size_t)slot * kPageBytes, &full[slot], pol_w, pol_kv, false);
+      if constexpr (RAW)
+        issue_page_raw(p, I, t, pages + (size_t)slot * kPageBytes, &full[slot], pol_w, pol_kv, false);
+      else
+        issue_page(p, I, t, pages + (size_t)slot * kPageBytes, &full[slot], pol_w, pol_kv, false);
     }
     if (px::ld_volatile(&sh->abort) || global_abort(p)) ok = false;
   }
@@ -1109,7 +1178,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
 }
 
 // ============================================================== kernel
-template <int NB>
+template <int NB, bool RAW = false>
 __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int NP = p.num_pages;
@@ -1141,7 +1210,7 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   q.base = p.instrs + p.q_off[blockIdx.x];
   q.len = p.q_len[blockIdx.x];
   if (warp == 0) {
-    if (lane == 0) run_loader(p, sh, pages, full, empty, q, dyn_fifo, dyn_tail, dyn_head, epoch);
+    if (lane == 0) run_loader<RAW>(p, sh, pages, full, empty, q, dyn_fifo, dyn_tail, dyn_head, epoch);
   } else {
     CCtx c{p, sh, pages, act, act_stride, full, empty, epoch, warp - 1, lane, (int)threadIdx.x - 32, 0u};
     run_compute<NB>(c, q, dyn_fifo, dyn_tail, dyn_head);
@@ -1186,6 +1255,16 @@ cudaError_t occupancy_interp(int nb, int smem, int *blocks_per_sm) {
   cudaError_t e = cudaFuncSetAttribute(interp_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks_per_sm, interp_kernel<1>, kThreads, smem);
+}
+
+// The raw-layout variant (weights read in the caller's layout), launched
+// cooperatively; used by the allocation-free entry point.
+cudaError_t launch_interp_raw(const KParams &p, int grid, int smem, cudaStream_t st) {
+  auto fn = interp_kernel<1, true>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  void *args[] = {const_cast<KParams *>(&p)};
+  return cudaLaunchCooperativeKernel((void *)fn, dim3(grid), dim3(kThreads), args, (size_t)smem, st);
 }
 
 }  // namespace mk

@@ -66,6 +66,12 @@ struct LayerDev {
   const uint16_t *ffn_norm;
 };
 
+// Per-layer pointers to the caller's weights in their own [out][in] layout
+// (used by the kernel variant that cannot keep a repacked copy).
+struct LayerRaw {
+  const uint16_t *wq, *wk, *wv, *wo, *wg, *wu, *wd;
+};
+
 // Mode bits.
 enum : uint32_t {
   MODE_NO_WAIT = 1u,      // per-op path: kernel boundaries order the stages
@@ -89,6 +95,7 @@ struct KParams {
   float eps, attn_scale;
   // weights
   const LayerDev *layers;
+  const LayerRaw *layers_raw;  // only read by the raw-layout kernel variant
   const uint16_t *embed, *lm_head, *final_norm;
   // kv cache
   uint16_t *kc, *vc;

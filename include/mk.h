@@ -211,6 +211,50 @@ int mk_get_plan_info(const mk_handle *h, mk_plan_info *info);
 #define MK_TRACE_WORDS 5
 int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
 
+/* ------------------------------------------------------------------ allocation-free step */
+/*
+ * mk_decode_step_noalloc: the same decode step as mk_decode_step, for callers
+ * that cannot allocate device memory when they run it.  (The pages have no
+ * counterpart of this call.)
+ *
+ * Who needs it: code that may not call cudaMalloc or any allocating routine at
+ * this point -- e.g. a host callback or a context where allocation calls are
+ * not allowed, a runtime whose device memory is owned and budgeted by another
+ * component, or a caller that must avoid the implicit synchronisation an
+ * allocation can cause.  mk_create is not available to them because it
+ * allocates the repacked weights, activation and counter buffers and the plan.
+ *
+ * How: no handle.  The step's scratch (plan, RoPE table, activations,
+ * attention and argmax partials, counters, status) lives in one file-scope
+ * device array of MK_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU that loads
+ * the library holds until the process exits.  The weights are read in the
+ * caller's own layout, so no repacked copy is made.  This call makes no
+ * cudaMalloc / cudaFree and uses no allocating library routine.
+ *  - cfg, w, kv: as for mk_create (host structs; device tensor pointers,
+ *    16-byte aligned).  cfg->max_batch must be 1 (the batch of this step).
+ *  - tokens, positions, logits_out (may be NULL), next_tokens_out, stream: as
+ *    for mk_decode_step.  The kernel plan is the one mk_plan builds with
+ *    default options on this device, so results are identical to mk_create +
+ *    mk_plan(NULL) + mk_decode_step.
+ *  - First call on a device (with that device current): looks up the array's
+ *    device address and uploads the plan and tables, synchronising `stream`.
+ *    Make that first call before any stream capture.  Later calls re-upload
+ *    (and synchronise) only when cfg or the weight pointers change.
+ *  - Every call shares the array and leaves its contents behind; each call
+ *    clears the counters and status it needs.  Calls that overlap on the GPU
+ *    (other streams, other threads) race on the array: serialise them.
+ *  - Errors: MK_ERR_INVALID_ARG (NULL or misaligned pointer, bad cfg),
+ *    MK_ERR_UNSUPPORTED_SHAPE (shape not implemented, batch != 1, or the
+ *    scratch this shape needs exceeds MK_NOALLOC_SCRATCH_BYTES -- roughly the
+ *    Llama-1B shape up to ~8K positions fits, the 8B shape does not),
+ *    MK_ERR_LAUNCH, MK_ERR_CUDA.  Device-side errors of the step (timeout,
+ *    clamped input) are not reported by this call.
+ */
+#define MK_NOALLOC_SCRATCH_BYTES (8u << 20)
+int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv,
+                           const int32_t *tokens, const int32_t *positions, float *logits_out,
+                           int32_t *next_tokens_out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
