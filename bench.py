@@ -44,6 +44,7 @@ def parse():
     ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--l2-prefetch-kb", type=int, default=0)
+    ap.add_argument("--inflight", type=int, default=0, help="bulk-copy pages in flight per CTA (0 = default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="add a per-instruction-class time breakdown")
@@ -240,17 +241,23 @@ def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
     torch.cuda.synchronize()
     tr = eng.trace().astype(np.int64)
     eng.plan(**eng.plan_kw)
-    ops = tr[:, 4] & 0xFF
+    ops = tr[:, 7] & 0xFF
     t_start = tr[:, 0].min()
-    total = tr[:, 3].max() - t_start
+    total = tr[:, 4].max() - t_start
     out = {"step_us_traced": total / 1e3}
+    if os.environ.get("MK_TRACE_DUMP"):
+        np.save(os.environ["MK_TRACE_DUMP"], tr)
     for op in sorted(set(ops.tolist())):
         m = ops == op
         wait = (tr[m, 1] - tr[m, 0]) / 1e3
-        body = (tr[m, 2] - tr[m, 1]) / 1e3
+        stage = (tr[m, 2] - tr[m, 1]) / 1e3
+        pages = (tr[m, 3] - tr[m, 2]) / 1e3
+        sig = (tr[m, 4] - tr[m, 3]) / 1e3
         out[mk.OP_NAMES[int(op)]] = {"count": int(m.sum()), "mean_wait_us": float(wait.mean()),
-                                     "mean_body_us": float(body.mean()),
-                                     "sum_body_us_per_cta": float(body.sum() / info.num_ctas)}
+                                     "mean_stage_us": float(stage.mean()), "mean_pages_us": float(pages.mean()),
+                                     "mean_signal_us": float(sig.mean()),
+                                     "mean_body_us": float((tr[m, 3] - tr[m, 1]).mean() / 1e3),
+                                     "consumer_page_waits": int(tr[m, 8].sum()), "loader_ring_full": int(tr[m, 9].sum())}
     return out
 
 
@@ -291,7 +298,7 @@ def main():
     del k, v
     eng = harness.make_engine(s, dev, kc, vc, B, max_seq)
     plan_kw = dict(batch=B, kv_splits=args.kv_splits, sched=args.sched, exec_mode=args.exec_mode,
-                   l2_prefetch_kb=args.l2_prefetch_kb)
+                   l2_prefetch_kb=args.l2_prefetch_kb, max_inflight_pages=args.inflight)
     eng.plan_kw = plan_kw
     info = eng.plan(**plan_kw)
     stream = torch.cuda.current_stream()

@@ -28,7 +28,7 @@ MK_ERR_OUT_OF_MEMORY = -8
 
 MK_SCHED_STATIC, MK_SCHED_DYNAMIC = 0, 1
 MK_EXEC_MEGAKERNEL, MK_EXEC_PER_OP, MK_EXEC_PER_OP_GRAPH = 0, 1, 2
-MK_TRACE_WORDS = 5
+MK_TRACE_WORDS = 10
 
 OP_NAMES = {0: "nop", 1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"}
 
@@ -64,7 +64,7 @@ class mk_plan_opts(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("kv_splits", ctypes.c_int32), ("sched_mode", ctypes.c_int32),
                 ("exec_mode", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("trace", ctypes.c_int32),
                 ("wait_timeout_ns", ctypes.c_int64), ("l2_prefetch_kb", ctypes.c_int32),
-                ("debug_drop_producer", ctypes.c_int32)]
+                ("debug_drop_producer", ctypes.c_int32), ("max_inflight_pages", ctypes.c_int32)]
 
 
 class mk_plan_info(ctypes.Structure):
@@ -106,6 +106,8 @@ def load(path: str = LIB_PATH):
     L.mk_status_string.argtypes = [i32]
     L.mk_destroy.restype = None
     L.mk_destroy.argtypes = [vp]
+    L.mk_get_error_detail.restype = i32
+    L.mk_get_error_detail.argtypes = [vp, P(i32)]
     L.mk_get_plan_info.restype = i32
     L.mk_get_plan_info.argtypes = [vp, P(mk_plan_info)]
     L.mk_trace_read.restype = i32
@@ -161,6 +163,14 @@ def mk_get_status(h: int, stream: int | None) -> int:
 
 def mk_destroy(h: int) -> None:
     load().mk_destroy(h)
+
+
+def mk_get_error_detail(h: int) -> list:
+    d = (ctypes.c_int32 * 6)()
+    rc = load().mk_get_error_detail(h, d)
+    if rc != MK_OK:
+        raise MkError(rc, "mk_get_error_detail")
+    return list(d)
 
 
 def mk_get_plan_info(h: int) -> mk_plan_info:
@@ -222,10 +232,10 @@ def make_config(shape, max_batch: int, max_seq: int) -> mk_config:
 
 def plan_opts(batch: int = 1, kv_splits: int = 0, sched: str = "static", exec_mode: str = "megakernel",
               num_sms: int = 0, trace: bool = False, wait_timeout_ns: int = 0, l2_prefetch_kb: int = 0,
-              debug_drop_producer: bool = False) -> mk_plan_opts:
+              debug_drop_producer: bool = False, max_inflight_pages: int = 0) -> mk_plan_opts:
     return mk_plan_opts(batch, kv_splits, {"static": 0, "dynamic": 1}[sched],
                         {"megakernel": 0, "per_op": 1, "per_op_graph": 2}[exec_mode], num_sms, int(trace),
-                        wait_timeout_ns, l2_prefetch_kb, int(debug_drop_producer))
+                        wait_timeout_ns, l2_prefetch_kb, int(debug_drop_producer), max_inflight_pages)
 
 
 class Engine:

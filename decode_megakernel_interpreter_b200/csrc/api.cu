@@ -49,6 +49,7 @@ struct mk_handle {
   mk_plan_opts opts;
   KParams kp;
   int smem = 0, grid = 0, nb = 1;
+  int last_detail[6] = {0, 0, 0, 0, 0, 0};
   // per-op graph mode
   cudaGraphExec_t gexec = nullptr;
   const void *g_tokens = nullptr, *g_pos = nullptr, *g_logits = nullptr, *g_next = nullptr;
@@ -253,7 +254,8 @@ int check_cfg(const mk_config *c, std::string *why) {
 
 size_t act_floats_for(const mk_config &c, const Plan &p, int nb) {
   const int G = c.n_q_heads / c.n_kv_heads;
-  size_t vec = (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim, p.KCd});
+  // input vector (+ the O projection's residual rows after it)
+  size_t vec = (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim + c.hidden, p.KCd});
   size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim;  // + cur K/V rows (bf16)
   size_t f = std::max(vec, attn);
   return (f + 31) / 32 * 32;
@@ -384,8 +386,13 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   const size_t act_floats = act_floats_for(h->cfg, p, nb);
   const int fixed = shared_bytes_fixed(0, act_floats);
   int num_pages = (h->smem_optin - fixed) / (kPageBytes + 16);
-  num_pages = std::min(num_pages, 16);
-  if (num_pages < 2) return MK_ERR_UNSUPPORTED_SHAPE;
+  // a multiple of the loader count (page g and the next user of its slot,
+  // g + num_pages, then belong to the same loader) with 2 * num_pages a
+  // multiple of the compute-warp count (page g - 2 * num_pages belongs to the
+  // same warp as page g): every mbarrier parity test is then unambiguous
+  num_pages = std::min(num_pages, 16) / kLoaders * kLoaders;
+  while (num_pages > 0 && (2 * num_pages) % kComputeWarps) num_pages -= kLoaders;
+  if (num_pages < 2 * kLoaders) return MK_ERR_UNSUPPORTED_SHAPE;
   const int smem = shared_bytes_fixed(num_pages, act_floats);
   int per_sm = 0;
   cudaError_t e = occupancy_interp(nb, smem, &per_sm);
@@ -480,6 +487,12 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   int pf_kb = o.l2_prefetch_kb;
   if (pf_kb == 0) pf_kb = -1;  // automatic: off until measured otherwise
   k.pf_pages = pf_kb > 0 ? (pf_kb * 1024) / kPageBytes : 0;
+  {
+    // rounded to a multiple of the loader count (same reason as num_pages)
+    const int want = o.max_inflight_pages > 0 ? std::min(o.max_inflight_pages, num_pages)
+                                              : (o.max_inflight_pages < 0 ? 0 : kDefaultInflight);
+    k.max_inflight = want > 0 ? std::max(kLoaders, want / kLoaders * kLoaders) : 0;
+  }
   k.timeout_ns = o.wait_timeout_ns > 0 ? o.wait_timeout_ns : 1000000000LL;
   k.trace = trace;
   k.mode = (o.trace ? MODE_TRACE : 0u) | (o.sched_mode == MK_SCHED_DYNAMIC ? MODE_DYNAMIC : 0u);
@@ -576,6 +589,7 @@ extern "C" int mk_get_status(mk_handle *h, void *stream) {
   }
   if (st[0] == 0) return MK_OK;
   const int code = st[0];
+  for (int i = 0; i < 6; ++i) h->last_detail[i] = st[i < 5 ? 2 + i : 1];
   // the step that failed left the counters inconsistent: start the step
   // numbering again
   e = cudaMemset(h->status, 0, sizeof(int) * kStatusWords);
@@ -597,6 +611,12 @@ extern "C" void mk_destroy(mk_handle *h) {
   drop_plan(h);
   free_list(h->allocs);
   delete h;
+}
+
+extern "C" int mk_get_error_detail(const mk_handle *h, int32_t detail[6]) {
+  if (!h || !detail) return MK_ERR_INVALID_ARG;
+  for (int i = 0; i < 6; ++i) detail[i] = h->last_detail[i];
+  return MK_OK;
 }
 
 extern "C" int mk_get_plan_info(const mk_handle *h, mk_plan_info *info) {

@@ -102,6 +102,8 @@ __device__ __forceinline__ unsigned atom_add_acq_rel(unsigned *p, unsigned v) {
   return old;
 }
 __device__ __forceinline__ int ld_volatile(const int *p) { return *(const volatile int *)p; }
+// release pattern: fence.acq_rel.gpu then a relaxed reduction (lighter than fence.sc)
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 // Named barrier over the 256 compute threads, returning the OR of `pred`
 // over them (a uniform decision for every compute thread).
 __device__ __forceinline__ bool cbar_or(bool pred) {
@@ -139,6 +141,9 @@ struct Shared {
   int abort;       // this CTA saw a failed wait
   int flag;        // broadcast slot
   int pad[2];
+  float2 rope[64]; // (cos, sin) of the current position (QKV instructions, batch 1)
+  int stat_cwait;  // trace mode: pages a compute warp found not yet landed (this instruction)
+  uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
   float red[kComputeWarps][kMaxBatch];
   float argv[kComputeWarps][kMaxBatch];
   int argi[kComputeWarps][kMaxBatch];
@@ -353,18 +358,63 @@ struct Queue {
 };
 
 // ============================================================== loader
+// Source of every page of one instruction: page t is one contiguous copy of
+// bytes(t) at a + t * stride (and for KV pages a second one at b, into the
+// page's second half).  Computed once per instruction.
+struct PageSrc {
+  const uint16_t *a, *b;
+  size_t stride;            // elements between consecutive pages' sources
+  uint32_t bytes, last;     // bytes per copy; of the last page's copies
+  int npg;
+};
+__device__ __forceinline__ PageSrc page_src(const KParams &p, const Instr &I) {
+  PageSrc s;
+  s.b = nullptr;
+  s.stride = kPageElems;
+  s.bytes = s.last = kPageBytes;
+  s.npg = (int)I.b;
+  switch (I.op) {
+    case OP_QKV: s.a = p.layers[I.layer].wqkv + (size_t)I.a * kPageElems; break;
+    case OP_OPROJ: s.a = p.layers[I.layer].wo + (size_t)I.a * kPageElems; break;
+    case OP_GATEUP: s.a = p.layers[I.layer].wgu + (size_t)I.a * kPageElems; break;
+    case OP_DOWN: s.a = p.layers[I.layer].wd + ((size_t)I.c * (p.H / p.Rd) + I.a) * kPageElems; break;
+    case OP_LMHEAD: {
+      s.a = p.lm_head + (size_t)I.a * p.Rh * p.H;
+      const int r_last = (int)(I.a + I.b - 1) * p.Rh;
+      s.last = (uint32_t)min(p.Rh, p.V - r_last) * p.H * 2;
+      break;
+    }
+    case OP_ATTN: {
+      const SplitRange r = split_range(p, I.c, I.b);
+      const int ppp = attn_ppp(p), n = r.pref_end - r.start;
+      s.npg = n > 0 ? (n + ppp - 1) / ppp : 0;
+      const size_t off = (size_t)I.layer * p.kv_ls + (size_t)I.c * p.kv_bs + (size_t)I.a * p.kv_hs + (size_t)r.start * p.d;
+      s.a = p.kc + off;
+      s.b = p.vc + off;
+      s.stride = (size_t)ppp * p.d;
+      s.bytes = (uint32_t)ppp * p.d * 2;
+      s.last = s.npg > 0 ? (uint32_t)(n - (s.npg - 1) * ppp) * p.d * 2 : 0;
+      break;
+    }
+    default: s.a = nullptr; s.npg = 0; break;
+  }
+  return s;
+}
+
+// One loader lane streams the pages g with g % nl == li of every instruction
+// of its CTA's queue into the ring (several loaders overlap the issue
+// latency of the bulk copies, which is long for a single thread).
 template <bool RAW>
 __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_t *full, uint64_t *empty,
                            Queue q, volatile int *dyn_fifo, volatile int *dyn_tail, volatile int *dyn_head,
-                           unsigned epoch) {
+                           unsigned epoch, int li, int nl) {
   const uint64_t pol_w = px::policy_evict_first();
   const uint64_t pol_kv = px::policy_evict_last();
-  const int NP = p.num_pages;
-  uint32_t g = 0;
-  bool ok = true;
-  // L2 prefetch cursor (instruction index, page index) running ahead of g
-  int pf_i = 0, pf_t = 0;
-  uint32_t pf_g = 0;
+  const uint32_t NP = (uint32_t)p.num_pages;
+  const uint32_t cap = (uint32_t)p.max_inflight;
+  const bool trace = (p.mode & MODE_TRACE) != 0;
+  uint32_t g = 0, last_issued = 0;
+  bool ok = true, any = false;
   const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
   const unsigned dyn_base = dyn ? (epoch - 1u) * (unsigned)(p.n_instr + gridDim.x) : 0u;
   int claimed = 0;
@@ -374,9 +424,8 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
       // claim the next instruction of the global queue; publish it to the compute warps
       unsigned k = atomicAdd(p.ctr + p.dyn_head, 1u) - dyn_base;
       int slot = claimed & 31;
-      // wait for FIFO space (bounded)
       const uint64_t t0 = px::gtimer();
-      while (claimed - *dyn_head >= 32) {
+      while (claimed - *dyn_head >= 32) {  // FIFO space (bounded)
         if (px::ld_volatile(&sh->abort) || global_abort(p) || px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
           ok = false;
           break;
@@ -393,43 +442,62 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
       I = q.base[qi];
       if (!selected(p, I)) continue;
     }
-    const int npg = pages_of(p, I);
-    for (int t = 0; t < npg; ++t, ++g) {
-      // keep the L2 prefetch cursor pf_pages ahead (static mode only)
-      if (p.pf_pages > 0 && !dyn) {
-        if (pf_g < g) {
-          pf_i = qi;
-          pf_t = t;
-          pf_g = g;
-        }
-        while (pf_g < g + (uint32_t)p.pf_pages && pf_i < q.len) {
-          const Instr &J = q.base[pf_i];
-          int nj = selected(p, J) ? pages_of(p, J) : 0;
-          if (pf_t >= nj) {
-            ++pf_i;
-            pf_t = 0;
-            continue;
-          }
-          if (pf_g >= g + (uint32_t)NP) {
-            if constexpr (RAW)
-              issue_page_raw(p, J, pf_t, nullptr, nullptr, 0, 0, true);
-            else
-              issue_page(p, J, pf_t, nullptr, nullptr, 0, 0, true);
-          }
-          ++pf_t;
-          ++pf_g;
+    unsigned long long *ltr = (trace && li == 0) ? p.trace + (size_t)I.seq * MK_TRACE_WORDS : nullptr;
+    if (ltr) ltr[5] = px::gtimer();
+    unsigned lwait = 0;
+    const PageSrc ps = page_src(p, I);
+    const uint32_t g0 = g;
+    g += (uint32_t)ps.npg;
+    // this loader's pages of the instruction
+    for (uint32_t gg = g0 + (uint32_t)((li - (int)(g0 % nl) + nl) % nl); gg < g; gg += nl) {
+      const int t = (int)(gg - g0);
+      const uint32_t slot = gg % NP;
+      const uint32_t ph = (gg / NP) & 1u;
+      if (gg >= NP) {
+        if (ltr && !px::mbar_test(&empty[slot], ph ^ 1u)) ++lwait;
+        if (!wait_bar(p, sh, &empty[slot], ph ^ 1u, 1)) {
+          ok = false;
+          break;
         }
       }
-      const int slot = g % NP;
-      const uint32_t ph = (g / NP) & 1u;
-      if (g >= (uint32_t)NP && !wait_bar(p, sh, &empty[slot], ph ^ 1u, 1)) {
-        ok = false;
-        break;
+      // keep at most `cap` pages in flight: more only queues in the memory
+      // system and delays every other access of this SM
+      if (cap > 0 && gg >= cap) {
+        const uint32_t k = gg - cap;
+        if (!wait_bar(p, sh, &full[k % NP], (k / NP) & 1u, 3)) {
+          ok = false;
+          break;
+        }
       }
-      if constexpr (RAW)
-        issue_page_raw(p, I, t, pages + (size_t)slot * kPageBytes, &full[slot], pol_w, pol_kv, false);
-      else
-        issue_page(p, I, t, pages + (size_t)slot * kPageBytes, &full[slot], pol_w, pol_kv, false);
+      uint8_t *dst = pages + (size_t)slot * kPageBytes;
+      sh->slot_last[slot] = gg + 1;
+      if constexpr (RAW) {
+        if (I.op == OP_QKV || I.op == OP_GATEUP || I.op == OP_DOWN || I.op == OP_OPROJ) {
+          issue_page_raw(p, I, t, dst, &full[slot], pol_w, pol_kv, false);
+          any = true;
+          last_issued = gg;
+          continue;
+        }
+      }
+      const uint32_t bytes = (t == ps.npg - 1) ? ps.last : ps.bytes;
+      if (ps.b) {
+        px::mbar_expect_tx(&full[slot], 2 * bytes);
+        px::bulk_g2s(dst, ps.a + (size_t)t * ps.stride, bytes, &full[slot], pol_kv);
+        px::bulk_g2s(dst + kPageBytes / 2, ps.b + (size_t)t * ps.stride, bytes, &full[slot], pol_kv);
+      } else {
+        px::mbar_expect_tx(&full[slot], bytes);
+        px::bulk_g2s(dst, ps.a + (size_t)t * ps.stride, bytes, &full[slot], pol_w);
+      }
+      any = true;
+      last_issued = gg;
+    }
+    if (ltr) {
+      ltr[6] = px::gtimer();
+      ltr[9] = lwait;
+    }
+    if (!ok) {
+      g = g0;  // not every page of this instruction was issued; drain by last_issued
+      break;
     }
     if (px::ld_volatile(&sh->abort) || global_abort(p)) ok = false;
   }
@@ -439,19 +507,8 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
     __threadfence_block();
     *dyn_tail = claimed + 1;
   }
-  // every copy issued must land before the CTA exits
-  const uint32_t issued = g;
-  for (uint32_t k = issued > (uint32_t)NP ? issued - NP : 0; k < issued; ++k) {
-    const int slot = k % NP;
-    const uint32_t ph = (k / NP) & 1u;
-    const uint64_t t0 = px::gtimer();
-    while (!px::mbar_test(&full[slot], ph)) {
-      if (px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
-        record_error(p, MK_ERR_TIMEOUT, -2, 2, (int)k, 0);
-        break;
-      }
-    }
-  }
+  (void)any;
+  (void)last_issued;
 }
 
 // ============================================================== compute
@@ -465,24 +522,57 @@ struct CCtx {
   unsigned epoch;
   int cw, lane, ctid;
   uint32_t g;     // page sequence number (same as the loader's)
+  unsigned long long *tr;  // this instruction's trace record (or null)
 };
 
+// Register-resident view of the page ring (copied out of the context once per
+// instruction so that no loop reloads it from memory after a barrier or an
+// mbarrier poll).
+struct Ring {
+  uint8_t *pages;
+  uint64_t *full, *empty;
+  Shared *sh;
+  uint32_t np;
+};
+__device__ __forceinline__ Ring ring_of(const CCtx &c) {
+  return Ring{c.pages, c.full, c.empty, c.sh, (uint32_t)c.p.num_pages};
+}
 // Wait for ring page g (every compute warp calls this for pages it reads).
-__device__ __forceinline__ bool page_ready(CCtx &c, uint32_t g) {
-  const int slot = g % c.p.num_pages;
-  const uint32_t ph = (g / c.p.num_pages) & 1u;
-  if (px::ld_volatile(&c.sh->abort)) return false;
-  if (!wait_bar(c.p, c.sh, &c.full[slot], ph, 0)) {
-    c.sh->abort = 1;
+// A parity test only tells the last two phases apart, so first make sure the
+// slot's previous page (g - np, possibly another warp's) has been released:
+// then its full barrier is in page g's phase (pending or complete) and the
+// parity test is unambiguous.  (The previous use of the empty barrier, page
+// g - 2np, belongs to this same warp because 2np is a multiple of the warp
+// count, so that test is unambiguous too.)
+__device__ __forceinline__ bool ring_wait(const KParams &p, const Ring &r, uint32_t g) {
+  const uint32_t slot = g % r.np;
+  const uint32_t ph = (g / r.np) & 1u;
+  if (g >= r.np && !px::mbar_test(&r.empty[slot], ph ^ 1u)) {
+    if (px::ld_volatile(&r.sh->abort)) return false;
+    if (!wait_bar(p, r.sh, &r.empty[slot], ph ^ 1u, 4)) {
+      r.sh->abort = 1;
+      return false;
+    }
+  }
+  if (px::mbar_test(&r.full[slot], ph)) return true;  // fast path: already landed
+  atomicAdd(&r.sh->stat_cwait, 1);
+  if (px::ld_volatile(&r.sh->abort)) return false;
+  if (!wait_bar(p, r.sh, &r.full[slot], ph, 0)) {
+    r.sh->abort = 1;
     return false;
   }
   return true;
 }
-__device__ __forceinline__ const uint8_t *page_ptr(CCtx &c, uint32_t g) {
-  return c.pages + (size_t)(g % c.p.num_pages) * kPageBytes;
+__device__ __forceinline__ const uint8_t *ring_page(const Ring &r, uint32_t g) {
+  return r.pages + (size_t)(g % r.np) * kPageBytes;
 }
+__device__ __forceinline__ void ring_release(const Ring &r, uint32_t g, uint32_t count) {
+  px::mbar_arrive(&r.empty[g % r.np], count);
+}
+__device__ __forceinline__ bool page_ready(CCtx &c, uint32_t g) { return ring_wait(c.p, ring_of(c), g); }
+__device__ __forceinline__ const uint8_t *page_ptr(CCtx &c, uint32_t g) { return ring_page(ring_of(c), g); }
 __device__ __forceinline__ void page_release(CCtx &c, uint32_t g, uint32_t count) {
-  px::mbar_arrive(&c.empty[g % c.p.num_pages], count);
+  ring_release(ring_of(c), g, count);
 }
 
 // Staging layout of an input vector of length K (fp32): element e of 8-chunk
@@ -500,12 +590,19 @@ __device__ __forceinline__ float4 layer_input4(const KParams &p, int l, int b, i
   }
   const size_t BH = (size_t)p.B * p.H;
   float4 x = px::ldcg4(p.xres + (size_t)(l - 1) * BH + (size_t)b * p.H + e4 * 4);
-  for (int k = 0; k < p.ndp; ++k) {
-    float4 d = px::ldcg4(p.dpart + ((size_t)(l - 1) * p.ndp + k) * BH + (size_t)b * p.H + e4 * 4);
-    x.x += d.x;
-    x.y += d.y;
-    x.z += d.z;
-    x.w += d.w;
+  for (int k0 = 0; k0 < p.ndp; k0 += 4) {  // four pieces' loads in flight at a time
+    float4 d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) d[k] = px::ldcg4(p.dpart + ((size_t)(l - 1) * p.ndp + k0 + k) * BH + (size_t)b * p.H + e4 * 4);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) {
+        x.x += d[k].x;
+        x.y += d[k].y;
+        x.z += d[k].z;
+        x.w += d[k].w;
+      }
   }
   return x;
 }
@@ -513,13 +610,23 @@ __device__ __forceinline__ float layer_input1(const KParams &p, int l, int b, in
   if (l == 0) return px::bf16f(__ldg(p.embed + (size_t)tok * p.H + e));
   const size_t BH = (size_t)p.B * p.H;
   float x = px::ldcg(p.xres + (size_t)(l - 1) * BH + (size_t)b * p.H + e);
-  for (int k = 0; k < p.ndp; ++k) x += px::ldcg(p.dpart + ((size_t)(l - 1) * p.ndp + k) * BH + (size_t)b * p.H + e);
+  for (int k0 = 0; k0 < p.ndp; k0 += 4) {
+    float d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) d[k] = px::ldcg(p.dpart + ((size_t)(l - 1) * p.ndp + k0 + k) * BH + (size_t)b * p.H + e);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) x += d[k];
+  }
   return x;
 }
 
 // Stage rms(x)*gamma for every sequence, x = layer_input(l) (l == L: final norm).
 // Contains two compute barriers.
-template <int NB>
+// IT = float4 loads per thread (H / 4 / 256, at least 1), fixed by the caller's
+// rows-per-page so that every load is issued before the first one is used.
+template <int NB, int IT>
 __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only) {
   const KParams &p = c.p;
   const int H = p.H, n4 = H / 4;
@@ -531,14 +638,21 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
     if (b >= p.B) break;
     const int tok = (l == 0 && !from_xres_only) ? read_tok(p, b) : 0;
     float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
-    for (int e4 = c.ctid; e4 < n4; e4 += kComputeThreads) {
-      float4 x;
-      if (from_xres_only)
-        x = px::ldcg4(p.xres + ((size_t)l * p.B + b) * H + e4 * 4);
-      else
-        x = layer_input4(p, l, b, tok, e4);
-      ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-      dst[stage_slot4(e4, H)] = x;
+    float4 xs[IT];
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4)
+        xs[it] = from_xres_only ? px::ldcg4(p.xres + ((size_t)l * p.B + b) * H + e4 * 4) : layer_input4(p, l, b, tok, e4);
+    }
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4) {
+        const float4 x = xs[it];
+        ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+        dst[stage_slot4(e4, H)] = x;
+      }
     }
   }
 #pragma unroll
@@ -559,7 +673,10 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
   for (int b = 0; b < NB; ++b) {
     if (b >= p.B) break;
     float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
-    for (int e4 = c.ctid; e4 < n4; e4 += kComputeThreads) {
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 >= n4) break;
       const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(gamma) + e4);
       float4 x = dst[stage_slot4(e4, H)];
       x.x = x.x * inv[b] * px::bf_lo(gw.x);
@@ -570,27 +687,47 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
     }
   }
   px::cbar();
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
 }
 
-// Stage a plain fp32 vector slice src[b*src_stride + k0 .. k0+K) for each sequence.
-template <int NB>
-__device__ void stage_copy(CCtx &c, const float *src, size_t src_stride, int K) {
+// Stage a plain fp32 vector slice src[b*src_stride .. + K) for each sequence.
+// With nrows > 0 (O projection, batch 1) also stage x_in(l) for output rows
+// row0 .. row0+nrows after the vector, loaded in the same round trip.
+template <int NB, int IT>
+__device__ void stage_copy(CCtx &c, const float *src, size_t src_stride, int K, int l = 0, int row0 = 0,
+                           int nrows = 0) {
   const KParams &p = c.p;
   const int n4 = K / 4;
+  float xr = 0.f;
+  const bool has_row = c.ctid < nrows;
+  if (has_row) xr = layer_input1(p, l, 0, l == 0 ? read_tok(p, 0) : 0, row0 + c.ctid);
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     if (b >= p.B) break;
     float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
-    for (int e4 = c.ctid; e4 < n4; e4 += kComputeThreads)
-      dst[stage_slot4(e4, K)] = px::ldcg4(src + (size_t)b * src_stride + e4 * 4);
+    float4 xs[IT];
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4) xs[it] = px::ldcg4(src + (size_t)b * src_stride + e4 * 4);
+    }
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4) dst[stage_slot4(e4, K)] = xs[it];
+    }
   }
+  for (int r = c.ctid; r < nrows; r += kComputeThreads)
+    c.act[K + r] = (r == c.ctid) ? xr : layer_input1(p, l, 0, l == 0 ? read_tok(p, 0) : 0, row0 + r);
   px::cbar();
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
 }
 
 // acc[b][r] = dot(page row r, staged vector b) for R rows of KC = 8192/R
 // columns; every lane ends with every result.
 template <int NB, int R>
-__device__ __forceinline__ void mv_page(const CCtx &c, const uint8_t *page, float (&acc)[NB][R]) {
+__device__ __forceinline__ void mv_page(const uint8_t *page, const float *act, int act_stride, int B, int lane,
+                                        float (&acc)[NB][R]) {
   constexpr int KC = kPageElems / R;
   constexpr int CH = KC / 8;  // 16-byte chunks per row
   const uint4 *pg = reinterpret_cast<const uint4 *>(page);
@@ -598,16 +735,16 @@ __device__ __forceinline__ void mv_page(const CCtx &c, const uint8_t *page, floa
   for (int b = 0; b < NB; ++b)
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[b][r] = 0.f;
-#pragma unroll(CH / 32 > 4 ? 4 : CH / 32)
+#pragma unroll(CH / 32 > 2 ? 2 : CH / 32)
   for (int j = 0; j < CH / 32; ++j) {
-    const int ch = c.lane + 32 * j;
+    const int ch = lane + 32 * j;
     uint4 w[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) w[r] = pg[r * CH + ch];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (b >= c.p.B) break;
-      const float4 *a = reinterpret_cast<const float4 *>(c.act + (size_t)b * c.act_stride);
+      if (NB > 1 && b >= B) break;
+      const float4 *a = reinterpret_cast<const float4 *>(act + (size_t)b * act_stride);
       const float4 a0 = a[ch], a1 = a[CH + ch];
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -626,7 +763,7 @@ __device__ __forceinline__ void mv_page(const CCtx &c, const uint8_t *page, floa
   }
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    if (b >= c.p.B) break;
+    if (NB > 1 && b >= B) break;
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[b][r] = px::warp_sum(acc[b][r]);
   }
@@ -642,23 +779,33 @@ __device__ __forceinline__ float pick(const float (&v)[R], int idx) {
   return out;
 }
 
+// float4 loads per compute thread to stage a K = 8192 / R vector
+template <int R>
+struct StageIt {
+  static constexpr int v = (8 / R) > 0 ? (8 / R) : 1;
+};
+
 // ---------------------------------------------------------------- matvec ops
 // Loop over the instruction's pages owned by this warp (page g -> warp g % 8).
 template <int NB, int R, class Epi>
-__device__ void matvec_pages(CCtx &c, const Instr &I, Epi epi) {
+__device__ __forceinline__ void matvec_pages(CCtx &c, const Instr &I, Epi epi) {
+  const KParams &p = c.p;
+  const Ring rg = ring_of(c);
   const uint32_t g0 = c.g;
-  const int np = (int)I.b;
-  for (int t = 0; t < np; ++t) {
-    const uint32_t g = g0 + t;
-    if ((int)(g % kComputeWarps) != c.cw) continue;
-    if (!page_ready(c, g)) break;
+  const int np = (int)I.b, first = (int)I.a, cw = c.cw, lane = c.lane, B = p.B, stride = c.act_stride;
+  const float *act = c.act;
+  // this warp's pages: g = g0 + t with g % 8 == cw
+  int t = (int)((uint32_t)(cw - (int)(g0 % kComputeWarps) + kComputeWarps) % kComputeWarps);
+  for (; t < np; t += kComputeWarps) {
+    const uint32_t g = g0 + (uint32_t)t;
+    if (!ring_wait(p, rg, g)) break;
     float acc[NB][R];
-    mv_page<NB, R>(c, page_ptr(c, g), acc);
+    mv_page<NB, R>(ring_page(rg, g), act, stride, B, lane, acc);
     __syncwarp();
-    if (c.lane == 0) page_release(c, g, kComputeWarps);
-    epi(I.a + t, acc);
+    if (lane == 0) ring_release(rg, g, kComputeWarps);
+    epi(first + t, acc);
   }
-  c.g = g0 + np;
+  c.g = g0 + (uint32_t)np;
 }
 
 template <int NB, int R>
@@ -670,32 +817,40 @@ __device__ __noinline__ void op_qkv(CCtx &c, const Instr &I) {
     const int t = __ldcg(p.tokens + c.ctid), pos = __ldg(p.positions + c.ctid);
     if (t < 0 || t >= p.V || pos < 0 || pos >= p.max_seq) record_error(p, MK_ERR_DEVICE_INPUT, c.ctid, t, pos, 0);
   }
-  stage_norm<NB>(c, l, p.layers[l].attn_norm, false);
   const int half = R / 2, pph = p.d / R, hd = p.d / 2;
+  const int pos0 = read_pos(p, 0);
+  if (NB == 1 && c.ctid < hd) c.sh->rope[c.ctid] = __ldg(p.rope + (size_t)pos0 * hd + c.ctid);
+  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].attn_norm, false);
+  const int nq = p.nq, nkv = p.nkv, d = p.d, lane = c.lane, Bn = p.B;
+  float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
+  uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
+  const long long kv_bs = p.kv_bs, kv_hs = p.kv_hs;
+  const int qdim = p.qdim;
+  const float2 *rope_s = c.sh->rope;
+  const float2 *rope_g = p.rope;
   matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
     const int head = j / pph, jj = j % pph;
-    if (c.lane >= half) return;
-    const int i = jj * half + c.lane;  // rotation pair index inside the head
+    if (lane >= half) return;
+    const int i = jj * half + lane;  // rotation pair index inside the head
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (b >= p.B) break;
-      float u = pick<R>(acc[b], c.lane), w = pick<R>(acc[b], c.lane + half);
-      const int pos = read_pos(p, b);
-      if (head < p.nq + p.nkv) {
-        const float2 cs = __ldg(p.rope + (size_t)pos * hd + i);
+      if (NB > 1 && b >= Bn) break;
+      float u = pick<R>(acc[b], lane), w = pick<R>(acc[b], lane + half);
+      const int pos = NB == 1 ? pos0 : read_pos(p, b);
+      if (head < nq + nkv) {
+        const float2 cs = NB == 1 ? rope_s[i] : __ldg(rope_g + (size_t)pos * hd + i);
         const float u2 = u * cs.x - w * cs.y, w2 = u * cs.y + w * cs.x;
         u = u2;
         w = w2;
       }
-      if (head < p.nq) {
-        float *q = p.qbuf + ((size_t)l * p.B + b) * p.qdim + head * p.d;
+      if (head < nq) {
+        float *q = qrow + (size_t)b * qdim + head * d;
         q[i] = u;
         q[i + hd] = w;
       } else {
-        const bool isk = head < p.nq + p.nkv;
-        const int gk = isk ? head - p.nq : head - p.nq - p.nkv;
-        uint16_t *dst = (isk ? p.kc : p.vc) + (size_t)l * p.kv_ls + (size_t)b * p.kv_bs + (size_t)gk * p.kv_hs +
-                        (size_t)pos * p.d;
+        const bool isk = head < nq + nkv;
+        const int gk = isk ? head - nq : head - nq - nkv;
+        uint16_t *dst = (isk ? kl : vl) + (size_t)b * kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
         dst[i] = px::f2bf(u);
         dst[i + hd] = px::f2bf(w);
       }
@@ -707,16 +862,20 @@ template <int NB, int R>
 __device__ __noinline__ void op_oproj(CCtx &c, const Instr &I) {
   const KParams &p = c.p;
   const int l = I.layer;
-  stage_copy<NB>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim);
+  const int row0 = (int)I.a * R, nrows = NB == 1 ? (int)I.b * R : 0;
+  stage_copy<NB, StageIt<R>::v>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim, l, row0, nrows);
+  const int lane = c.lane, Bn = p.B, H = p.H;
+  const float *xrows = c.act + p.qdim - row0;
+  float *const xout = p.xres + (size_t)l * Bn * H;
   matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    if (c.lane >= R) return;
-    const int row = j * R + c.lane;
+    if (lane >= R) return;
+    const int row = j * R + lane;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (b >= p.B) break;
-      const float v = pick<R>(acc[b], c.lane);
-      const float xin = layer_input1(p, l, b, l == 0 ? read_tok(p, b) : 0, row);
-      p.xres[((size_t)l * p.B + b) * p.H + row] = xin + v;
+      if (NB > 1 && b >= Bn) break;
+      const float v = pick<R>(acc[b], lane);
+      const float xin = NB == 1 ? xrows[row] : layer_input1(p, l, b, l == 0 ? read_tok(p, b) : 0, row);
+      xout[(size_t)b * H + row] = xin + v;
     }
   });
 }
@@ -725,17 +884,18 @@ template <int NB, int R>
 __device__ __noinline__ void op_gateup(CCtx &c, const Instr &I) {
   const KParams &p = c.p;
   const int l = I.layer;
-  stage_norm<NB>(c, l, p.layers[l].ffn_norm, true);
-  const int half = R / 2;
+  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].ffn_norm, true);
+  const int half = R / 2, lane = c.lane, Bn = p.B, F = p.F;
+  float *const aout = p.actb + (size_t)l * Bn * F;
   matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    if (c.lane >= half) return;
-    const int row = j * half + c.lane;
+    if (lane >= half) return;
+    const int row = j * half + lane;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (b >= p.B) break;
-      const float gt = pick<R>(acc[b], c.lane), up = pick<R>(acc[b], c.lane + half);
+      if (NB > 1 && b >= Bn) break;
+      const float gt = pick<R>(acc[b], lane), up = pick<R>(acc[b], lane + half);
       const float silu = gt / (1.0f + expf(-gt));
-      p.actb[((size_t)l * p.B + b) * p.F + row] = silu * up;
+      aout[(size_t)b * F + row] = silu * up;
     }
   });
 }
@@ -744,14 +904,16 @@ template <int NB, int R>
 __device__ __noinline__ void op_down(CCtx &c, const Instr &I) {
   const KParams &p = c.p;
   const int l = I.layer, k = I.c;
-  stage_copy<NB>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
+  stage_copy<NB, StageIt<R>::v>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
+  const int lane = c.lane, Bn = p.B, H = p.H;
+  float *const dout = p.dpart + ((size_t)l * p.ndp + k) * Bn * H;
   matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    if (c.lane >= R) return;
-    const int row = j * R + c.lane;
+    if (lane >= R) return;
+    const int row = j * R + lane;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (b >= p.B) break;
-      p.dpart[(((size_t)l * p.ndp + k) * p.B + b) * p.H + row] = pick<R>(acc[b], c.lane);
+      if (NB > 1 && b >= Bn) break;
+      dout[(size_t)b * H + row] = pick<R>(acc[b], lane);
     }
   });
 }
@@ -763,7 +925,7 @@ __device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi) {
 template <int NB, int R>
 __device__ __noinline__ void op_lmhead(CCtx &c, const Instr &I) {
   const KParams &p = c.p;
-  stage_norm<NB>(c, p.L, p.final_norm, false);
+  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false);
   float bv[NB];
   int bi[NB];
 #pragma unroll
@@ -771,15 +933,17 @@ __device__ __noinline__ void op_lmhead(CCtx &c, const Instr &I) {
     bv[b] = -INFINITY;
     bi[b] = 0x7fffffff;
   }
+  const int lane = c.lane, Bn = p.B, V = p.V;
+  float *const logits = p.logits;
   matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    const int row = j * R + c.lane;
-    const bool valid = c.lane < R && row < p.V;
+    const int row = j * R + lane;
+    const bool valid = lane < R && row < V;
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (b >= p.B) break;
-      const float v = pick<R>(acc[b], c.lane);
+      if (NB > 1 && b >= Bn) break;
+      const float v = pick<R>(acc[b], lane);
       if (valid) {
-        if (p.logits) p.logits[(size_t)b * p.V + row] = v;
+        if (logits) logits[(size_t)b * V + row] = v;
         if (arg_better(v, row, bv[b], bi[b])) {
           bv[b] = v;
           bi[b] = row;
@@ -821,27 +985,52 @@ __device__ __noinline__ void op_lmhead(CCtx &c, const Instr &I) {
     p.arg_idx[(size_t)b * p.n_lm + I.c] = i;
   }
   px::cbar();
-  // the last LM instruction to finish merges every slot
+  // the last LM instruction to finish merges every slot (all compute threads
+  // load a share of the slots at once, then a tree reduction)
   if (c.ctid == 0) {
-    __threadfence();
+    px::fence_acq_rel_gpu();
     const unsigned old = px::atom_add_acq_rel(p.ctr + p.arg_ticket0, 1u);
     c.sh->flag = (old == c.epoch * (unsigned)p.n_lm - 1u);
   }
   px::cbar();
-  if (c.sh->flag && c.ctid < p.B) {
-    __threadfence();
-    const int b = c.ctid;
-    float v = -INFINITY;
-    int i = 0x7fffffff;
-    for (int s = 0; s < p.n_lm; ++s) {
-      const float sv = __ldcg(p.arg_val + (size_t)b * p.n_lm + s);
-      const int si = __ldcg(p.arg_idx + (size_t)b * p.n_lm + s);
-      if (arg_better(sv, si, v, i)) {
-        v = sv;
-        i = si;
+  if (c.sh->flag) {  // uniform: every compute thread reads the same flag
+    for (int b = 0; b < p.B; ++b) {
+      float v = -INFINITY;
+      int i = 0x7fffffff;
+      for (int s0 = c.ctid; s0 < p.n_lm; s0 += kComputeThreads) {
+        const float sv = __ldcg(p.arg_val + (size_t)b * p.n_lm + s0);
+        const int si = __ldcg(p.arg_idx + (size_t)b * p.n_lm + s0);
+        if (arg_better(sv, si, v, i)) {
+          v = sv;
+          i = si;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+        if (arg_better(v2, i2, v, i)) {
+          v = v2;
+          i = i2;
+        }
+      }
+      if (c.lane == 0) {
+        c.sh->argv[c.cw][b] = v;
+        c.sh->argi[c.cw][b] = i;
       }
     }
-    p.next_tokens[b] = (i == 0x7fffffff) ? 0 : i;
+    px::cbar();
+    if (c.ctid < p.B) {
+      const int b = c.ctid;
+      float v = -INFINITY;
+      int i = 0x7fffffff;
+      for (int w = 0; w < kComputeWarps; ++w)
+        if (arg_better(c.sh->argv[w][b], c.sh->argi[w][b], v, i)) {
+          v = c.sh->argv[w][b];
+          i = c.sh->argi[w][b];
+        }
+      p.next_tokens[b] = (i == 0x7fffffff) ? 0 : i;
+    }
   }
 }
 
@@ -976,6 +1165,7 @@ __device__ __noinline__ void op_attn_t(CCtx &c, const Instr &I) {
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int i = 0; i < DPL; ++i) q[h][i] = px::ldcg(qb + h * D + c.lane * DPL + i) * p.attn_scale;
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
   float m[G], lsum[G], o[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -995,23 +1185,25 @@ __device__ __noinline__ void op_attn_t(CCtx &c, const Instr &I) {
       reinterpret_cast<uint32_t *>(cur + D)[i] = __ldcg(reinterpret_cast<const unsigned int *>(p.vc + off) + i);
     }
   }
+  const Ring rg = ring_of(c);
+  const int cw = c.cw, lane = c.lane;
   for (int t = 0; t < npg; ++t) {
     const uint32_t gg = c.g + t;
-    if (!page_ready(c, gg)) break;
-    const uint8_t *pg = page_ptr(c, gg);
+    if (!ring_wait(p, rg, gg)) break;
+    const uint8_t *pg = ring_page(rg, gg);
     const int p0 = r.start + t * PPP;
     const int cnt = min(PPP, r.pref_end - p0);
 #pragma unroll
     for (int sb = 0; sb < PW / PB; ++sb) {
-      const int jb = c.cw * PW + sb * PB;
+      const int jb = cw * PW + sb * PB;
       const int nvalid = max(0, min(PB, cnt - jb));
       if (nvalid > 0)
         attn_block<G, DPL, PB>(q, reinterpret_cast<const uint16_t *>(pg) + (size_t)jb * D,
                                reinterpret_cast<const uint16_t *>(pg + kPageBytes / 2) + (size_t)jb * D, nvalid,
-                               c.lane, m, lsum, o);
+                               lane, m, lsum, o);
     }
     __syncwarp();
-    if (c.lane == 0) page_release(c, gg, 1);
+    if (lane == 0) ring_release(rg, gg, 1);
   }
   c.g += npg;
   __syncwarp();
@@ -1054,26 +1246,68 @@ __device__ __noinline__ void op_attn_t(CCtx &c, const Instr &I) {
   }
   px::cbar();
   if (c.ctid == 0) {
-    __threadfence();
+    px::fence_acq_rel_gpu();
     const unsigned t = p.attn_ticket0 + ((unsigned)l * p.B + b) * p.nkv + g;
     const unsigned old = px::atom_add_acq_rel(p.ctr + t, 1u);
     c.sh->flag = (old == c.epoch * (unsigned)p.S - 1u);
   }
   px::cbar();
-  if (c.sh->flag) {
-    __threadfence();
-    for (int e = c.ctid; e < G * D; e += kComputeThreads) {
-      const int h = e / D, dd = e % D;
-      const size_t hb = (hbase + h) * p.S;
+  if (c.sh->flag) {  // uniform: the last split of the group merges all S splits
+    constexpr int NE = G * D;                            // outputs of the group
+    constexpr int EPT = (NE + kComputeThreads - 1) / kComputeThreads;
+    constexpr int SB = (64 / EPT) < 32 ? (64 / EPT) : 32;  // splits per load batch
+    const int S = p.S;
+    float *sml = scr;  // [G][S] (m, l) then (weight, -)
+    for (int i = c.ctid; i < G * S; i += kComputeThreads) {
+      const int h = i / S, sp = i % S;
+      const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml) + (hbase + h) * S + sp);
+      sml[2 * i] = ml.x;
+      sml[2 * i + 1] = ml.y;
+    }
+    // the first batch of this thread's partial outputs, in flight with the table
+    float ov[EPT][SB];
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int idx = c.ctid + e * kComputeThreads;
+      const int h = idx / D, dd = idx % D;
+#pragma unroll
+      for (int j = 0; j < SB; ++j)
+        ov[e][j] = (idx < NE && j < S) ? __ldcg(p.part_o + ((hbase + h) * S + j) * D + dd) : 0.f;
+    }
+    px::cbar();
+    if (c.ctid < G) {  // per head: max, weights exp(m_s - M), and the total weight L
+      const int h = c.ctid;
       float M = -INFINITY;
-      for (int sp = 0; sp < p.S; ++sp) M = fmaxf(M, __ldcg(p.part_ml + (hb + sp) * 2));
-      float L = 0.f, O = 0.f;
-      for (int sp = 0; sp < p.S; ++sp) {
-        const float ms = __ldcg(p.part_ml + (hb + sp) * 2);
-        const float f = (ms == -INFINITY) ? 0.f : expf(ms - M);
-        L += f * __ldcg(p.part_ml + (hb + sp) * 2 + 1);
-        O += f * __ldcg(p.part_o + (hb + sp) * D + dd);
+      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, sml[2 * (h * S + sp)]);
+      float L = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float ms = sml[2 * (h * S + sp)];
+        const float wgt = (ms == -INFINITY) ? 0.f : expf(ms - M);
+        L += wgt * sml[2 * (h * S + sp) + 1];
+        sml[2 * (h * S + sp)] = wgt;
       }
+      c.sh->red[h % kComputeWarps][h / kComputeWarps] = L;
+    }
+    px::cbar();
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int idx = c.ctid + e * kComputeThreads;
+      if (idx >= NE) break;
+      const int h = idx / D, dd = idx % D;
+      float O = 0.f;
+#pragma unroll
+      for (int j = 0; j < SB; ++j)
+        if (j < S) O += sml[2 * (h * S + j)] * ov[e][j];
+      for (int s0 = SB; s0 < S; s0 += SB) {  // further batches (S > SB)
+        float tmp[SB];
+#pragma unroll
+        for (int j = 0; j < SB; ++j)
+          tmp[j] = (s0 + j < S) ? __ldcg(p.part_o + ((hbase + h) * S + s0 + j) * D + dd) : 0.f;
+#pragma unroll
+        for (int j = 0; j < SB; ++j)
+          if (s0 + j < S) O += sml[2 * (h * S + s0 + j)] * tmp[j];
+      }
+      const float L = c.sh->red[h % kComputeWarps][h / kComputeWarps];
       p.obuf[((size_t)l * p.B + b) * p.qdim + (size_t)(g * G + h) * D + dd] = O / L;
     }
   }
@@ -1107,6 +1341,8 @@ __device__ void op_attn(CCtx &c, const Instr &I) {
     case 16: fn<NB, 16>(c, I); break;             \
     default: fn<NB, 32>(c, I); break;             \
   }
+
+__device__ __forceinline__ int &sh_stat(CCtx &c) { return c.sh->stat_cwait; }
 
 template <int NB>
 __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile int *dyn_tail,
@@ -1151,6 +1387,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
     if (bad) c.sh->abort = 1;
     if (px::cbar_or(bad || px::ld_volatile(&c.sh->abort))) break;
     if (tr && c.ctid == 0) tr[1] = px::gtimer();
+    c.tr = tr;
     switch (I.op) {
       case OP_QKV: MK_DISPATCH_R(op_qkv, NB, p.Rh, c, I); break;
       case OP_ATTN: op_attn(c, I); break;
@@ -1160,18 +1397,19 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
       case OP_LMHEAD: MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I); break;
       default: break;
     }
-    if (tr && c.ctid == 0) tr[2] = px::gtimer();
+    if (tr && c.ctid == 0) tr[3] = px::gtimer();
     const bool abort_now = px::cbar_or(px::ld_volatile(&c.sh->abort) != 0);
     if (abort_now) break;
     // all of this CTA's outputs of the instruction are written: publish
     const bool sig = I.sig_ctr != kNoCounter && (I.op != OP_ATTN || c.sh->flag);
     if (c.ctid == 0 && sig) {
-      __threadfence();
+      px::fence_acq_rel_gpu();
       for (int k = 0; k < I.sig_n; ++k) px::red_release_add(p.ctr + I.sig_ctr + k, 1u);
     }
     if (tr && c.ctid == 0) {
-      tr[3] = px::gtimer();
-      tr[4] = (uint64_t)I.op | ((uint64_t)I.layer << 8) | ((uint64_t)blockIdx.x << 16);
+      tr[4] = px::gtimer();
+      tr[7] = (uint64_t)I.op | ((uint64_t)I.layer << 8) | ((uint64_t)blockIdx.x << 16);
+      tr[8] = (unsigned)atomicExch(&sh_stat(c), 0);
     }
     px::cbar();  // the staging region and the broadcast flag are reused next
   }
@@ -1201,6 +1439,8 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
     px::fence_mbar_init();
     sh->abort = 0;
     sh->flag = 0;
+    sh->stat_cwait = 0;
+    for (int i = 0; i < 16; ++i) sh->slot_last[i] = 0;
     *dyn_tail = 0;
     *dyn_head = 0;
   }
@@ -1209,13 +1449,33 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   Queue q;
   q.base = p.instrs + p.q_off[blockIdx.x];
   q.len = p.q_len[blockIdx.x];
-  if (warp == 0) {
-    if (lane == 0) run_loader<RAW>(p, sh, pages, full, empty, q, dyn_fifo, dyn_tail, dyn_head, epoch);
+  if (warp < kLoaders) {
+    // the dynamic queue is claimed by one loader only
+    const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
+    if (lane == 0 && (!dyn || warp == 0))
+      run_loader<RAW>(p, sh, pages, full, empty, q, dyn_fifo, dyn_tail, dyn_head, epoch, warp, dyn ? 1 : kLoaders);
   } else {
-    CCtx c{p, sh, pages, act, act_stride, full, empty, epoch, warp - 1, lane, (int)threadIdx.x - 32, 0u};
+    CCtx c{p, sh, pages, act, act_stride, full, empty, epoch, warp - kLoaders, lane,
+           (int)threadIdx.x - 32 * kLoaders, 0u, nullptr};
     run_compute<NB>(c, q, dyn_fifo, dyn_tail, dyn_head);
   }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    // every bulk copy must land before the CTA exits: after an abort the
+    // compute warps stop consuming pages, so wait on each slot's latest use
+    for (int s = 0; s < NP; ++s) {
+      const uint32_t last = sh->slot_last[s];
+      if (last == 0) continue;
+      const uint32_t ph = ((last - 1) / (uint32_t)NP) & 1u;
+      const uint64_t t0 = px::gtimer();
+      while (!px::mbar_test(&full[s], ph)) {
+        if (px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
+          record_error(p, MK_ERR_TIMEOUT, -2, 2, s, (int)last);
+          break;
+        }
+      }
+    }
+  }
   if (threadIdx.x == 0 && (p.mode & MODE_FINAL_LAUNCH)) {
     __threadfence();
     const unsigned old = px::atom_add_acq_rel(p.ctr + p.exit_ticket, 1u);

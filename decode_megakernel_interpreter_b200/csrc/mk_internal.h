@@ -13,11 +13,14 @@ namespace mk {
 // page holds R rows x KC columns of bf16 with R * KC = 8192.
 constexpr int kPageBytes = 16384;
 constexpr int kPageElems = kPageBytes / 2;
-constexpr int kComputeWarps = 8;              // warps 1..8
-constexpr int kThreads = 32 * (1 + kComputeWarps);
+constexpr int kLoaders = 2;                   // loader warps (lane 0 of each issues bulk copies)
+constexpr int kComputeWarps = 8;              // warps kLoaders .. kLoaders+7
+constexpr int kThreads = 32 * (kLoaders + kComputeWarps);
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kMaxKc = 4096;                  // largest K staged in one page row
 constexpr int kMaxBatch = 16;
+constexpr int kMaxDownPieces = 8;             // ffn / 2048 at most
+constexpr int kDefaultInflight = 6;           // bulk-copy pages in flight per CTA
 
 // ---------------------------------------------------------------- opcodes
 // The instruction set of the decode step (the fused instructions the
@@ -127,6 +130,7 @@ struct KParams {
   int num_pages;          // ring pages per CTA
   long long act_floats;   // floats of the staging region (input vectors, attention scratch)
   int pf_pages;           // L2 prefetch distance in pages (0 = off)
+  int max_inflight;       // bulk-copy pages in flight per CTA (0 = no cap)
   long long timeout_ns;
   unsigned long long *trace;  // [n_instr][5]
   uint32_t mode;

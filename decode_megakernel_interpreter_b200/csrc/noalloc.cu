@@ -150,11 +150,13 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
 
   // shared memory geometry (as mk_plan)
   const int G = s.nq / s.nkv;
-  size_t act = std::max(std::max((size_t)s.H, qd), (size_t)p.KCd);
+  size_t act = std::max(std::max((size_t)s.H, qd + (size_t)s.H), (size_t)p.KCd);
   act = std::max(act, (size_t)kComputeWarps * G * (s.d + 2) + s.d);
   act = (act + 31) / 32 * 32;
   int num_pages = std::min(16, (slot->smem_optin - shared_bytes_fixed(0, act)) / (kPageBytes + 16));
-  if (num_pages < 2) return MK_ERR_UNSUPPORTED_SHAPE;
+  num_pages = num_pages / kLoaders * kLoaders;  // as mk_plan: unambiguous mbarrier phases
+  while (num_pages > 0 && (2 * num_pages) % kComputeWarps) num_pages -= kLoaders;
+  if (num_pages < 2 * kLoaders) return MK_ERR_UNSUPPORTED_SHAPE;
   const int smem = shared_bytes_fixed(num_pages, act);
 
   unsigned char *base = slot->scratch;
@@ -271,6 +273,7 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   k.num_pages = num_pages;
   k.act_floats = (long long)act;
   k.pf_pages = 0;
+  k.max_inflight = std::max(kLoaders, std::min(kDefaultInflight, num_pages) / kLoaders * kLoaders);
   k.timeout_ns = 1000000000LL;
   k.trace = nullptr;
   k.mode = MODE_FINAL_LAUNCH;

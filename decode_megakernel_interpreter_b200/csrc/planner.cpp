@@ -48,6 +48,7 @@ std::string check_shape(const Shape &s, int B) {
     return buf;
   }
   if (s.F % (Rh / 2)) return "ffn must be a multiple of half the rows per page";
+  if (s.F / kc > kMaxDownPieces) return "ffn above 16384 is not implemented";
   if (B < 1 || B > kMaxBatch) return "batch must be in [1, 16]";
   return "";
 }

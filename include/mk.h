@@ -128,11 +128,15 @@ typedef struct {
   int32_t num_sms;        /* CTAs of the persistent grid; 0 = every SM */
   int32_t trace;          /* 1: record per-instruction timestamps (mk_trace_read) */
   int64_t wait_timeout_ns;/* bound on every device-side wait; 0 = 1 second */
-  int32_t l2_prefetch_kb; /* per-SM L2 prefetch distance ahead of shared memory;
-                             0 = automatic, -1 = off */
+  int32_t l2_prefetch_kb; /* reserved (an L2 prefetch cursor measured slower on
+                             B200 and was removed); accepted and ignored */
   int32_t debug_drop_producer; /* TEST HOOK: 1 drops one producer instruction so
                              that a dependency can never be met and the bounded
                              wait must report MK_ERR_TIMEOUT; 0 in normal use */
+  int32_t max_inflight_pages; /* 16 KiB weight/KV pages a CTA keeps in flight
+                             (the rest of its page ring only buffers landed
+                             pages); 0 = automatic (6), -1 = no cap; rounded
+                             down to a multiple of the loader count (2) */
 } mk_plan_opts;
 
 /*
@@ -197,6 +201,14 @@ typedef struct {
   int64_t weight_bytes_per_step; /* weight bytes the plan streams per step */
 } mk_plan_info;
 
+/*
+ * mk_get_error_detail: the detail words of the last device-side error that
+ * mk_get_status returned (host int32 [6]): instruction sequence number (-1:
+ * a shared-memory page wait, -2: the final drain), counter index or wait kind,
+ * observed value, target value, CTA, and the abort flag.  All zero if none.
+ */
+int mk_get_error_detail(const mk_handle *h, int32_t detail[6]);
+
 /* Fill *info for the current plan.  MK_ERR_NOT_PLANNED before mk_plan. */
 int mk_get_plan_info(const mk_handle *h, mk_plan_info *info);
 
@@ -205,10 +217,13 @@ int mk_get_plan_info(const mk_handle *h, mk_plan_info *info);
  * `out` (host, uint64 [num_instructions][MK_TRACE_WORDS], nanoseconds of the
  * device global timer).  Requires a plan with trace = 1; synchronises.
  * Word meaning: 0 = instruction fetched by the compute warps, 1 = its
- * dependencies were met, 2 = its input vector was staged, 3 = it signalled
- * completion; 4 = (opcode | layer << 8 | cta << 16).
+ * dependencies were met, 2 = its input vector was staged, 3 = its pages were
+ * consumed and its outputs written, 4 = it signalled completion, 5 / 6 = the
+ * loader issued its first / last page (5 == 6 when it has no pages),
+ * 7 = (opcode | layer << 8 | cta << 16), 8 = pages the compute warps found
+ * not yet landed, 9 = pages the loader found no free ring slot for.
  */
-#define MK_TRACE_WORDS 5
+#define MK_TRACE_WORDS 10
 int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
 
 /* ------------------------------------------------------------------ allocation-free step */

@@ -72,4 +72,4 @@ def test_unsupported_shape_rejected_before_any_device_call():
 def test_struct_layouts_match_headers():
     assert ctypes.sizeof(mk.mk_instr_desc) == 32
     assert ctypes.sizeof(mk.mk_config) == 56
-    assert ctypes.sizeof(mk.mk_plan_opts) == 40
+    assert ctypes.sizeof(mk.mk_plan_opts) == 48

@@ -40,7 +40,8 @@ def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan
             tokens.fill_(tok)
             pos.fill_(p)
             eng.decode_step(tokens, pos, logits, nxt)
-            assert eng.status() == mk.MK_OK
+            rc = eng.status()
+            assert rc == mk.MK_OK, (rc, mk.mk_get_error_detail(eng.h))
             gl = logits[b].cpu().numpy()
             gn = int(nxt[b].item())
             assert gn == int(np.argmax(gl)), "next token must be the first maximal logit"
@@ -215,10 +216,12 @@ def test_trace_records_every_instruction(tiny_model):
     tr = eng.trace()
     eng.close()
     assert tr.shape == (info.num_instructions, mk.MK_TRACE_WORDS)
-    ops = tr[:, 4] & 0xFF
+    ops = tr[:, 7] & 0xFF
     assert set(ops.tolist()) == {1, 2, 3, 4, 5, 6}
-    assert np.all(tr[:, 0] <= tr[:, 1]) and np.all(tr[:, 1] <= tr[:, 2]) and np.all(tr[:, 2] <= tr[:, 3])
-    assert np.all(tr[:, 3] - tr[:, 0] < 1_000_000_000)
+    for a, b in ((0, 1), (1, 2), (2, 3), (3, 4), (5, 6)):
+        assert np.all(tr[:, a] <= tr[:, b]), (a, b)
+    assert np.all(tr[:, 4] - tr[:, 0] < 1_000_000_000)
+    assert np.all(tr[:, 5] > 0)
 
 
 # ------------------------------------------------------------------ full-size shapes
