@@ -40,7 +40,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--workload", default="llama1b")
-    ap.add_argument("--exec-mode", default="megakernel", choices=["megakernel", "per_op", "per_op_graph"])
+    ap.add_argument("--exec-mode", default="megakernel",
+                    choices=["megakernel", "megakernel_generic", "per_op", "per_op_graph"])
     ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--l2-prefetch-kb", type=int, default=0)
@@ -257,7 +258,9 @@ def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
                                      "mean_stage_us": float(stage.mean()), "mean_pages_us": float(pages.mean()),
                                      "mean_signal_us": float(sig.mean()),
                                      "mean_body_us": float((tr[m, 3] - tr[m, 1]).mean() / 1e3),
-                                     "consumer_page_waits": int(tr[m, 8].sum()), "loader_ring_full": int(tr[m, 9].sum())}
+                                     "consumer_page_waits": int((tr[m, 8] & 0xffffffff).sum()),
+                                     "tagged_load_retries": int((tr[m, 8] >> 32).sum()),
+                                     "loader_ring_full": int(tr[m, 9].sum())}
     return out
 
 
@@ -343,7 +346,7 @@ def main():
         ms = float(t.item())
     us_step = 1e3 * ms / K
     value = world * K / (ms / 1e3)
-    launches_per_step = 1 if args.exec_mode == "megakernel" else s.n_layers * 5 + 1
+    launches_per_step = 1 if args.exec_mode.startswith("megakernel") else s.n_layers * 5 + 1
 
     # end to end through the C ABI with host buffers: per step copy the token
     # and position in from pinned memory, run, read the next token back
@@ -399,12 +402,13 @@ def main():
                                    f"{K} greedy steps" if w.name == "llama1b" else w.name,
                        "batch": B, "context": ctx, "exec_mode": args.exec_mode, "sched": args.sched,
                        "kv_splits": info.kv_splits, "ctas": info.num_ctas, "smem_pages": info.num_pages,
+                       "interpreter": "shape-specialised" if info.kernel_variant == 1 else "shape-generic",
                        "parallelism": "replicas only" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2 (weights streamed once per step, 2.5 GB)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                          "traffic": ncu_traffic(args.workload), "algorithmic_bytes_per_step": bytes_step,
-                         "kernel": "mk::interp_kernel<1>"},
+                         "kernel": "mk::interp_kernel"},
             "clocks": clk.summary(),
             "gpu_launches": K * launches_per_step,
         }

@@ -27,7 +27,7 @@ MK_ERR_DEVICE_INPUT = -7
 MK_ERR_OUT_OF_MEMORY = -8
 
 MK_SCHED_STATIC, MK_SCHED_DYNAMIC = 0, 1
-MK_EXEC_MEGAKERNEL, MK_EXEC_PER_OP, MK_EXEC_PER_OP_GRAPH = 0, 1, 2
+MK_EXEC_MEGAKERNEL, MK_EXEC_PER_OP, MK_EXEC_PER_OP_GRAPH, MK_EXEC_MEGAKERNEL_GENERIC = 0, 1, 2, 3
 MK_TRACE_WORDS = 10
 
 OP_NAMES = {0: "nop", 1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"}
@@ -71,7 +71,8 @@ class mk_plan_info(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int32), ("threads_per_cta", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32), ("num_instructions", ctypes.c_int32),
                 ("num_counters", ctypes.c_int32), ("kv_splits", ctypes.c_int32), ("max_queue_len", ctypes.c_int32),
-                ("weight_bytes_per_step", ctypes.c_int64)]
+                ("weight_bytes_per_step", ctypes.c_int64), ("kernel_variant", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class mk_instr_desc(ctypes.Structure):
@@ -234,7 +235,7 @@ def plan_opts(batch: int = 1, kv_splits: int = 0, sched: str = "static", exec_mo
               num_sms: int = 0, trace: bool = False, wait_timeout_ns: int = 0, l2_prefetch_kb: int = 0,
               debug_drop_producer: bool = False, max_inflight_pages: int = 0) -> mk_plan_opts:
     return mk_plan_opts(batch, kv_splits, {"static": 0, "dynamic": 1}[sched],
-                        {"megakernel": 0, "per_op": 1, "per_op_graph": 2}[exec_mode], num_sms, int(trace),
+                        {"megakernel": 0, "per_op": 1, "per_op_graph": 2, "megakernel_generic": 3}[exec_mode], num_sms, int(trace),
                         wait_timeout_ns, l2_prefetch_kb, int(debug_drop_producer), max_inflight_pages)
 
 

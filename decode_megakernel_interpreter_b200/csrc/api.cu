@@ -13,14 +13,9 @@
 
 #include "../../include/mk.h"
 #include "../../include/mk_host.h"
+#include "interp_launch.h"
 #include "mk_internal.h"
 #include "planner.h"
-
-namespace mk {
-cudaError_t launch_interp(const KParams &p, int nb, int grid, int smem, cudaStream_t st, bool cooperative);
-cudaError_t occupancy_interp(int nb, int smem, int *blocks_per_sm);
-int shared_bytes_fixed(int num_pages, size_t act_floats);
-}  // namespace mk
 
 using namespace mk;
 
@@ -39,8 +34,12 @@ struct mk_handle {
   uint16_t *wqkv = nullptr, *wgu = nullptr, *wd = nullptr;
   LayerDev *d_layers = nullptr;
   float2 *d_rope = nullptr;
-  float *qbuf = nullptr, *obuf = nullptr, *xres = nullptr, *actb = nullptr, *dpart = nullptr;
+  // tagged fp32 activation words (the step number mod 4 in the two low
+  // mantissa bits)
+  float *qbuf = nullptr, *obuf = nullptr, *xres = nullptr, *actb = nullptr, *dpart = nullptr, *kvcur = nullptr;
   unsigned *ctr_epoch = nullptr;  // [0] = epoch
+  // every tagged buffer (pointer, bytes): zeroed whenever the step number restarts
+  std::vector<std::pair<void *, size_t>> tagged;
   int *status = nullptr;
   // owned per plan
   std::vector<void *> plan_allocs;
@@ -49,6 +48,8 @@ struct mk_handle {
   mk_plan_opts opts;
   KParams kp;
   int smem = 0, grid = 0, nb = 1;
+  const void *kernel = nullptr;  // the interpreter build this plan launches
+  int kernel_variant = 0;        // 1: specialised for this model's shape
   int last_detail[6] = {0, 0, 0, 0, 0, 0};
   // per-op graph mode
   cudaGraphExec_t gexec = nullptr;
@@ -333,11 +334,17 @@ extern "C" int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_
   if ((rc = build_rope(h))) return fail(rc);
   const Shape &s = h->shape;
   const size_t Bm = cfg->max_batch;
-  if ((rc = dalloc(h->allocs, &h->qbuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
-  if ((rc = dalloc(h->allocs, &h->obuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
-  if ((rc = dalloc(h->allocs, &h->xres, (size_t)s.L * Bm * s.H))) return fail(rc);
-  if ((rc = dalloc(h->allocs, &h->actb, (size_t)s.L * Bm * s.F))) return fail(rc);
-  if ((rc = dalloc(h->allocs, &h->dpart, (size_t)s.L * geo.ndp * Bm * s.H))) return fail(rc);
+  auto tagged = [&](float **ptr, size_t n) {
+    int r = dalloc(h->allocs, ptr, n);
+    if (!r) h->tagged.push_back({*ptr, n * sizeof(float)});
+    return r;
+  };
+  if ((rc = tagged(&h->qbuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
+  if ((rc = tagged(&h->obuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
+  if ((rc = tagged(&h->xres, (size_t)s.L * Bm * s.H))) return fail(rc);
+  if ((rc = tagged(&h->actb, (size_t)s.L * Bm * s.F))) return fail(rc);
+  if ((rc = tagged(&h->dpart, (size_t)s.L * geo.ndp * Bm * s.H))) return fail(rc);
+  if ((rc = tagged(&h->kvcur, (size_t)s.L * Bm * 2 * s.nkv * s.d))) return fail(rc);
   if ((rc = dalloc(h->allocs, &h->ctr_epoch, 4))) return fail(rc);
   if ((rc = dalloc(h->allocs, &h->status, kStatusWords))) return fail(rc);
   e = cudaDeviceSynchronize();
@@ -363,8 +370,9 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   mk_plan_opts o = opts_in ? *opts_in : default_opts(h->cfg);
   if (o.batch < 1 || o.batch > h->cfg.max_batch) return MK_ERR_INVALID_ARG;
   if (o.sched_mode != MK_SCHED_STATIC && o.sched_mode != MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
-  if (o.exec_mode < MK_EXEC_MEGAKERNEL || o.exec_mode > MK_EXEC_PER_OP_GRAPH) return MK_ERR_INVALID_ARG;
-  if (o.exec_mode != MK_EXEC_MEGAKERNEL && o.sched_mode == MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
+  if (o.exec_mode < MK_EXEC_MEGAKERNEL || o.exec_mode > MK_EXEC_MEGAKERNEL_GENERIC) return MK_ERR_INVALID_ARG;
+  const bool one_launch = o.exec_mode == MK_EXEC_MEGAKERNEL || o.exec_mode == MK_EXEC_MEGAKERNEL_GENERIC;
+  if (!one_launch && o.sched_mode == MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
   if (o.kv_splits < 0 || o.num_sms < 0 || o.wait_timeout_ns < 0) return MK_ERR_INVALID_ARG;
   if (o.batch > 1) return MK_ERR_UNSUPPORTED_SHAPE;  // batched instructions: not in this build yet
   cudaError_t ce = cudaDeviceSynchronize();
@@ -394,8 +402,19 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   while (num_pages > 0 && (2 * num_pages) % kComputeWarps) num_pages -= kLoaders;
   if (num_pages < 2 * kLoaders) return MK_ERR_UNSUPPORTED_SHAPE;
   const int smem = shared_bytes_fixed(num_pages, act_floats);
+  // the interpreter build: specialised for this shape unless asked otherwise
+  KParams sel;
+  memset(&sel, 0, sizeof sel);
+  sel.nq = h->shape.nq;
+  sel.nkv = h->shape.nkv;
+  sel.d = h->shape.d;
+  sel.Rh = p.Rh;
+  sel.Ro = p.Ro;
+  sel.Rd = p.Rd;
+  int variant = 0;
+  const void *kernel = interp_kernel_for(sel, o.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC, &variant);
   int per_sm = 0;
-  cudaError_t e = occupancy_interp(nb, smem, &per_sm);
+  cudaError_t e = interp_prepare(kernel, smem, &per_sm);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MK_ERR_CUDA;
@@ -407,8 +426,9 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   KParams &k = h->kp;
   memset(&k, 0, sizeof k);
   int rc;
-  float *part_o, *part_ml, *arg_val;
-  int *arg_idx, *q_off, *q_len;
+  float *part_o;
+  unsigned long long *part_ml, *arg_val, *arg_idx;
+  int *q_off, *q_len;
   unsigned *ctr;
   Instr *instrs;
   unsigned long long *trace = nullptr;
@@ -416,6 +436,13 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   if ((rc = dalloc(h->plan_allocs, &part_ml, (size_t)s.L * B * s.nq * p.S * 2))) return rc;
   if ((rc = dalloc(h->plan_allocs, &arg_val, (size_t)B * p.n_lm))) return rc;
   if ((rc = dalloc(h->plan_allocs, &arg_idx, (size_t)B * p.n_lm))) return rc;
+  // the handle's tagged buffers may hold tags of earlier steps: the step
+  // number restarts at 1, so clear them (the plan's own buffers are new)
+  for (auto &tb : h->tagged)
+    if ((e = cudaMemset(tb.first, 0, tb.second)) != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
   if ((rc = dalloc(h->plan_allocs, &ctr, (size_t)p.n_counters))) return rc;
   if ((rc = dalloc(h->plan_allocs, &instrs, p.instrs.size(), false))) return rc;
   if ((rc = dalloc(h->plan_allocs, &q_off, (size_t)num_ctas, false))) return rc;
@@ -462,6 +489,7 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   k.kv_ls = k.kv_bs * h->cfg.max_batch;
   k.rope = h->d_rope;
   k.qbuf = h->qbuf;
+  k.kvcur = h->kvcur;
   k.part_o = part_o;
   k.part_ml = part_ml;
   k.obuf = h->obuf;
@@ -502,6 +530,8 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   h->smem = smem;
   h->grid = num_ctas;
   h->nb = nb;
+  h->kernel = kernel;
+  h->kernel_variant = variant;
   h->planned = true;
   return MK_OK;
 }
@@ -512,7 +542,7 @@ static int launch_per_op(mk_handle *h, KParams k, cudaStream_t st) {
     // skip the empty per-layer stage slot of the LM head
     k.stage_filter = sidx;
     k.mode = (h->kp.mode & MODE_TRACE) | MODE_NO_WAIT | (sidx == n_stage - 1 ? MODE_FINAL_LAUNCH : 0u);
-    cudaError_t e = launch_interp(k, h->nb, h->grid, h->smem, st, false);
+    cudaError_t e = launch_interp(h->kernel, k, h->grid, h->smem, st, false);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return cuda_code(e);
@@ -531,9 +561,9 @@ extern "C" int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t
   k.positions = positions;
   k.logits = logits_out;
   k.next_tokens = next_tokens_out;
-  if (h->opts.exec_mode == MK_EXEC_MEGAKERNEL) {
+  if (h->opts.exec_mode == MK_EXEC_MEGAKERNEL || h->opts.exec_mode == MK_EXEC_MEGAKERNEL_GENERIC) {
     k.mode |= MODE_FINAL_LAUNCH;
-    cudaError_t e = launch_interp(k, h->nb, h->grid, h->smem, st, true);
+    cudaError_t e = launch_interp(h->kernel, k, h->grid, h->smem, st, true);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return cuda_code(e);
@@ -594,8 +624,16 @@ extern "C" int mk_get_status(mk_handle *h, void *stream) {
   // numbering again
   e = cudaMemset(h->status, 0, sizeof(int) * kStatusWords);
   if (e == cudaSuccess && h->planned) {
+    // restart the step numbering; every tagged word must then look stale
     const unsigned one = 1;
     e = cudaMemset(h->kp.ctr, 0, sizeof(unsigned) * h->plan.n_counters);
+    for (auto &tb : h->tagged)
+      if (e == cudaSuccess) e = cudaMemset(tb.first, 0, tb.second);
+    const size_t S = (size_t)h->plan.S, L = h->shape.L, B = h->kp.B, nq = h->shape.nq, d = h->shape.d;
+    if (e == cudaSuccess) e = cudaMemset(h->kp.part_o, 0, sizeof(float) * L * B * nq * S * d);
+    if (e == cudaSuccess) e = cudaMemset(h->kp.part_ml, 0, 8 * L * B * nq * S * 2);
+    if (e == cudaSuccess) e = cudaMemset(h->kp.arg_val, 0, 8 * B * h->plan.n_lm);
+    if (e == cudaSuccess) e = cudaMemset(h->kp.arg_idx, 0, 8 * B * h->plan.n_lm);
     if (e == cudaSuccess) e = cudaMemcpy(h->ctr_epoch, &one, sizeof one, cudaMemcpyHostToDevice);
   }
   if (e != cudaSuccess) {
@@ -633,6 +671,8 @@ extern "C" int mk_get_plan_info(const mk_handle *h, mk_plan_info *info) {
   for (int l : h->plan.q_len) mx = std::max(mx, l);
   info->max_queue_len = mx;
   info->weight_bytes_per_step = h->plan.weight_bytes;
+  info->kernel_variant = h->kernel_variant;
+  info->reserved = 0;
   return MK_OK;
 }
 

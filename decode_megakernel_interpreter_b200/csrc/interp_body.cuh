@@ -1,0 +1,1680 @@
+// The decode interpreter: one persistent CTA per SM runs a queue of
+// instructions (fetch -> wait for dependency counters -> stage the input
+// vector -> stream weight pages -> compute -> store -> signal), after the
+// on-GPU interpreter of the "Hazy megakernel summary" page (section 四(二))
+// and the task loop of the "Mirage Persistent Kernel" article (Part 2).
+//
+// Warp roles (this build's design for sm_100a):
+//   warp 0, lane 0  loader: walks the same queue ahead of the compute warps and
+//                   streams every weight / KV page of every instruction into a
+//                   ring of 16 KiB shared-memory pages with 1-D bulk copies
+//                   (cp.async.bulk, mbarrier completion).  Weights never depend
+//                   on activations, so the next instructions' pages load while
+//                   the current one is still waiting or storing (the paged
+//                   shared memory of the same section, whose freed pages go to
+//                   the next instruction).  Optionally it also runs an L2
+//                   prefetch cursor further ahead (cp.async.bulk.prefetch.L2).
+//   warps 1..8      compute: CUDA-core fp32 FMA matrix-vector products over
+//                   bf16 pages (batch 1 is a matrix-vector product; tensor
+//                   cores do not help there, section 五(二)), warp-shuffle
+//                   reductions, fused epilogues, and the counter protocol.
+// Synchronisation between instructions: an array of counters in global memory
+// (section 四(二) "同步"): a producer adds 1 (release) when done, a consumer
+// waits (acquire) until the counter reaches epoch * producers.  Counters are
+// never reset; `epoch` is the step number.  Every wait is bounded by a
+// global-timer deadline; a timeout records MK_ERR_TIMEOUT and makes every CTA
+// leave cleanly.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mk.h"
+#include "mk_internal.h"
+
+namespace mk {
+// Internal linkage: every translation unit that includes this file (the
+// generic build and each shape-specialised build) gets its own copy.
+namespace {
+typedef unsigned long long llw;
+
+// ============================================================== PTX helpers
+namespace px {
+
+__device__ __forceinline__ uint32_t sa(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(sa(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sa(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(sa(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(sa(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(sa(dst)),
+      "l"(src), "r"(bytes), "r"(sa(bar)), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned *p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ int ld_volatile(const int *p) { return *(const volatile int *)p; }
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void red_relaxed_add(unsigned *p, unsigned v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned atom_relaxed_add(unsigned *p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+// Tagged activation words: (step tag << 32 | value bits), stored and loaded as
+// single-copy-atomic 64-bit accesses, so a reader can tell this step's value
+// from a stale one without any fence between the writer's data and a flag.
+__device__ __forceinline__ void st_ll(llw *a, float v, uint32_t tag) {
+  const llw w = ((llw)tag << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(w) : "memory");
+}
+__device__ __forceinline__ llw ld_ll(const llw *a) {
+  llw w;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(a));
+  return w;
+}
+__device__ __forceinline__ void ld_ll2(const llw *a, llw &x, llw &y) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(x), "=l"(y) : "l"(a));
+}
+__device__ __forceinline__ bool ll_fresh(llw w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
+__device__ __forceinline__ float ll_f(llw w) { return __uint_as_float((uint32_t)w); }
+// Tagged fp32 activations (the bulk of the exchanged data): the value rounded
+// to 21 significant bits, its two lowest mantissa bits replaced by the step
+// number mod 4.  Every such word is rewritten every step, so the only stale
+// value a reader can meet is the previous step's (or zero-filled memory
+// before the first step): a 2-bit tag tells them apart, and 4-byte words keep
+// the traffic and registers of plain fp32.
+__device__ __forceinline__ uint32_t tf_pack(float v, uint32_t tag) {
+  return ((__float_as_uint(v) + 2u) & ~3u) | (tag & 3u);
+}
+__device__ __forceinline__ void st_tf(float *a, float v, uint32_t tag) {
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(a), "r"(tf_pack(v, tag)) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_tf(const float *a) {
+  uint32_t u;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(u) : "l"(a));
+  return u;
+}
+__device__ __forceinline__ uint4 ld_tf4(const float *a) {
+  uint4 u;
+  asm volatile("ld.relaxed.gpu.global.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+               : "l"(a));
+  return u;
+}
+__device__ __forceinline__ uint2 ld_tf2(const float *a) {
+  uint2 u;
+  asm volatile("ld.relaxed.gpu.global.v2.b32 {%0, %1}, [%2];" : "=r"(u.x), "=r"(u.y) : "l"(a));
+  return u;
+}
+// Named barrier over the 256 compute threads, returning the OR of `pred`
+// over them (a uniform decision for every compute thread).
+__device__ __forceinline__ bool cbar_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " barrier.cta.red.or.pred q, 2, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "n"(kComputeThreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void cbar() {
+  asm volatile("barrier.cta.sync 1, %0;" ::"n"(kComputeThreads) : "memory");
+}
+__device__ __forceinline__ float4 ldcg4(const float *p) { return __ldcg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ float ldcg(const float *p) { return __ldcg(p); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+}  // namespace px
+
+// ============================================================== shared state
+struct Shared {
+  int abort;       // this CTA saw a failed wait
+  int flag;        // broadcast slot
+  int pad[2];
+  float2 rope[64]; // (cos, sin) of sequence 0's position
+  int pos[kMaxBatch], tok[kMaxBatch];  // this step's (clamped) positions and token ids
+  int stat_cwait;  // trace mode: pages a compute warp found not yet landed (this instruction)
+  int stat_llretry;  // tagged-load groups re-issued because a word was stale (this instruction)
+  uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
+  float red[kComputeWarps][kMaxBatch];
+  float argv[kComputeWarps][kMaxBatch];
+  int argi[kComputeWarps][kMaxBatch];
+};
+
+// ============================================================== small helpers
+
+__device__ void record_error(const KParams &p, int code, int a, int b, int c, int d) {
+  if (atomicCAS(p.status, 0, code) == 0) {
+    p.status[2] = a;
+    p.status[3] = b;
+    p.status[4] = c;
+    p.status[5] = d;
+    p.status[6] = blockIdx.x;
+  }
+  if (code == MK_ERR_TIMEOUT) atomicExch(p.status + 1, 1);
+}
+
+__device__ __forceinline__ bool global_abort(const KParams &p) { return px::ld_volatile(p.status + 1) != 0; }
+
+// positions and token ids are read once per launch into shared memory
+__device__ __forceinline__ int read_pos(const Shared *sh, int b) { return sh->pos[b]; }
+__device__ __forceinline__ int read_tok(const Shared *sh, int b) { return sh->tok[b]; }
+
+// Tagged loads are consumed in groups: every word of a group is loaded, the
+// values are used as loaded, and `ok` collects whether each word carried this
+// step's tag.  A group with a stale word is re-issued as a whole (one round
+// trip per retry, not one per stale word), bounded like every other wait.
+__device__ __forceinline__ float ll_chk(llw w, uint32_t tag, bool &ok) {
+  ok &= px::ll_fresh(w, tag);
+  return px::ll_f(w);
+}
+__device__ __forceinline__ float tf_chk(uint32_t u, uint32_t tag, bool &ok) {
+  ok &= ((u ^ tag) & 3u) == 0;
+  return __uint_as_float(u & ~3u);
+}
+__device__ __forceinline__ float4 tf_chk4(uint4 u, uint32_t tag, bool &ok) {
+  ok &= (((u.x ^ tag) | (u.y ^ tag) | (u.z ^ tag) | (u.w ^ tag)) & 3u) == 0;
+  return make_float4(__uint_as_float(u.x & ~3u), __uint_as_float(u.y & ~3u), __uint_as_float(u.z & ~3u),
+                     __uint_as_float(u.w & ~3u));
+}
+__device__ __noinline__ bool ll_give_up(const KParams *p, Shared *sh, uint64_t t0, int where) {
+  if (px::ld_volatile(&sh->abort) || global_abort(*p)) return true;
+  if (px::gtimer() - t0 > (uint64_t)p->timeout_ns) {
+    record_error(*p, MK_ERR_TIMEOUT, -3, where, 0, 0);
+    sh->abort = 1;
+    return true;
+  }
+  return false;
+}
+// Called after a group came back with a stale word: true = re-issue it,
+// false = give up (timeout or abort; the CTA is aborting, values are unused).
+struct LLRetry {
+  unsigned n = 0;
+  uint64_t t0 = 0;
+};
+__device__ __forceinline__ bool ll_retry(const KParams &p, Shared *sh, LLRetry &r, int where) {
+  if (r.n++ == 0) {
+    r.t0 = px::gtimer();
+    atomicAdd(&sh->stat_llretry, 1);
+  } else if ((r.n & 7u) == 0 && ll_give_up(&p, sh, r.t0, where)) {
+    return false;
+  }
+  return true;
+}
+
+// Wait until counter idx reaches target; one thread.  false on timeout/abort.
+__device__ bool wait_counter(const KParams &p, unsigned idx, unsigned target, int seq) {
+  const unsigned *c = p.ctr + idx;
+  if ((int)(px::ld_relaxed(c) - target) >= 0) return true;
+  const uint64_t t0 = px::gtimer();
+  for (unsigned it = 1;; ++it) {
+    unsigned v = px::ld_relaxed(c);
+    if ((int)(v - target) >= 0) return true;
+    if ((it & 31u) == 0) {
+      if (global_abort(p)) return false;
+      if (px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
+        record_error(p, MK_ERR_TIMEOUT, seq, (int)idx, (int)v, (int)target);
+        return false;
+      }
+    }
+  }
+}
+
+// Wait for an mbarrier phase; bounded, abort-aware.  Any thread.
+__device__ bool wait_bar(const KParams &p, Shared *sh, uint64_t *bar, uint32_t parity, int what) {
+  if (px::mbar_test(bar, parity)) return true;
+  const uint64_t t0 = px::gtimer();
+  for (unsigned it = 1;; ++it) {
+    if (px::mbar_test(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (px::ld_volatile(&sh->abort) || global_abort(p)) return false;
+      if (px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
+        record_error(p, MK_ERR_TIMEOUT, -1, what, (int)parity, 0);
+        return false;
+      }
+    }
+  }
+}
+
+// Attention split geometry of sequence b: positions [start, end) of split s
+// (of S), the cached prefix [start, pref_end) that the loader streams, and
+// whether the current position belongs to this split.
+struct SplitRange {
+  int pos, start, end, pref_end;
+  bool has_cur;
+};
+__device__ __forceinline__ SplitRange split_range(const KParams &p, const Shared *sh, int b, int s) {
+  SplitRange r;
+  r.pos = read_pos(sh, b);
+  int n = r.pos + 1;
+  int chunk = (n + p.S - 1) / p.S;
+  r.start = min(n, s * chunk);
+  r.end = min(n, r.start + chunk);
+  r.pref_end = min(r.end, r.pos);
+  r.has_cur = r.start <= r.pos && r.pos < r.end;
+  return r;
+}
+__device__ __forceinline__ int attn_ppp(const KParams &p) { return kPageBytes / (4 * p.d); }  // positions per page
+
+__device__ __forceinline__ bool selected(const KParams &p, const Instr &I) {
+  if (p.stage_filter < 0) return true;
+  int st = I.op == OP_LMHEAD ? p.L * kStagesPerLayer : I.layer * kStagesPerLayer + (I.op - 1);
+  return st == p.stage_filter;
+}
+
+// The pages of the packed layout, gathered from the caller's weights in their
+// own layout (several smaller bulk copies per page instead of one): the QKV page
+// of rotation pairs is two row runs, a gate/up page is a run of gate rows and
+// a run of up rows, a down page is Rd row segments of one K piece.  The page
+// contents are identical, so the compute side is unchanged.
+__device__ __forceinline__ void issue_page_raw(const KParams &p, const Instr &I, int t, uint8_t *dst,
+                                               uint64_t *bar, uint64_t pol_w, uint64_t pol_kv, bool prefetch_only) {
+  (void)pol_kv;
+  if (I.op == OP_OPROJ) {
+    const uint16_t *src = p.layers_raw[I.layer].wo + (size_t)(I.a + t) * kPageElems;
+    if (prefetch_only) {
+      px::bulk_prefetch_l2(src, kPageBytes);
+      return;
+    }
+    px::mbar_expect_tx(bar, kPageBytes);
+    px::bulk_g2s(dst, src, kPageBytes, bar, pol_w);
+    return;
+  }
+  const LayerRaw &W = p.layers_raw[I.layer];
+  const int j = I.a + t;
+  if (!prefetch_only) px::mbar_expect_tx(bar, kPageBytes);
+  auto copy = [&](const uint16_t *src, uint32_t off, uint32_t bytes) {
+    if (prefetch_only)
+      px::bulk_prefetch_l2(src, bytes);
+    else
+      px::bulk_g2s(dst + off, src, bytes, bar, pol_w);
+  };
+  if (I.op == OP_QKV) {
+    const int half = p.Rh / 2, pph = p.d / p.Rh;
+    const int head = j / pph, jj = j % pph;
+    const uint16_t *base;
+    int hh;
+    if (head < p.nq) {
+      base = W.wq;
+      hh = head;
+    } else if (head < p.nq + p.nkv) {
+      base = W.wk;
+      hh = head - p.nq;
+    } else {
+      base = W.wv;
+      hh = head - p.nq - p.nkv;
+    }
+    const uint32_t run = (uint32_t)half * p.H * 2;
+    copy(base + ((size_t)hh * p.d + jj * half) * p.H, 0, run);
+    copy(base + ((size_t)hh * p.d + p.d / 2 + jj * half) * p.H, run, run);
+  } else if (I.op == OP_GATEUP) {
+    const int half = p.Rh / 2;
+    const uint32_t run = (uint32_t)half * p.H * 2;
+    copy(W.wg + (size_t)j * half * p.H, 0, run);
+    copy(W.wu + (size_t)j * half * p.H, run, run);
+  } else {
+    const uint32_t seg = (uint32_t)p.KCd * 2;
+    for (int r = 0; r < p.Rd; ++r)
+      copy(W.wd + (size_t)(j * p.Rd + r) * p.F + (size_t)I.c * p.KCd, r * seg, seg);
+  }
+}
+
+// Instruction iterator shared by the loader and the compute warps.  Static
+// mode: the CTA's own queue.  (The dynamic mode hands instructions from the
+// loader to the compute warps through a small shared-memory FIFO.)
+struct Queue {
+  const Instr *base;
+  int len;
+};
+
+// ============================================================== loader
+// Source of every page of one instruction: page t is one contiguous copy of
+// bytes(t) at a + t * stride (and for KV pages a second one at b, into the
+// page's second half).  Computed once per instruction.
+struct PageSrc {
+  const uint16_t *a, *b;
+  size_t stride;            // elements between consecutive pages' sources
+  uint32_t bytes, last;     // bytes per copy; of the last page's copies
+  int npg;
+};
+__device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, const Instr &I) {
+  PageSrc s;
+  s.b = nullptr;
+  s.stride = kPageElems;
+  s.bytes = s.last = kPageBytes;
+  s.npg = (int)I.b;
+  switch (I.op) {
+    case OP_QKV: s.a = p.layers[I.layer].wqkv + (size_t)I.a * kPageElems; break;
+    case OP_OPROJ: s.a = p.layers[I.layer].wo + (size_t)I.a * kPageElems; break;
+    case OP_GATEUP: s.a = p.layers[I.layer].wgu + (size_t)I.a * kPageElems; break;
+    case OP_DOWN: s.a = p.layers[I.layer].wd + ((size_t)I.c * (p.H / p.Rd) + I.a) * kPageElems; break;
+    case OP_LMHEAD: {
+      s.a = p.lm_head + (size_t)I.a * p.Rh * p.H;
+      const int r_last = (int)(I.a + I.b - 1) * p.Rh;
+      s.last = (uint32_t)min(p.Rh, p.V - r_last) * p.H * 2;
+      break;
+    }
+    case OP_ATTN: {
+      const SplitRange r = split_range(p, sh, I.c, I.b);
+      const int ppp = attn_ppp(p), n = r.pref_end - r.start;
+      s.npg = n > 0 ? (n + ppp - 1) / ppp : 0;
+      const size_t off = (size_t)I.layer * p.kv_ls + (size_t)I.c * p.kv_bs + (size_t)I.a * p.kv_hs + (size_t)r.start * p.d;
+      s.a = p.kc + off;
+      s.b = p.vc + off;
+      s.stride = (size_t)ppp * p.d;
+      s.bytes = (uint32_t)ppp * p.d * 2;
+      s.last = s.npg > 0 ? (uint32_t)(n - (s.npg - 1) * ppp) * p.d * 2 : 0;
+      break;
+    }
+    default: s.a = nullptr; s.npg = 0; break;
+  }
+  return s;
+}
+
+// One loader lane streams the pages g with g % nl == li of every instruction
+// of its CTA's queue into the ring (several loaders overlap the issue
+// latency of the bulk copies, which is long for a single thread).
+template <bool RAW>
+__device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_t *full, uint64_t *empty,
+                           Queue q, volatile int *dyn_fifo, volatile int *dyn_tail, volatile int *dyn_head,
+                           unsigned epoch, int li, int nl) {
+  const uint64_t pol_w = px::policy_evict_first();
+  const uint64_t pol_kv = px::policy_evict_last();
+  const uint32_t NP = (uint32_t)p.num_pages;
+  const uint32_t cap = (uint32_t)p.max_inflight;
+  const bool trace = (p.mode & MODE_TRACE) != 0;
+  uint32_t g = 0, last_issued = 0;
+  bool ok = true, any = false;
+  const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
+  const unsigned dyn_base = dyn ? (epoch - 1u) * (unsigned)(p.n_instr + gridDim.x) : 0u;
+  int claimed = 0;
+  for (int qi = 0; ok; ++qi) {
+    Instr I;
+    if (dyn) {
+      // claim the next instruction of the global queue; publish it to the compute warps
+      unsigned k = atomicAdd(p.ctr + p.dyn_head, 1u) - dyn_base;
+      int slot = claimed & 31;
+      const uint64_t t0 = px::gtimer();
+      while (claimed - *dyn_head >= 32) {  // FIFO space (bounded)
+        if (px::ld_volatile(&sh->abort) || global_abort(p) || px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) break;
+      dyn_fifo[slot] = k < (unsigned)p.n_instr ? (int)k : -1;
+      __threadfence_block();
+      *dyn_tail = ++claimed;
+      if (k >= (unsigned)p.n_instr) break;
+      I = p.instrs[k];
+    } else {
+      if (qi >= q.len) break;
+      I = q.base[qi];
+      if (!selected(p, I)) continue;
+    }
+    unsigned long long *ltr = (trace && li == 0) ? p.trace + (size_t)I.seq * MK_TRACE_WORDS : nullptr;
+    if (ltr) ltr[5] = px::gtimer();
+    unsigned lwait = 0;
+    const PageSrc ps = page_src(p, sh, I);
+    const uint32_t g0 = g;
+    g += (uint32_t)ps.npg;
+    // this loader's pages of the instruction
+    for (uint32_t gg = g0 + (uint32_t)((li - (int)(g0 % nl) + nl) % nl); gg < g; gg += nl) {
+      const int t = (int)(gg - g0);
+      const uint32_t slot = gg % NP;
+      const uint32_t ph = (gg / NP) & 1u;
+      if (gg >= NP) {
+        if (ltr && !px::mbar_test(&empty[slot], ph ^ 1u)) ++lwait;
+        if (!wait_bar(p, sh, &empty[slot], ph ^ 1u, 1)) {
+          ok = false;
+          break;
+        }
+      }
+      // keep at most `cap` pages in flight: more only queues in the memory
+      // system and delays every other access of this SM
+      if (cap > 0 && gg >= cap) {
+        const uint32_t k = gg - cap;
+        if (!wait_bar(p, sh, &full[k % NP], (k / NP) & 1u, 3)) {
+          ok = false;
+          break;
+        }
+      }
+      uint8_t *dst = pages + (size_t)slot * kPageBytes;
+      sh->slot_last[slot] = gg + 1;
+      if constexpr (RAW) {
+        if (I.op == OP_QKV || I.op == OP_GATEUP || I.op == OP_DOWN || I.op == OP_OPROJ) {
+          issue_page_raw(p, I, t, dst, &full[slot], pol_w, pol_kv, false);
+          any = true;
+          last_issued = gg;
+          continue;
+        }
+      }
+      const uint32_t bytes = (t == ps.npg - 1) ? ps.last : ps.bytes;
+      if (ps.b) {
+        px::mbar_expect_tx(&full[slot], 2 * bytes);
+        px::bulk_g2s(dst, ps.a + (size_t)t * ps.stride, bytes, &full[slot], pol_kv);
+        px::bulk_g2s(dst + kPageBytes / 2, ps.b + (size_t)t * ps.stride, bytes, &full[slot], pol_kv);
+      } else {
+        px::mbar_expect_tx(&full[slot], bytes);
+        px::bulk_g2s(dst, ps.a + (size_t)t * ps.stride, bytes, &full[slot], pol_w);
+      }
+      any = true;
+      last_issued = gg;
+    }
+    if (ltr) {
+      ltr[6] = px::gtimer();
+      ltr[9] = lwait;
+    }
+    if (!ok) {
+      g = g0;  // not every page of this instruction was issued; drain by last_issued
+      break;
+    }
+    if (px::ld_volatile(&sh->abort) || global_abort(p)) ok = false;
+  }
+  if (dyn && ok == false) {
+    // make sure the compute warps see the end of the queue
+    dyn_fifo[claimed & 31] = -1;
+    __threadfence_block();
+    *dyn_tail = claimed + 1;
+  }
+  (void)any;
+  (void)last_issued;
+}
+
+// ============================================================== compute
+struct CCtx {
+  const KParams &p;
+  Shared *sh;
+  uint8_t *pages;
+  float *act;     // staging region (input vector(s), attention scratch)
+  int act_stride; // floats per sequence in the staging region
+  uint64_t *full, *empty;
+  unsigned epoch;
+  int cw, lane, ctid;
+  uint32_t g;     // page sequence number (same as the loader's)
+  unsigned long long *tr;  // this instruction's trace record (or null)
+};
+
+// Register-resident view of the page ring (copied out of the context once per
+// instruction so that no loop reloads it from memory after a barrier or an
+// mbarrier poll).
+struct Ring {
+  uint8_t *pages;
+  uint64_t *full, *empty;
+  Shared *sh;
+  uint32_t np;
+};
+__device__ __forceinline__ Ring ring_of(const CCtx &c) {
+  return Ring{c.pages, c.full, c.empty, c.sh, (uint32_t)c.p.num_pages};
+}
+// Wait for ring page g (every compute warp calls this for pages it reads).
+// A parity test only tells the last two phases apart, so first make sure the
+// slot's previous page (g - np, possibly another warp's) has been released:
+// then its full barrier is in page g's phase (pending or complete) and the
+// parity test is unambiguous.  (The previous use of the empty barrier, page
+// g - 2np, belongs to this same warp because 2np is a multiple of the warp
+// count, so that test is unambiguous too.)
+__device__ __forceinline__ bool ring_wait(const KParams &p, const Ring &r, uint32_t g) {
+  const uint32_t slot = g % r.np;
+  const uint32_t ph = (g / r.np) & 1u;
+  if (g >= r.np && !px::mbar_test(&r.empty[slot], ph ^ 1u)) {
+    if (px::ld_volatile(&r.sh->abort)) return false;
+    if (!wait_bar(p, r.sh, &r.empty[slot], ph ^ 1u, 4)) {
+      r.sh->abort = 1;
+      return false;
+    }
+  }
+  if (px::mbar_test(&r.full[slot], ph)) return true;  // fast path: already landed
+  atomicAdd(&r.sh->stat_cwait, 1);
+  if (px::ld_volatile(&r.sh->abort)) return false;
+  if (!wait_bar(p, r.sh, &r.full[slot], ph, 0)) {
+    r.sh->abort = 1;
+    return false;
+  }
+  return true;
+}
+__device__ __forceinline__ const uint8_t *ring_page(const Ring &r, uint32_t g) {
+  return r.pages + (size_t)(g % r.np) * kPageBytes;
+}
+__device__ __forceinline__ void ring_release(const Ring &r, uint32_t g, uint32_t count) {
+  px::mbar_arrive(&r.empty[g % r.np], count);
+}
+__device__ __forceinline__ bool page_ready(CCtx &c, uint32_t g) { return ring_wait(c.p, ring_of(c), g); }
+__device__ __forceinline__ const uint8_t *page_ptr(CCtx &c, uint32_t g) { return ring_page(ring_of(c), g); }
+__device__ __forceinline__ void page_release(CCtx &c, uint32_t g, uint32_t count) {
+  ring_release(ring_of(c), g, count);
+}
+
+// Staging layout of an input vector of length K (fp32): element e of 8-chunk
+// ch = e / 8 lives at float4 slot ch (elements 0..3 of the chunk) or at
+// K/8 + ch (elements 4..7), so lane-consecutive chunks are bank-conflict free.
+__device__ __forceinline__ int stage_slot4(int e4, int K) { return (e4 & 1) * (K / 8) + (e4 >> 1); }
+
+// x_in of layer l (the residual stream entering layer l) for elements
+// 4*e4 .. 4*e4+3 of sequence b: the embedding for l == 0, else xres[l-1] +
+// the down-projection pieces of layer l-1 (fixed order).  Tagged loads: all
+// issued before any is checked.
+__device__ __forceinline__ float4 layer_input4(const KParams &p, uint32_t tag, int l, int b, int tok, int e4,
+                                               bool &ok) {
+  if (l == 0) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2 *>(p.embed + (size_t)tok * p.H) + e4);
+    return make_float4(px::bf_lo(w.x), px::bf_hi(w.x), px::bf_lo(w.y), px::bf_hi(w.y));
+  }
+  const size_t BH = (size_t)p.B * p.H;
+  float4 x = tf_chk4(px::ld_tf4(p.xres + (size_t)(l - 1) * BH + (size_t)b * p.H + e4 * 4), tag, ok);
+  for (int k0 = 0; k0 < p.ndp; k0 += 4) {  // four pieces' loads in flight at a time
+    uint4 d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) d[k] = px::ld_tf4(p.dpart + ((size_t)(l - 1) * p.ndp + k0 + k) * BH + (size_t)b * p.H + e4 * 4);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) {
+        const float4 v = tf_chk4(d[k], tag, ok);
+        x.x += v.x;
+        x.y += v.y;
+        x.z += v.z;
+        x.w += v.w;
+      }
+  }
+  return x;
+}
+__device__ __forceinline__ float layer_input1(const KParams &p, uint32_t tag, int l, int b, int tok, int e,
+                                              bool &ok) {
+  if (l == 0) return px::bf16f(__ldg(p.embed + (size_t)tok * p.H + e));
+  const size_t BH = (size_t)p.B * p.H;
+  float x = tf_chk(px::ld_tf(p.xres + (size_t)(l - 1) * BH + (size_t)b * p.H + e), tag, ok);
+  for (int k0 = 0; k0 < p.ndp; k0 += 4) {
+    uint32_t d[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) d[k] = px::ld_tf(p.dpart + ((size_t)(l - 1) * p.ndp + k0 + k) * BH + (size_t)b * p.H + e);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (k0 + k < p.ndp) x += tf_chk(d[k], tag, ok);
+  }
+  return x;
+}
+__device__ __noinline__ float layer_input1_settled(const KParams &p, Shared *sh, uint32_t tag, int l, int b, int tok,
+                                                   int e) {
+  float x;
+  for (LLRetry r;;) {
+    bool ok = true;
+    x = layer_input1(p, tag, l, b, tok, e, ok);
+    if (ok || !ll_retry(p, sh, r, 1)) break;
+  }
+  return x;
+}
+
+// four consecutive tagged words as a float4
+__device__ __forceinline__ float4 ll_load4(uint32_t tag, const float *a, bool &ok) {
+  return tf_chk4(px::ld_tf4(a), tag, ok);
+}
+
+// Stage rms(x)*gamma for every sequence, x = layer_input(l) (l == L: final norm).
+// Contains two compute barriers.
+// IT = float4 loads per thread (H / 4 / 256, at least 1), fixed by the caller's
+// rows-per-page so that every load is issued before the first one is used.
+template <int NB, int IT>
+__device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only) {
+  const KParams &p = c.p;
+  const int H = p.H, n4 = H / 4;
+  float ss[NB];
+  uint2 gws[IT];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) ss[b] = 0.f;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if (b >= p.B) break;
+    const int tok = (l == 0 && !from_xres_only) ? read_tok(c.sh, b) : 0;
+    float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
+    float4 xs[IT];
+    for (LLRetry r;;) {
+      bool ok = true;
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int e4 = c.ctid + it * kComputeThreads;
+        if (e4 < n4) {
+          if (b == 0) gws[it] = __ldg(reinterpret_cast<const uint2 *>(gamma) + e4);  // with x: one round trip
+          xs[it] = from_xres_only ? ll_load4(c.epoch, p.xres + ((size_t)l * p.B + b) * H + e4 * 4, ok)
+                                  : layer_input4(p, c.epoch, l, b, tok, e4, ok);
+        }
+      }
+      if (ok || !ll_retry(p, c.sh, r, 2)) break;
+    }
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4) {
+        const float4 x = xs[it];
+        ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+        dst[stage_slot4(e4, H)] = x;
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    float v = px::warp_sum(ss[b]);
+    if (c.lane == 0) c.sh->red[c.cw][b] = v;
+  }
+  px::cbar();
+  float inv[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kComputeWarps; ++w) t += c.sh->red[w][b];
+    inv[b] = 1.0f / sqrtf(t / (float)H + p.eps);
+  }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if (b >= p.B) break;
+    float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 >= n4) break;
+      const uint2 gw = gws[it];
+      float4 x = dst[stage_slot4(e4, H)];
+      x.x = x.x * inv[b] * px::bf_lo(gw.x);
+      x.y = x.y * inv[b] * px::bf_hi(gw.x);
+      x.z = x.z * inv[b] * px::bf_lo(gw.y);
+      x.w = x.w * inv[b] * px::bf_hi(gw.y);
+      dst[stage_slot4(e4, H)] = x;
+    }
+  }
+  px::cbar();
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+}
+
+// Stage a plain fp32 vector slice src[b*src_stride .. + K) for each sequence.
+// With nrows > 0 (O projection, batch 1) also stage x_in(l) for output rows
+// row0 .. row0+nrows after the vector, loaded in the same round trip.
+template <int NB, int IT>
+__device__ void stage_copy(CCtx &c, const float *src, size_t src_stride, int K, int l = 0, int row0 = 0,
+                           int nrows = 0) {
+  const KParams &p = c.p;
+  const int n4 = K / 4;
+  float xr = 0.f;
+  const bool has_row = c.ctid < nrows;
+  const int tok0 = l == 0 ? read_tok(c.sh, 0) : 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if (b >= p.B) break;
+    float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
+    float4 vs[IT];
+    for (LLRetry r;;) {  // the row of x_in rides along with sequence 0's vector
+      bool ok = true;
+      if (b == 0 && has_row) xr = layer_input1(p, c.epoch, l, 0, tok0, row0 + c.ctid, ok);
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int e4 = c.ctid + it * kComputeThreads;
+        if (e4 < n4) vs[it] = ll_load4(c.epoch, src + (size_t)b * src_stride + e4 * 4, ok);
+      }
+      if (ok || !ll_retry(p, c.sh, r, 3)) break;
+    }
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4) dst[stage_slot4(e4, K)] = vs[it];
+    }
+  }
+  for (int r = c.ctid; r < nrows; r += kComputeThreads)
+    c.act[K + r] = (r == c.ctid) ? xr : layer_input1_settled(p, c.sh, c.epoch, l, 0, tok0, row0 + r);
+  px::cbar();
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+}
+
+// acc[b][r] = dot(page row r, staged vector b) for R rows of KC = 8192/R
+// columns; every lane ends with every result.
+template <int NB, int R>
+__device__ __forceinline__ void mv_page(const uint8_t *page, const float *act, int act_stride, int B, int lane,
+                                        float (&acc)[NB][R]) {
+  constexpr int KC = kPageElems / R;
+  constexpr int CH = KC / 8;  // 16-byte chunks per row
+  const uint4 *pg = reinterpret_cast<const uint4 *>(page);
+#pragma unroll
+  for (int b = 0; b < NB; ++b)
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[b][r] = 0.f;
+#pragma unroll(CH / 32 > 2 ? 2 : CH / 32)
+  for (int j = 0; j < CH / 32; ++j) {
+    const int ch = lane + 32 * j;
+    uint4 w[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) w[r] = pg[r * CH + ch];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= B) break;
+      const float4 *a = reinterpret_cast<const float4 *>(act + (size_t)b * act_stride);
+      const float4 a0 = a[ch], a1 = a[CH + ch];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float s = acc[b][r];
+        s = fmaf(px::bf_lo(w[r].x), a0.x, s);
+        s = fmaf(px::bf_hi(w[r].x), a0.y, s);
+        s = fmaf(px::bf_lo(w[r].y), a0.z, s);
+        s = fmaf(px::bf_hi(w[r].y), a0.w, s);
+        s = fmaf(px::bf_lo(w[r].z), a1.x, s);
+        s = fmaf(px::bf_hi(w[r].z), a1.y, s);
+        s = fmaf(px::bf_lo(w[r].w), a1.z, s);
+        s = fmaf(px::bf_hi(w[r].w), a1.w, s);
+        acc[b][r] = s;
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if (NB > 1 && b >= B) break;
+#pragma unroll
+    for (int r = 0; r < R; ++r) acc[b][r] = px::warp_sum(acc[b][r]);
+  }
+}
+
+// pick acc[idx] with a compile-time-unrolled select (no local memory)
+template <int R>
+__device__ __forceinline__ float pick(const float (&v)[R], int idx) {
+  float out = 0.f;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+    if (r == idx) out = v[r];
+  return out;
+}
+
+// float4 loads per compute thread to stage a K = 8192 / R vector
+template <int R>
+struct StageIt {
+  static constexpr int v = (8 / R) > 0 ? (8 / R) : 1;
+};
+
+// ---------------------------------------------------------------- matvec ops
+// Loop over the instruction's pages owned by this warp (page g -> warp g % 8).
+template <int NB, int R, class Epi>
+__device__ __forceinline__ void matvec_pages(CCtx &c, const Instr &I, Epi epi) {
+  const KParams &p = c.p;
+  const Ring rg = ring_of(c);
+  const uint32_t g0 = c.g;
+  const int np = (int)I.b, first = (int)I.a, cw = c.cw, lane = c.lane, B = p.B, stride = c.act_stride;
+  const float *act = c.act;
+  // this warp's pages: g = g0 + t with g % 8 == cw
+  int t = (int)((uint32_t)(cw - (int)(g0 % kComputeWarps) + kComputeWarps) % kComputeWarps);
+  for (; t < np; t += kComputeWarps) {
+    const uint32_t g = g0 + (uint32_t)t;
+    if (!ring_wait(p, rg, g)) break;
+    float acc[NB][R];
+    mv_page<NB, R>(ring_page(rg, g), act, stride, B, lane, acc);
+    __syncwarp();
+    if (lane == 0) ring_release(rg, g, kComputeWarps);
+    epi(first + t, acc);
+  }
+  c.g = g0 + (uint32_t)np;
+}
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer;
+  const int half = R / 2, pph = p.d / R, hd = p.d / 2;
+  const int pos0 = read_pos(c.sh, 0);
+  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].attn_norm, false);
+  const int nq = p.nq, nkv = p.nkv, d = p.d, lane = c.lane, Bn = p.B, kvdim = p.kvdim;
+  const uint32_t tag = c.epoch;
+  float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
+  float *const kvc = p.kvcur + (size_t)l * Bn * 2 * kvdim;
+  uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
+  const long long kv_bs = p.kv_bs, kv_hs = p.kv_hs;
+  const int qdim = p.qdim;
+  const float2 *rope_s = c.sh->rope;
+  const float2 *rope_g = p.rope;
+  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    const int head = j / pph, jj = j % pph;
+    if (lane >= half) return;
+    const int i = jj * half + lane;  // rotation pair index inside the head
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= Bn) break;
+      float u = pick<R>(acc[b], lane), w = pick<R>(acc[b], lane + half);
+      const int pos = NB == 1 ? pos0 : read_pos(c.sh, b);
+      if (head < nq + nkv) {
+        const float2 cs = NB == 1 ? rope_s[i] : __ldg(rope_g + (size_t)pos * hd + i);
+        const float u2 = u * cs.x - w * cs.y, w2 = u * cs.y + w * cs.x;
+        u = u2;
+        w = w2;
+      }
+      if (head < nq) {
+        float *q = qrow + (size_t)b * qdim + head * d;
+        px::st_tf(q + i, u, tag);
+        px::st_tf(q + i + hd, w, tag);
+      } else {
+        // the cache row (bf16) for later steps, and the rounded values for
+        // this step's attention as tagged words
+        const bool isk = head < nq + nkv;
+        const int gk = isk ? head - nq : head - nq - nkv;
+        uint16_t *dst = (isk ? kl : vl) + (size_t)b * kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
+        const uint16_t bu = px::f2bf(u), bw = px::f2bf(w);
+        dst[i] = bu;
+        dst[i + hd] = bw;
+        float *cur = kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + gk * d;
+        px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 21 bits
+        px::st_tf(cur + i + hd, px::bf16f(bw), tag);
+      }
+    }
+  });
+  return c.g;
+}
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_qkv(CCtx c, const Instr I) { return qkv_body<NB, R>(c, I); }
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t oproj_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer;
+  const int row0 = (int)I.a * R, nrows = NB == 1 ? (int)I.b * R : 0;
+  stage_copy<NB, StageIt<R>::v>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim, l, row0, nrows);
+  const int lane = c.lane, Bn = p.B, H = p.H;
+  const uint32_t tag = c.epoch;
+  const float *xrows = c.act + p.qdim - row0;
+  float *const xout = p.xres + (size_t)l * Bn * H;
+  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    if (lane >= R) return;
+    const int row = j * R + lane;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= Bn) break;
+      const float v = pick<R>(acc[b], lane);
+      const float xin =
+          NB == 1 ? xrows[row] : layer_input1_settled(p, c.sh, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row);
+      px::st_tf(xout + (size_t)b * H + row, xin + v, tag);
+    }
+  });
+  return c.g;
+}
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_oproj(CCtx c, const Instr I) { return oproj_body<NB, R>(c, I); }
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t gateup_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer;
+  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].ffn_norm, true);
+  const int half = R / 2, lane = c.lane, Bn = p.B, F = p.F;
+  const uint32_t tag = c.epoch;
+  float *const aout = p.actb + (size_t)l * Bn * F;
+  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    if (lane >= half) return;
+    const int row = j * half + lane;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= Bn) break;
+      const float gt = pick<R>(acc[b], lane), up = pick<R>(acc[b], lane + half);
+      const float silu = gt / (1.0f + expf(-gt));
+      px::st_tf(aout + (size_t)b * F + row, silu * up, tag);
+    }
+  });
+  return c.g;
+}
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_gateup(CCtx c, const Instr I) { return gateup_body<NB, R>(c, I); }
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t down_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, k = I.c;
+  stage_copy<NB, StageIt<R>::v>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
+  const int lane = c.lane, Bn = p.B, H = p.H;
+  const uint32_t tag = c.epoch;
+  float *const dout = p.dpart + ((size_t)l * p.ndp + k) * Bn * H;
+  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    if (lane >= R) return;
+    const int row = j * R + lane;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= Bn) break;
+      px::st_tf(dout + (size_t)b * H + row, pick<R>(acc[b], lane), tag);
+    }
+  });
+  return c.g;
+}
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_down(CCtx c, const Instr I) { return down_body<NB, R>(c, I); }
+
+__device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false);
+  float bv[NB];
+  int bi[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    bv[b] = -INFINITY;
+    bi[b] = 0x7fffffff;
+  }
+  const int lane = c.lane, Bn = p.B, V = p.V;
+  float *const logits = p.logits;
+  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    const int row = j * R + lane;
+    const bool valid = lane < R && row < V;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= Bn) break;
+      const float v = pick<R>(acc[b], lane);
+      if (valid) {
+        if (logits) logits[(size_t)b * V + row] = v;
+        if (arg_better(v, row, bv[b], bi[b])) {
+          bv[b] = v;
+          bi[b] = row;
+        }
+      }
+    }
+  });
+  // CTA-wide argmax of this instruction
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if (b >= p.B) break;
+    float v = bv[b];
+    int i = bi[b];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+      int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+      if (arg_better(v2, i2, v, i)) {
+        v = v2;
+        i = i2;
+      }
+    }
+    if (c.lane == 0) {
+      c.sh->argv[c.cw][b] = v;
+      c.sh->argi[c.cw][b] = i;
+    }
+  }
+  px::cbar();
+  if (c.ctid < p.B) {
+    const int b = c.ctid;
+    float v = -INFINITY;
+    int i = 0x7fffffff;
+    for (int w = 0; w < kComputeWarps; ++w)
+      if (arg_better(c.sh->argv[w][b], c.sh->argi[w][b], v, i)) {
+        v = c.sh->argv[w][b];
+        i = c.sh->argi[w][b];
+      }
+    px::st_ll(p.arg_val + (size_t)b * p.n_lm + I.c, v, c.epoch);
+    px::st_ll(p.arg_idx + (size_t)b * p.n_lm + I.c, __int_as_float(i), c.epoch);
+  }
+  px::cbar();
+  // the last LM instruction to finish merges every slot (all compute threads
+  // load a share of the slots at once, then a tree reduction); the slots are
+  // tagged words, so the ticket needs no fence
+  if (c.ctid == 0) {
+    const unsigned old = px::atom_relaxed_add(p.ctr + p.arg_ticket0, 1u);
+    c.sh->flag = (old == c.epoch * (unsigned)p.n_lm - 1u);
+  }
+  px::cbar();
+  if (c.sh->flag) {  // uniform: every compute thread reads the same flag
+    for (int b = 0; b < p.B; ++b) {
+      float v = -INFINITY;
+      int i = 0x7fffffff;
+      for (int s0 = c.ctid; s0 < p.n_lm; s0 += kComputeThreads) {
+        const llw *av = p.arg_val + (size_t)b * p.n_lm + s0, *ai = p.arg_idx + (size_t)b * p.n_lm + s0;
+        float sv;
+        int si;
+        for (LLRetry r;;) {
+          bool ok = true;
+          const llw wv = px::ld_ll(av), wi = px::ld_ll(ai);
+          sv = ll_chk(wv, c.epoch, ok);
+          si = __float_as_int(ll_chk(wi, c.epoch, ok));
+          if (ok || !ll_retry(p, c.sh, r, 4)) break;
+        }
+        if (arg_better(sv, si, v, i)) {
+          v = sv;
+          i = si;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+        const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+        if (arg_better(v2, i2, v, i)) {
+          v = v2;
+          i = i2;
+        }
+      }
+      if (c.lane == 0) {
+        c.sh->argv[c.cw][b] = v;
+        c.sh->argi[c.cw][b] = i;
+      }
+    }
+    px::cbar();
+    if (c.ctid < p.B) {
+      const int b = c.ctid;
+      float v = -INFINITY;
+      int i = 0x7fffffff;
+      for (int w = 0; w < kComputeWarps; ++w)
+        if (arg_better(c.sh->argv[w][b], c.sh->argi[w][b], v, i)) {
+          v = c.sh->argv[w][b];
+          i = c.sh->argi[w][b];
+        }
+      p.next_tokens[b] = (i == 0x7fffffff) ? 0 : i;
+    }
+  }
+  return c.g;
+}
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_lmhead(CCtx c, const Instr I) { return lmhead_body<NB, R>(c, I); }
+
+// ---------------------------------------------------------------- attention
+// One (sequence b, kv head g, split s) item: online softmax over the split's
+// cached positions (streamed through the ring, all compute warps per page,
+// a block of positions per warp), plus the current position (read from the
+// cache row this step's QKV instruction wrote).  Unnormalised partials
+// (o, max, sum) go to global memory; the last split to finish merges all
+// splits of the head group with log-sum-exp weights.
+template <int G, int DPL, int PB>
+__device__ __forceinline__ void load_row(const uint16_t *rowp, int lane, float (&f)[DPL]) {
+  if constexpr (DPL == 2) {
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(rowp + lane * 2);
+    f[0] = px::bf_lo(w);
+    f[1] = px::bf_hi(w);
+  } else {
+    const uint2 w = *reinterpret_cast<const uint2 *>(rowp + lane * 4);
+    f[0] = px::bf_lo(w.x);
+    f[1] = px::bf_hi(w.x);
+    f[2] = px::bf_lo(w.y);
+    f[3] = px::bf_hi(w.y);
+  }
+}
+
+// PB consecutive positions (rows of kb / vb, row stride D) for one warp, of
+// which the first `nvalid` are real.  G*PB <= 32 scores are reduced with a
+// transposed butterfly so that one lane ends with one score; the softmax
+// update is then one exp per lane.
+template <int G, int DPL, int PB>
+__device__ void attn_block(const float (&q)[G][DPL], const uint16_t *kb, const uint16_t *vb, int nvalid,
+                           int lane, float (&m)[G], float (&l)[G], float (&o)[G][DPL]) {
+  constexpr int D = DPL * 32;
+  constexpr int NV = G * PB;
+  static_assert(NV <= 32 && (NV & (NV - 1)) == 0, "block size");
+  float v[NV];
+#pragma unroll
+  for (int j = 0; j < PB; ++j) {
+    float kf[DPL];
+    if (j < nvalid) {
+      load_row<G, DPL, PB>(kb + j * D, lane, kf);
+    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) kf[i] = 0.f;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) s = fmaf(q[h][i], kf[i], s);
+      v[h * PB + j] = s;
+    }
+  }
+  // transposed reduction: afterwards the lane holds the full score of value
+  // index (lane >> SH), index = h * PB + j
+  int n = NV;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const int hn = n / 2;
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < (NV > 1 ? NV / 2 : 1); ++i) {
+        if (i < hn) {
+          const float send = up ? v[i] : v[i + hn];
+          const float keep = up ? v[i + hn] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      n = hn;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+  constexpr int LOGNV = (NV >= 32) ? 5 : (NV >= 16) ? 4 : (NV >= 8) ? 3 : (NV >= 4) ? 2 : (NV >= 2) ? 1 : 0;
+  constexpr int SH = 5 - LOGNV;
+  constexpr int GRP = 32 / G;  // lanes per head after the reduction
+  const int idx = lane >> SH;
+  const int myh = idx / PB, myj = idx % PB;
+  const float s = (myj < nvalid) ? v[0] : -INFINITY;
+  float bm = s;
+#pragma unroll
+  for (int off = GRP / 2; off >= 1; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+  float mh_old = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+    if (h == myh) mh_old = m[h];
+  const float mnew = fmaxf(mh_old, bm);
+  const float pr = (s == -INFINITY) ? 0.f : expf(s - mnew);
+  // 2^SH lanes hold each score: count one of them in the sum
+  float ps = (lane & ((1 << SH) - 1)) == 0 ? pr : 0.f;
+#pragma unroll
+  for (int off = GRP / 2; off >= 1; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float mn = __shfl_sync(0xffffffffu, mnew, h * GRP);
+    const float bs = __shfl_sync(0xffffffffu, ps, h * GRP);
+    const float corr = (m[h] == -INFINITY) ? 0.f : expf(m[h] - mn);
+    l[h] = l[h] * corr + bs;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) o[h][i] *= corr;
+    m[h] = mn;
+  }
+#pragma unroll
+  for (int j = 0; j < PB; ++j) {
+    if (j >= nvalid) break;
+    float vf[DPL];
+    load_row<G, DPL, PB>(vb + j * D, lane, vf);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float ph = __shfl_sync(0xffffffffu, pr, (h * PB + j) << SH);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) o[h][i] = fmaf(ph, vf[i], o[h][i]);
+    }
+  }
+}
+
+template <int G, int DPL>
+__device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  constexpr int D = DPL * 32;
+  constexpr int PPP = kPageBytes / (4 * D);
+  constexpr int PW = PPP / kComputeWarps;        // positions per warp per page
+  constexpr int PB = PW < 32 / G ? PW : 32 / G;  // positions per reduction block
+  const int l = I.layer, g = I.a, s = I.b, b = I.c;
+  const SplitRange r = split_range(p, c.sh, b, s);
+  const int npg = r.pref_end > r.start ? (r.pref_end - r.start + PPP - 1) / PPP : 0;
+  // q of the G heads of this group (pre-scaled by 1/sqrt(d)) and, for the
+  // split holding the current position, that position's K and V rows (this
+  // step's QKV wrote them as tagged words): one group of loads
+  const uint32_t tag = c.epoch;
+  const bool load_cur = r.has_cur && c.cw == 0;
+  const float *kcur = p.kvcur + (((size_t)l * p.B + b) * 2) * p.kvdim + (size_t)g * D;
+  const float *vcur = kcur + p.kvdim;
+  const float *qb = p.qbuf + ((size_t)l * p.B + b) * p.qdim + (size_t)g * G * D;
+  float q[G][DPL], ck[DPL], cv[DPL];
+  for (LLRetry rr;;) {
+    bool ok = true;
+    uint32_t wk[DPL], wv[DPL], wq[G][DPL];
+    if (load_cur) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        wk[i] = px::ld_tf(kcur + c.lane * DPL + i);
+        wv[i] = px::ld_tf(vcur + c.lane * DPL + i);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) wq[h][i] = px::ld_tf(qb + h * D + c.lane * DPL + i);
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) q[h][i] = tf_chk(wq[h][i], tag, ok) * p.attn_scale;
+    if (load_cur) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        ck[i] = tf_chk(wk[i], tag, ok);
+        cv[i] = tf_chk(wv[i], tag, ok);
+      }
+    }
+    if (ok || !ll_retry(p, c.sh, rr, 5)) break;
+  }
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+  float m[G], lsum[G], o[G][DPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m[h] = -INFINITY;
+    lsum[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
+  }
+  // scratch in the staging region: [warp][G][D + 2] floats, then the
+  // current position's K and V rows (bf16)
+  float *scr = c.act;
+  uint16_t *cur = reinterpret_cast<uint16_t *>(c.act + kComputeWarps * G * (D + 2));
+  if (load_cur) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      cur[c.lane * DPL + i] = px::f2bf(ck[i]);
+      cur[D + c.lane * DPL + i] = px::f2bf(cv[i]);
+    }
+  }
+  const Ring rg = ring_of(c);
+  const int cw = c.cw, lane = c.lane;
+  for (int t = 0; t < npg; ++t) {
+    const uint32_t gg = c.g + t;
+    if (!ring_wait(p, rg, gg)) break;
+    const uint8_t *pg = ring_page(rg, gg);
+    const int p0 = r.start + t * PPP;
+    const int cnt = min(PPP, r.pref_end - p0);
+#pragma unroll
+    for (int sb = 0; sb < PW / PB; ++sb) {
+      const int jb = cw * PW + sb * PB;
+      const int nvalid = max(0, min(PB, cnt - jb));
+      if (nvalid > 0)
+        attn_block<G, DPL, PB>(q, reinterpret_cast<const uint16_t *>(pg) + (size_t)jb * D,
+                               reinterpret_cast<const uint16_t *>(pg + kPageBytes / 2) + (size_t)jb * D, nvalid,
+                               lane, m, lsum, o);
+    }
+    __syncwarp();
+    if (lane == 0) ring_release(rg, gg, 1);
+  }
+  c.g += npg;
+  __syncwarp();
+  if (r.has_cur && c.cw == 0 && !c.sh->abort) {
+    // one valid position; the block reads PW rows, rows past the first are masked
+    attn_block<G, DPL, PB>(q, cur, cur + D, 1, c.lane, m, lsum, o);
+  }
+  // merge the warps
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float *w = scr + ((size_t)c.cw * G + h) * (D + 2);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) w[c.lane * DPL + i] = o[h][i];
+    if (c.lane == 0) {
+      w[D] = m[h];
+      w[D + 1] = lsum[h];
+    }
+  }
+  px::cbar();
+  const size_t hbase = ((size_t)l * p.B + b) * p.nq + (size_t)g * G;  // [l][b][head]
+  for (int e = c.ctid; e < G * D; e += kComputeThreads) {
+    const int h = e / D, dd = e % D;
+    float M = -INFINITY;
+    for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, scr[((size_t)w * G + h) * (D + 2) + D]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int w = 0; w < kComputeWarps; ++w) {
+        const float *ws = scr + ((size_t)w * G + h) * (D + 2);
+        const float mw = ws[D];
+        const float f = (mw == -INFINITY) ? 0.f : expf(mw - M);
+        L += f * ws[D + 1];
+        O += f * ws[dd];
+      }
+    }
+    px::st_tf(p.part_o + ((hbase + h) * p.S + s) * D + dd, O, tag);
+    if (dd == 0) {
+      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 0, M, tag);
+      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 1, L, tag);
+    }
+  }
+  px::cbar();
+  if (c.ctid == 0) {  // tagged partials: the ticket needs no fence
+    const unsigned t = p.attn_ticket0 + ((unsigned)l * p.B + b) * p.nkv + g;
+    const unsigned old = px::atom_relaxed_add(p.ctr + t, 1u);
+    c.sh->flag = (old == c.epoch * (unsigned)p.S - 1u);
+  }
+  px::cbar();
+  if (c.sh->flag) {  // uniform: the last split of the group merges all S splits
+    constexpr int NE = G * D;                            // outputs of the group
+    constexpr int EPT = (NE + kComputeThreads - 1) / kComputeThreads;
+    constexpr int SB = (64 / EPT) < 32 ? (64 / EPT) : 32;  // splits per load batch
+    const int S = p.S;
+    float *sml = scr;  // [G][S] (m, l) then (weight, -)
+    for (int i = c.ctid; i < G * S; i += kComputeThreads) {
+      const int h = i / S, sp = i % S;
+      const llw *a = p.part_ml + ((hbase + h) * S + sp) * 2;
+      for (LLRetry rr;;) {
+        bool ok = true;
+        llw w0, w1;
+        px::ld_ll2(a, w0, w1);
+        sml[2 * i] = ll_chk(w0, tag, ok);
+        sml[2 * i + 1] = ll_chk(w1, tag, ok);
+        if (ok || !ll_retry(p, c.sh, rr, 6)) break;
+      }
+    }
+    // the first batch of this thread's partial outputs, in flight with the table
+    uint32_t ov[EPT][SB];
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int idx = c.ctid + e * kComputeThreads;
+      const int h = idx / D, dd = idx % D;
+#pragma unroll
+      for (int j = 0; j < SB; ++j) ov[e][j] = (idx < NE && j < S) ? px::ld_tf(p.part_o + ((hbase + h) * S + j) * D + dd) : 0u;
+    }
+    px::cbar();
+    if (c.ctid < G) {  // per head: max, weights exp(m_s - M), and the total weight L
+      const int h = c.ctid;
+      float M = -INFINITY;
+      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, sml[2 * (h * S + sp)]);
+      float L = 0.f;
+      for (int sp = 0; sp < S; ++sp) {
+        const float ms = sml[2 * (h * S + sp)];
+        const float wgt = (ms == -INFINITY) ? 0.f : expf(ms - M);
+        L += wgt * sml[2 * (h * S + sp) + 1];
+        sml[2 * (h * S + sp)] = wgt;
+      }
+      c.sh->red[h % kComputeWarps][h / kComputeWarps] = L;
+    }
+    px::cbar();
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int idx = c.ctid + e * kComputeThreads;
+      if (idx >= NE) break;
+      const int h = idx / D, dd = idx % D;
+      float O = 0.f;
+      bool ok = true;
+#pragma unroll
+      for (int j = 0; j < SB; ++j)
+        if (j < S) O += sml[2 * (h * S + j)] * tf_chk(ov[e][j], tag, ok);
+      for (int s0 = ok ? SB : 0; s0 < S; s0 += SB) {  // further batches (S > SB), or all again
+        float Ob = 0.f;
+        for (LLRetry rr;;) {
+          bool okb = true;
+          uint32_t tmp[SB];
+#pragma unroll
+          for (int j = 0; j < SB; ++j)
+            tmp[j] = (s0 + j < S) ? px::ld_tf(p.part_o + ((hbase + h) * S + s0 + j) * D + dd) : 0u;
+          Ob = 0.f;
+#pragma unroll
+          for (int j = 0; j < SB; ++j)
+            if (s0 + j < S) Ob += sml[2 * (h * S + s0 + j)] * tf_chk(tmp[j], tag, okb);
+          if (okb || !ll_retry(p, c.sh, rr, 7)) break;
+        }
+        O = (s0 == 0) ? Ob : O + Ob;
+      }
+      const float L = c.sh->red[h % kComputeWarps][h / kComputeWarps];
+      px::st_tf(p.obuf + ((size_t)l * p.B + b) * p.qdim + (size_t)(g * G + h) * D + dd, O / L, tag);
+    }
+  }
+  return c.g;
+}
+template <int G, int DPL>
+__device__ __noinline__ uint32_t op_attn_t(CCtx c, const Instr I) { return attn_body<G, DPL>(c, I); }
+
+__device__ __forceinline__ uint32_t op_attn(const CCtx &c, const Instr &I) {
+  const int G = c.p.nq / c.p.nkv;
+  if (c.p.d == 64) {
+    switch (G) {
+      case 1: return op_attn_t<1, 2>(c, I);
+      case 2: return op_attn_t<2, 2>(c, I);
+      case 4: return op_attn_t<4, 2>(c, I);
+      default: return op_attn_t<8, 2>(c, I);
+    }
+  }
+  switch (G) {
+    case 1: return op_attn_t<1, 4>(c, I);
+    case 2: return op_attn_t<2, 4>(c, I);
+    case 4: return op_attn_t<4, 4>(c, I);
+    default: return op_attn_t<8, 4>(c, I);
+  }
+}
+
+// dispatch on the rows-per-page of the instruction's matrix
+#define MK_DISPATCH_R(fn, NB, R, c, I)            \
+  switch (R) {                                    \
+    case 2: c.g = fn<NB, 2>(c, I); break;         \
+    case 4: c.g = fn<NB, 4>(c, I); break;         \
+    case 8: c.g = fn<NB, 8>(c, I); break;         \
+    case 16: c.g = fn<NB, 16>(c, I); break;       \
+    default: c.g = fn<NB, 32>(c, I); break;       \
+  }
+
+__device__ __forceinline__ int &sh_stat(CCtx &c) { return c.sh->stat_cwait; }
+
+// Shape specialisation of the interpreter: rows per page of the QKV / gate-up /
+// LM-head pages (RH), of the output-projection pages (RO) and of the
+// down-projection pages (RD), the query heads per KV head (G) and head_dim / 32
+// (DPL).  With every value fixed, each op body is inlined into the interpreter
+// loop (no call, no spills across a call boundary); the shape-generic build
+// (all zero) reaches the bodies through calls selected at run time.
+template <int RH_, int RO_, int RD_, int G_, int DPL_>
+struct Spec {
+  static constexpr bool fixed = RH_ > 0;
+  static constexpr int RH = RH_, RO = RO_, RD = RD_, G = G_, DPL = DPL_;
+};
+using SpecGeneric = Spec<0, 0, 0, 0, 0>;
+
+template <int NB, class S>
+__device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile int *dyn_tail,
+                            volatile int *dyn_head) {
+  const KParams &p = c.p;
+  const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
+  const bool trace = (p.mode & MODE_TRACE) != 0;
+  for (int qi = 0;; ++qi) {
+    Instr I;
+    if (dyn) {
+      // next claimed instruction from the loader (bounded wait, thread 0)
+      if (c.ctid == 0) {
+        const uint64_t t0 = px::gtimer();
+        int k = -1;
+        bool okw = true;
+        while (*dyn_tail <= qi) {
+          if (px::ld_volatile(&c.sh->abort) || global_abort(p) || px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
+            okw = false;
+            break;
+          }
+        }
+        if (okw) k = dyn_fifo[qi & 31];
+        c.sh->flag = k;
+      }
+      px::cbar();
+      const int k = c.sh->flag;
+      px::cbar();
+      if (c.ctid == 0) *dyn_head = qi + 1;
+      if (k < 0) break;
+      I = p.instrs[k];
+    } else {
+      if (qi >= q.len) break;
+      I = q.base[qi];
+      if (!selected(p, I)) continue;
+    }
+    if (I.op == OP_NOP) continue;
+    unsigned long long *tr = trace ? p.trace + (size_t)I.seq * MK_TRACE_WORDS : nullptr;
+    if (tr && c.ctid == 0) tr[0] = px::gtimer();
+    bool bad = false;
+    if (I.wait_ctr != kNoCounter && !(p.mode & MODE_NO_WAIT) && c.ctid == 0)
+      bad = !wait_counter(p, I.wait_ctr, c.epoch * I.wait_cnt, I.seq);
+    if (bad) c.sh->abort = 1;
+    if (px::cbar_or(bad || px::ld_volatile(&c.sh->abort))) break;
+    if (tr && c.ctid == 0) tr[1] = px::gtimer();
+    c.tr = tr;
+    switch (I.op) {
+      case OP_QKV:
+        if constexpr (S::fixed) c.g = qkv_body<NB, S::RH>(c, I);
+        else MK_DISPATCH_R(op_qkv, NB, p.Rh, c, I);
+        break;
+      case OP_ATTN:
+        if constexpr (S::fixed) c.g = attn_body<S::G, S::DPL>(c, I);
+        else c.g = op_attn(c, I);
+        break;
+      case OP_OPROJ:
+        if constexpr (S::fixed) c.g = oproj_body<NB, S::RO>(c, I);
+        else MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);
+        break;
+      case OP_GATEUP:
+        if constexpr (S::fixed) c.g = gateup_body<NB, S::RH>(c, I);
+        else MK_DISPATCH_R(op_gateup, NB, p.Rh, c, I);
+        break;
+      case OP_DOWN:
+        if constexpr (S::fixed) c.g = down_body<NB, S::RD>(c, I);
+        else MK_DISPATCH_R(op_down, NB, p.Rd, c, I);
+        break;
+      case OP_LMHEAD:
+        if constexpr (S::fixed) c.g = lmhead_body<NB, S::RH>(c, I);
+        else MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I);
+        break;
+      default: break;
+    }
+    if (tr && c.ctid == 0) tr[3] = px::gtimer();
+    const bool abort_now = px::cbar_or(px::ld_volatile(&c.sh->abort) != 0);
+    if (abort_now) break;
+    // all of this CTA's outputs of the instruction are written: publish
+    const bool sig = I.sig_ctr != kNoCounter && (I.op != OP_ATTN || c.sh->flag);
+    if (c.ctid == 0 && sig) {
+      // a hint only: the data words carry this step's tag, so no fence
+      for (int k = 0; k < I.sig_n; ++k) px::red_relaxed_add(p.ctr + I.sig_ctr + k, 1u);
+    }
+    if (tr && c.ctid == 0) {
+      tr[4] = px::gtimer();
+      tr[7] = (uint64_t)I.op | ((uint64_t)I.layer << 8) | ((uint64_t)blockIdx.x << 16);
+      tr[8] = (uint64_t)(unsigned)atomicExch(&sh_stat(c), 0) |
+              ((uint64_t)(unsigned)atomicExch(&c.sh->stat_llretry, 0) << 32);
+    }
+    px::cbar();  // the staging region and the broadcast flag are reused next
+  }
+}
+
+// ============================================================== kernel
+template <int NB, bool RAW, class S>
+__global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_constant__ KParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int NP = p.num_pages;
+  uint8_t *pages = smem;
+  const int act_stride = (int)(p.act_floats / NB);
+  float *act = reinterpret_cast<float *>(smem + (size_t)NP * kPageBytes);
+  uint64_t *full = reinterpret_cast<uint64_t *>(act + p.act_floats);
+  uint64_t *empty = full + NP;
+  Shared *sh = reinterpret_cast<Shared *>(empty + NP);
+  volatile int *dyn_fifo = reinterpret_cast<volatile int *>(sh + 1);
+  volatile int *dyn_tail = dyn_fifo + 32;
+  volatile int *dyn_head = dyn_tail + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NP; ++i) {
+      px::mbar_init(&full[i], 1);
+      px::mbar_init(&empty[i], kComputeWarps);
+    }
+    px::fence_mbar_init();
+    sh->abort = 0;
+    sh->flag = 0;
+    sh->stat_cwait = 0;
+    sh->stat_llretry = 0;
+    for (int i = 0; i < 16; ++i) sh->slot_last[i] = 0;
+    *dyn_tail = 0;
+    *dyn_head = 0;
+  }
+  if (threadIdx.x < (unsigned)p.B) {
+    // this step's inputs, clamped once (out-of-range values are reported)
+    const int b = threadIdx.x;
+    const int t = __ldcg(p.tokens + b), pos = __ldcg(p.positions + b);  // tokens may alias next_tokens
+    if (t < 0 || t >= p.V || pos < 0 || pos >= p.max_seq) record_error(p, MK_ERR_DEVICE_INPUT, b, t, pos, 0);
+    sh->tok[b] = (t < 0 || t >= p.V) ? 0 : t;
+    sh->pos[b] = pos < 0 ? 0 : (pos >= p.max_seq ? p.max_seq - 1 : pos);
+  }
+  __syncthreads();
+  if (threadIdx.x < (unsigned)(p.d / 2)) sh->rope[threadIdx.x] = __ldg(p.rope + (size_t)sh->pos[0] * (p.d / 2) + threadIdx.x);
+  __syncthreads();
+  const unsigned epoch = *reinterpret_cast<volatile unsigned *>(p.epoch);
+  Queue q;
+  q.base = p.instrs + p.q_off[blockIdx.x];
+  q.len = p.q_len[blockIdx.x];
+  if (warp < kLoaders) {
+    // the dynamic queue is claimed by one loader only
+    const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
+    if (lane == 0 && (!dyn || warp == 0))
+      run_loader<RAW>(p, sh, pages, full, empty, q, dyn_fifo, dyn_tail, dyn_head, epoch, warp, dyn ? 1 : kLoaders);
+  } else {
+    CCtx c{p, sh, pages, act, act_stride, full, empty, epoch, warp - kLoaders, lane,
+           (int)threadIdx.x - 32 * kLoaders, 0u, nullptr};
+    run_compute<NB, S>(c, q, dyn_fifo, dyn_tail, dyn_head);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // every bulk copy must land before the CTA exits: after an abort the
+    // compute warps stop consuming pages, so wait on each slot's latest use
+    for (int s = 0; s < NP; ++s) {
+      const uint32_t last = sh->slot_last[s];
+      if (last == 0) continue;
+      const uint32_t ph = ((last - 1) / (uint32_t)NP) & 1u;
+      const uint64_t t0 = px::gtimer();
+      while (!px::mbar_test(&full[s], ph)) {
+        if (px::gtimer() - t0 > (uint64_t)p.timeout_ns) {
+          record_error(p, MK_ERR_TIMEOUT, -2, 2, s, (int)last);
+          break;
+        }
+      }
+    }
+  }
+  if (threadIdx.x == 0 && (p.mode & MODE_FINAL_LAUNCH)) {
+    __threadfence();
+    const unsigned old = px::atom_add_acq_rel(p.ctr + p.exit_ticket, 1u);
+    if (old == epoch * gridDim.x - 1u) {
+      // every CTA of the step has finished: advance the step number
+      atomicExch(p.epoch, epoch + 1u);
+    }
+  }
+}
+
+}  // namespace
+}  // namespace mk

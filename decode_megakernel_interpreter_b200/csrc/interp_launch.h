@@ -1,0 +1,30 @@
+// Host-side entry points of the interpreter kernels.  The shape-generic
+// kernel (and the raw-layout variant) live in interp.cu; each shape-
+// specialised kernel is built in its own translation unit so that the
+// builds compile in parallel.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "mk_internal.h"
+
+namespace mk {
+// Dynamic shared memory of a CTA with `num_pages` ring pages and a staging
+// region of `act_floats` floats.
+int shared_bytes_fixed(int num_pages, size_t act_floats);
+// The interpreter kernel for the model shape in p: a shape-specialised build
+// when one exists and `specialised` is set (*variant = 1), else the
+// shape-generic one (*variant = 0).
+const void *interp_kernel_for(const KParams &p, bool specialised, int *variant);
+// The raw-layout variant (weights read in the caller's layout).
+const void *interp_kernel_raw();
+// Allow `smem` bytes of dynamic shared memory for fn and report how many of
+// its CTAs fit on one SM.
+cudaError_t interp_prepare(const void *fn, int smem, int *blocks_per_sm);
+// Launch fn over `grid` CTAs (cooperatively when asked).
+cudaError_t launch_interp(const void *fn, const KParams &p, int grid, int smem, cudaStream_t st, bool cooperative);
+
+// shape-specialised kernels (interp_spec_*.cu)
+const void *spec_kernel_llama1b();
+const void *spec_kernel_llama8b();
+}  // namespace mk

@@ -20,7 +20,7 @@ constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kMaxKc = 4096;                  // largest K staged in one page row
 constexpr int kMaxBatch = 16;
 constexpr int kMaxDownPieces = 8;             // ffn / 2048 at most
-constexpr int kDefaultInflight = 6;           // bulk-copy pages in flight per CTA
+constexpr int kDefaultInflight = 4;           // bulk-copy pages in flight per CTA
 
 // ---------------------------------------------------------------- opcodes
 // The instruction set of the decode step (the fused instructions the
@@ -104,16 +104,20 @@ struct KParams {
   uint16_t *kc, *vc;
   long long kv_ls, kv_bs, kv_hs;   // element strides: layer, batch, head (position stride = d)
   const float2 *rope;              // [max_seq][d/2] (cos, sin)
-  // activations (fp32)
-  float *qbuf;     // [L][B][q_dim]
-  float *part_o;   // [L][B][nq][S][d]
-  float *part_ml;  // [L][B][nq][S][2]
-  float *obuf;     // [L][B][q_dim]
-  float *xres;     // [L][B][H]
-  float *actb;     // [L][B][F]
-  float *dpart;    // [L][ndp][B][H]
-  float *arg_val;  // [B][n_lm]
-  int *arg_idx;    // [B][n_lm]
+  // activations: tagged fp32 words (value rounded to 21 significant bits, the
+  // two low mantissa bits = step number mod 4)
+  float *qbuf;                  // [L][B][q_dim]
+  float *kvcur;                 // [L][B][2][kv_dim]  this step's K and V rows (bf16-rounded)
+  float *part_o;                // [L][B][nq][S][d]
+  float *obuf;                  // [L][B][q_dim]
+  float *xres;                  // [L][B][H]
+  float *actb;                  // [L][B][F]
+  float *dpart;                 // [L][ndp][B][H]
+  // tagged 64-bit words (step number << 32 | 32-bit value): values that may
+  // be -inf, and indices
+  unsigned long long *part_ml;  // [L][B][nq][S][2]
+  unsigned long long *arg_val;  // [B][n_lm]
+  unsigned long long *arg_idx;  // [B][n_lm] (index bits in the value field)
   int n_lm;        // LM-head instructions (argmax slots) per step
   // sync
   unsigned *ctr;      // counters + tickets

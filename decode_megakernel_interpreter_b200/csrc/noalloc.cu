@@ -25,14 +25,9 @@
 #include <vector>
 
 #include "../../include/mk.h"
+#include "interp_launch.h"
 #include "mk_internal.h"
 #include "planner.h"
-
-namespace mk {
-cudaError_t launch_interp_raw(const KParams &p, int grid, int smem, cudaStream_t st);
-cudaError_t occupancy_interp(int nb, int smem, int *blocks_per_sm);
-int shared_bytes_fixed(int num_pages, size_t act_floats);
-}  // namespace mk
 
 using namespace mk;
 
@@ -140,12 +135,16 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   const size_t o_layers = lay.take(sizeof(LayerDev) * s.L), o_raw = lay.take(sizeof(LayerRaw) * s.L);
   const size_t o_rope = lay.take(sizeof(float2) * (size_t)cfg->max_seq * hd);
   const size_t qd = (size_t)s.nq * s.d;
+  // activations are tagged words; all of them, with the counters, are cleared
+  // by every call (the step number restarts at 1 each call)
+  const size_t tagged_begin = lay.off;
   const size_t o_q = lay.take(4 * (size_t)s.L * B * qd), o_o = lay.take(4 * (size_t)s.L * B * qd);
   const size_t o_x = lay.take(4 * (size_t)s.L * B * s.H), o_act = lay.take(4 * (size_t)s.L * B * s.F);
   const size_t o_dp = lay.take(4 * (size_t)s.L * p.ndp * B * s.H);
+  const size_t o_kv = lay.take(4 * (size_t)s.L * B * 2 * s.nkv * s.d);
   const size_t o_po = lay.take(4 * (size_t)s.L * B * s.nq * p.S * s.d);
-  const size_t o_pml = lay.take(4 * (size_t)s.L * B * s.nq * p.S * 2);
-  const size_t o_av = lay.take(4 * (size_t)B * p.n_lm), o_ai = lay.take(4 * (size_t)B * p.n_lm);
+  const size_t o_pml = lay.take(8 * (size_t)s.L * B * s.nq * p.S * 2);
+  const size_t o_av = lay.take(8 * (size_t)B * p.n_lm), o_ai = lay.take(8 * (size_t)B * p.n_lm);
   if (lay.off > MK_NOALLOC_SCRATCH_BYTES) return MK_ERR_UNSUPPORTED_SHAPE;
 
   // shared memory geometry (as mk_plan)
@@ -208,9 +207,11 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
     }
     slot->key = key;
   }
-  // every call starts from zeroed counters and status, step number 1
+  // every call starts from zeroed counters, status and tagged activations,
+  // step number 1
   static const unsigned kOne = 1;
   e = cudaMemsetAsync(base, 0, sync_end, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(base + tagged_begin, 0, lay.off - tagged_begin, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(base + o_epoch, &kOne, sizeof kOne, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -249,15 +250,17 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   k.kv_bs = k.kv_hs * s.nkv;
   k.kv_ls = k.kv_bs * cfg->max_batch;
   k.rope = reinterpret_cast<const float2 *>(base + o_rope);
+  typedef unsigned long long llw;
   k.qbuf = reinterpret_cast<float *>(base + o_q);
+  k.kvcur = reinterpret_cast<float *>(base + o_kv);
   k.part_o = reinterpret_cast<float *>(base + o_po);
-  k.part_ml = reinterpret_cast<float *>(base + o_pml);
+  k.part_ml = reinterpret_cast<llw *>(base + o_pml);
   k.obuf = reinterpret_cast<float *>(base + o_o);
   k.xres = reinterpret_cast<float *>(base + o_x);
   k.actb = reinterpret_cast<float *>(base + o_act);
   k.dpart = reinterpret_cast<float *>(base + o_dp);
-  k.arg_val = reinterpret_cast<float *>(base + o_av);
-  k.arg_idx = reinterpret_cast<int *>(base + o_ai);
+  k.arg_val = reinterpret_cast<llw *>(base + o_av);
+  k.arg_idx = reinterpret_cast<llw *>(base + o_ai);
   k.n_lm = p.n_lm;
   k.ctr = reinterpret_cast<unsigned *>(base + o_ctr);
   k.epoch = reinterpret_cast<unsigned *>(base + o_epoch);
@@ -282,7 +285,11 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   k.positions = positions;
   k.logits = logits_out;
   k.next_tokens = next_tokens_out;
-  e = launch_interp_raw(k, p.num_ctas, smem, st);
+  const void *fn = interp_kernel_raw();
+  int per_sm = 0;
+  e = interp_prepare(fn, smem, &per_sm);
+  if (e == cudaSuccess && per_sm < 1) return MK_ERR_LAUNCH;
+  if (e == cudaSuccess) e = launch_interp(fn, k, p.num_ctas, smem, st, true);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorLaunchOutOfResources) ? MK_ERR_LAUNCH

@@ -115,7 +115,15 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv,
 
 /* ------------------------------------------------------------------ plan */
 enum { MK_SCHED_STATIC = 0, MK_SCHED_DYNAMIC = 1 };
-enum { MK_EXEC_MEGAKERNEL = 0, MK_EXEC_PER_OP = 1, MK_EXEC_PER_OP_GRAPH = 2 };
+enum {
+  MK_EXEC_MEGAKERNEL = 0,        /* one persistent launch per step */
+  MK_EXEC_PER_OP = 1,            /* comparison path: one launch per instruction class */
+  MK_EXEC_PER_OP_GRAPH = 2,      /* the same launches replayed as a CUDA graph */
+  MK_EXEC_MEGAKERNEL_GENERIC = 3 /* one persistent launch of the shape-generic
+                                    interpreter build (identical results; the
+                                    default picks a shape-specialised build when
+                                    the model's shape has one) */
+};
 
 typedef struct {
   int32_t batch;          /* sequences per step, 1..max_batch */
@@ -124,7 +132,8 @@ typedef struct {
                              (one global queue claimed with an atomic) */
   int32_t exec_mode;      /* MK_EXEC_MEGAKERNEL, or the comparison path:
                              one launch per instruction class (PER_OP), optionally
-                             replayed as a CUDA graph (PER_OP_GRAPH) */
+                             replayed as a CUDA graph (PER_OP_GRAPH), or
+                             MK_EXEC_MEGAKERNEL_GENERIC */
   int32_t num_sms;        /* CTAs of the persistent grid; 0 = every SM */
   int32_t trace;          /* 1: record per-instruction timestamps (mk_trace_read) */
   int64_t wait_timeout_ns;/* bound on every device-side wait; 0 = 1 second */
@@ -135,7 +144,7 @@ typedef struct {
                              wait must report MK_ERR_TIMEOUT; 0 in normal use */
   int32_t max_inflight_pages; /* 16 KiB weight/KV pages a CTA keeps in flight
                              (the rest of its page ring only buffers landed
-                             pages); 0 = automatic (6), -1 = no cap; rounded
+                             pages); 0 = automatic (4), -1 = no cap; rounded
                              down to a multiple of the loader count (2) */
 } mk_plan_opts;
 
@@ -199,12 +208,17 @@ typedef struct {
   int32_t kv_splits;
   int32_t max_queue_len;   /* longest per-CTA queue (static mode) */
   int64_t weight_bytes_per_step; /* weight bytes the plan streams per step */
+  int32_t kernel_variant;  /* 0: the shape-generic interpreter build, 1: a build
+                              specialised for this model's shape (every op body
+                              inlined into the interpreter loop) */
+  int32_t reserved;
 } mk_plan_info;
 
 /*
  * mk_get_error_detail: the detail words of the last device-side error that
  * mk_get_status returned (host int32 [6]): instruction sequence number (-1:
- * a shared-memory page wait, -2: the final drain), counter index or wait kind,
+ * a shared-memory page wait, -2: the final drain, -3: a group of tagged
+ * activation loads that never saw this step's tag), counter index or wait kind,
  * observed value, target value, CTA, and the abort flag.  All zero if none.
  */
 int mk_get_error_detail(const mk_handle *h, int32_t detail[6]);
@@ -221,7 +235,9 @@ int mk_get_plan_info(const mk_handle *h, mk_plan_info *info);
  * consumed and its outputs written, 4 = it signalled completion, 5 / 6 = the
  * loader issued its first / last page (5 == 6 when it has no pages),
  * 7 = (opcode | layer << 8 | cta << 16), 8 = pages the compute warps found
- * not yet landed, 9 = pages the loader found no free ring slot for.
+ * not yet landed (low 32 bits) | groups of tagged activation loads re-issued
+ * because a word was not yet this step's (high 32 bits), 9 = pages the loader
+ * found no free ring slot for.
  */
 #define MK_TRACE_WORDS 10
 int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
@@ -241,7 +257,7 @@ int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
  *
  * How: no handle.  The step's scratch (plan, RoPE table, activations,
  * attention and argmax partials, counters, status) lives in one file-scope
- * device array of MK_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU that loads
+ * device array of MK_NOALLOC_SCRATCH_BYTES (16 MiB), which every GPU that loads
  * the library holds until the process exits.  The weights are read in the
  * caller's own layout, so no repacked copy is made.  This call makes no
  * cudaMalloc / cudaFree and uses no allocating library routine.
@@ -256,7 +272,7 @@ int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
  *    Make that first call before any stream capture.  Later calls re-upload
  *    (and synchronise) only when cfg or the weight pointers change.
  *  - Every call shares the array and leaves its contents behind; each call
- *    clears the counters and status it needs.  Calls that overlap on the GPU
+ *    clears the counters, status and activation words it needs.  Calls that overlap on the GPU
  *    (other streams, other threads) race on the array: serialise them.
  *  - Errors: MK_ERR_INVALID_ARG (NULL or misaligned pointer, bad cfg),
  *    MK_ERR_UNSUPPORTED_SHAPE (shape not implemented, batch != 1, or the
@@ -265,7 +281,7 @@ int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
  *    MK_ERR_LAUNCH, MK_ERR_CUDA.  Device-side errors of the step (timeout,
  *    clamped input) are not reported by this call.
  */
-#define MK_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define MK_NOALLOC_SCRATCH_BYTES (16u << 20)
 int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv,
                            const int32_t *tokens, const int32_t *positions, float *logits_out,
                            int32_t *next_tokens_out, void *stream);

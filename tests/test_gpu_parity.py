@@ -34,7 +34,8 @@ def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan
     logits = torch.empty(hs.batch, s.vocab, dtype=torch.float32, device="cuda")
     nxt = torch.empty(hs.batch, dtype=torch.int32, device="cuda")
     tok, p = first_token, first_pos
-    stats = {"near_ties": 0, "max_abs": 0.0, "max_rel": 0.0, "tokens": [], "logits": []}
+    stats = {"near_ties": 0, "max_abs": 0.0, "max_rel": 0.0, "tokens": [], "logits": [],
+             "kernel_variant": int(eng.info.kernel_variant)}
     try:
         for step in range(steps):
             tokens.fill_(tok)
@@ -98,11 +99,12 @@ def tiny_setup(model, max_seq=96):
     dict(),
     dict(exec_mode="per_op"),
     dict(exec_mode="per_op_graph"),
+    dict(exec_mode="megakernel_generic"),
     dict(sched="dynamic"),
     dict(num_sms=3, kv_splits=7),
     dict(num_sms=1, kv_splits=1),
     dict(l2_prefetch_kb=256),
-], ids=["mk", "per_op", "per_op_graph", "dynamic", "3sm", "1sm", "l2pf"])
+], ids=["mk", "per_op", "per_op_graph", "mk_generic", "dynamic", "3sm", "1sm", "l2pf"])
 def test_tiny_16_steps(tiny_model, kw):
     hs, tok, pos = tiny_setup(tiny_model)
     run_parity(hs, tok, pos, 16, kw)
@@ -246,15 +248,19 @@ def test_llama1b_8k_context(llama1b_model):
     run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 2, dict())
 
 
-def test_llama1b_per_op_matches_megakernel(llama1b_model):
+def test_llama1b_per_op_and_generic_match_megakernel(llama1b_model):
+    """The shape-specialised interpreter (the default for this shape), the
+    shape-generic one and the per-op launches compute bit-identical steps."""
     w = synth.WORKLOADS["llama1b"]
     outs = []
-    for kw in (dict(), dict(exec_mode="per_op")):
+    for kw in (dict(), dict(exec_mode="per_op"), dict(exec_mode="megakernel_generic")):
         hs = HostSetup(w.shape, 1, w.context + 4, llama1b_model)
         hs.fill_prefix(w.lengths())
         outs.append(run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 2, kw, check_kv=False))
-    for a, b in zip(outs[0]["logits"], outs[1]["logits"]):
-        np.testing.assert_array_equal(a, b)
+    assert [o["kernel_variant"] for o in outs] == [1, 1, 0]
+    for o in outs[1:]:
+        for a, b in zip(outs[0]["logits"], o["logits"]):
+            np.testing.assert_array_equal(a, b)
 
 
 def test_llama8b_2048_context():
