@@ -67,6 +67,10 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Bring [src, src + bytes) into L2 (no completion to wait for).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
                                          uint64_t policy) {
   asm volatile(
@@ -74,9 +78,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       " [%0], [%1], %2, [%3], %4;" ::"r"(sa(dst)),
       "l"(src), "r"(bytes), "r"(sa(bar)), "l"(policy)
       : "memory");
-}
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t pol;
@@ -208,6 +209,11 @@ struct Shared {
   int pos[kMaxBatch], tok[kMaxBatch];  // this step's (clamped) positions and token ids
   int stat_cwait;  // trace mode: pages a compute warp found not yet landed (this instruction)
   int stat_llretry;  // tagged-load groups re-issued because a word was stale (this instruction)
+  // the current instruction's dependency: its producers' completion counter
+  // (kNoCounter: none), the count that means "all done", and who polls it
+  uint32_t dep_ctr, dep_target;
+  int dep_seq;
+  int dep_state;   // 0: not checked, 1: a thread is polling, 2: met, 3: failed
   uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
   float red[kComputeWarps][kMaxBatch];
   float argv[kComputeWarps][kMaxBatch];
@@ -259,18 +265,44 @@ __device__ __noinline__ bool ll_give_up(const KParams *p, Shared *sh, uint64_t t
   }
   return false;
 }
+// Wait until the current instruction's producers have all signalled.  One
+// thread of the CTA polls the counter (a relaxed hint: the data words still
+// carry their own tags); the others watch shared memory.  false on timeout
+// or abort.
+__device__ bool wait_counter(const KParams &p, unsigned idx, unsigned target, int seq);
+__device__ __noinline__ bool dep_wait(const KParams *p, Shared *sh) {
+  int st = px::ld_volatile(&sh->dep_state);
+  if (st == 2) return true;
+  if (st == 0 && atomicCAS(&sh->dep_state, 0, 1) == 0) {
+    const bool ok = sh->dep_ctr == kNoCounter || wait_counter(*p, sh->dep_ctr, sh->dep_target, sh->dep_seq);
+    if (!ok) sh->abort = 1;
+    atomicExch(&sh->dep_state, ok ? 2 : 3);
+    return ok;
+  }
+  const uint64_t t0 = px::gtimer();
+  while ((st = px::ld_volatile(&sh->dep_state)) == 1) {
+    __nanosleep(64);
+    if (px::gtimer() - t0 > (uint64_t)p->timeout_ns + 1000000ull) return false;  // the poller reports
+  }
+  return st == 2;
+}
 // Called after a group came back with a stale word: true = re-issue it,
 // false = give up (timeout or abort; the CTA is aborting, values are unused).
+// The first miss waits for the producers' completion count; later misses
+// (the count can become visible before the data) re-issue at once.
 struct LLRetry {
   unsigned n = 0;
   uint64_t t0 = 0;
 };
 __device__ __forceinline__ bool ll_retry(const KParams &p, Shared *sh, LLRetry &r, int where) {
   if (r.n++ == 0) {
-    r.t0 = px::gtimer();
     atomicAdd(&sh->stat_llretry, 1);
-  } else if ((r.n & 7u) == 0 && ll_give_up(&p, sh, r.t0, where)) {
-    return false;
+    if (!dep_wait(&p, sh)) return false;
+    r.t0 = px::gtimer();
+  } else {
+    // the words are on their way: back off instead of flooding L2 with loads
+    __nanosleep(128);
+    if ((r.n & 7u) == 0 && ll_give_up(&p, sh, r.t0, where)) return false;
   }
   return true;
 }
@@ -444,6 +476,39 @@ __device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, 
   return s;
 }
 
+// L2 prefetch cursor of one loader lane: it walks this loader's future pages
+// (the same order as the copies) and, only while the ring is full (the
+// compute warps are waiting on a dependency, so HBM would idle), asks L2 for
+// pages up to `pf_pages` ahead of the next copy.  The copies of those pages
+// then read L2 instead of HBM when their slots free up.
+struct PfCursor {
+  int qi = -1;         // instruction index in the queue (-1: not started)
+  uint32_t g0 = 0;     // its first page number
+  uint32_t gp = 0;     // next page number to prefetch (this loader's)
+  PageSrc ps;
+};
+// Issue one page prefetch; false when the budget is used up or the queue ends.
+__device__ __forceinline__ bool pf_step(const KParams &p, const Shared *sh, const Queue &q, PfCursor &c,
+                                        uint32_t g_next, int li, int nl) {
+  if (c.gp >= g_next + (uint32_t)p.pf_pages) return false;
+  while (c.gp >= c.g0 + (uint32_t)c.ps.npg) {
+    const uint32_t g_end = c.g0 + (uint32_t)c.ps.npg;
+    int k = c.qi + 1;
+    while (k < q.len && !selected(p, q.base[k])) ++k;
+    if (k >= q.len) return false;
+    c.qi = k;
+    c.g0 = g_end;
+    c.ps = page_src(p, sh, q.base[k]);
+    c.gp = g_end + (uint32_t)((li - (int)(g_end % nl) + nl) % nl);
+  }
+  const int t = (int)(c.gp - c.g0);
+  const uint32_t bytes = (t == c.ps.npg - 1) ? c.ps.last : c.ps.bytes;
+  px::bulk_prefetch_l2(c.ps.a + (size_t)t * c.ps.stride, bytes);
+  if (c.ps.b) px::bulk_prefetch_l2(c.ps.b + (size_t)t * c.ps.stride, bytes);
+  c.gp += (uint32_t)nl;
+  return true;
+}
+
 // One loader lane streams the pages g with g % nl == li of every instruction
 // of its CTA's queue into the ring (several loaders overlap the issue
 // latency of the bulk copies, which is long for a single thread).
@@ -461,6 +526,8 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
   const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
   const unsigned dyn_base = dyn ? (epoch - 1u) * (unsigned)(p.n_instr + gridDim.x) : 0u;
   int claimed = 0;
+  const bool use_pf = !RAW && !dyn && p.pf_pages > 0;
+  PfCursor pf;
   for (int qi = 0; ok; ++qi) {
     Instr I;
     if (dyn) {
@@ -497,7 +564,20 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
       const uint32_t slot = gg % NP;
       const uint32_t ph = (gg / NP) & 1u;
       if (gg >= NP) {
-        if (ltr && !px::mbar_test(&empty[slot], ph ^ 1u)) ++lwait;
+        if (!px::mbar_test(&empty[slot], ph ^ 1u)) {
+          if (ltr) ++lwait;
+          if (use_pf) {
+            // ring full: spend the wait bringing later pages into L2
+            if (pf.qi < qi || (pf.qi == qi && pf.gp < gg)) {
+              pf.qi = qi;
+              pf.g0 = g0;
+              pf.gp = gg;
+              pf.ps = ps;
+            }
+            while (!px::mbar_test(&empty[slot], ph ^ 1u) && pf_step(p, sh, q, pf, gg, li, nl)) {
+            }
+          }
+        }
         if (!wait_bar(p, sh, &empty[slot], ph ^ 1u, 1)) {
           ok = false;
           break;
@@ -1504,6 +1584,12 @@ struct Spec {
 };
 using SpecGeneric = Spec<0, 0, 0, 0, 0>;
 
+// Ops that start before their producers are known to be done (bit op).
+#ifndef MK_SPECULATIVE_OPS
+#define MK_SPECULATIVE_OPS ((1u << OP_QKV) | (1u << OP_GATEUP) | (1u << OP_DOWN) | (1u << OP_LMHEAD))
+#endif
+constexpr unsigned kSpeculativeOps = MK_SPECULATIVE_OPS;
+
 template <int NB, class S>
 __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile int *dyn_tail,
                             volatile int *dyn_head) {
@@ -1541,11 +1627,24 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
     if (I.op == OP_NOP) continue;
     unsigned long long *tr = trace ? p.trace + (size_t)I.seq * MK_TRACE_WORDS : nullptr;
     if (tr && c.ctid == 0) tr[0] = px::gtimer();
-    bool bad = false;
-    if (I.wait_ctr != kNoCounter && !(p.mode & MODE_NO_WAIT) && c.ctid == 0)
-      bad = !wait_counter(p, I.wait_ctr, c.epoch * I.wait_cnt, I.seq);
-    if (bad) c.sh->abort = 1;
-    if (px::cbar_or(bad || px::ld_volatile(&c.sh->abort))) break;
+    if (c.ctid == 0) {
+      // every input of the instruction carries this step's tag, so an op in
+      // kSpeculativeOps starts at once and polls its producers' completion
+      // count only when a load comes back stale; the others wait for the
+      // count first
+      const bool has_dep = I.wait_ctr != kNoCounter && !(p.mode & MODE_NO_WAIT);
+      c.sh->dep_ctr = has_dep ? I.wait_ctr : kNoCounter;
+      c.sh->dep_target = c.epoch * I.wait_cnt;
+      c.sh->dep_seq = I.seq;
+      c.sh->dep_state = 0;
+      if (has_dep && !((kSpeculativeOps >> I.op) & 1u)) {
+        c.sh->dep_state = 1;
+        const bool ok = wait_counter(p, I.wait_ctr, c.epoch * I.wait_cnt, I.seq);
+        if (!ok) c.sh->abort = 1;
+        c.sh->dep_state = ok ? 2 : 3;
+      }
+    }
+    if (px::cbar_or(px::ld_volatile(&c.sh->abort))) break;
     if (tr && c.ctid == 0) tr[1] = px::gtimer();
     c.tr = tr;
     switch (I.op) {

@@ -137,8 +137,10 @@ typedef struct {
   int32_t num_sms;        /* CTAs of the persistent grid; 0 = every SM */
   int32_t trace;          /* 1: record per-instruction timestamps (mk_trace_read) */
   int64_t wait_timeout_ns;/* bound on every device-side wait; 0 = 1 second */
-  int32_t l2_prefetch_kb; /* reserved (an L2 prefetch cursor measured slower on
-                             B200 and was removed); accepted and ignored */
+  int32_t l2_prefetch_kb; /* L2 look-ahead per CTA, KiB: while its page ring is
+                             full (the compute warps wait on a dependency), the
+                             loader asks L2 for up to this many bytes of later
+                             weight / KV pages; 0 = automatic, -1 = off */
   int32_t debug_drop_producer; /* TEST HOOK: 1 drops one producer instruction so
                              that a dependency can never be met and the bounded
                              wait must report MK_ERR_TIMEOUT; 0 in normal use */
