@@ -477,6 +477,7 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   k.S = p.S;
   k.max_seq = h->cfg.max_seq;
   k.eps = h->cfg.rms_eps;
+  k.inv_H = 1.0f / (float)s.H;
   k.attn_scale = (float)(1.0 / std::sqrt((double)s.d));
   k.layers = h->d_layers;
   k.embed = h->embed;

@@ -487,6 +487,10 @@ struct PfCursor {
   uint32_t gp = 0;     // next page number to prefetch (this loader's)
   PageSrc ps;
 };
+#ifndef MK_PF_GAP_NS
+#define MK_PF_GAP_NS 0
+#endif
+constexpr uint64_t kPfGapNs = MK_PF_GAP_NS;
 // Issue one page prefetch; false when the budget is used up or the queue ends.
 __device__ __forceinline__ bool pf_step(const KParams &p, const Shared *sh, const Queue &q, PfCursor &c,
                                         uint32_t g_next, int li, int nl) {
@@ -528,6 +532,7 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
   int claimed = 0;
   const bool use_pf = !RAW && !dyn && p.pf_pages > 0;
   PfCursor pf;
+  uint64_t pf_last = 0;
   for (int qi = 0; ok; ++qi) {
     Instr I;
     if (dyn) {
@@ -554,6 +559,16 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
     }
     unsigned long long *ltr = (trace && li == 0) ? p.trace + (size_t)I.seq * MK_TRACE_WORDS : nullptr;
     if (ltr) ltr[5] = px::gtimer();
+    if (li == 0) {
+      // the RMSNorm weight the compute warps load with the instruction's
+      // input: bring it into L2 now (it is small, and read from HBM it would
+      // add a memory round trip to the staging)
+      const uint16_t *gamma = I.op == OP_QKV      ? p.layers[I.layer].attn_norm
+                              : I.op == OP_GATEUP ? p.layers[I.layer].ffn_norm
+                              : I.op == OP_LMHEAD ? p.final_norm
+                                                  : nullptr;
+      if (gamma && ((uintptr_t)gamma & 15u) == 0 && (p.H * 2) % 16 == 0) px::bulk_prefetch_l2(gamma, (uint32_t)p.H * 2);
+    }
     unsigned lwait = 0;
     const PageSrc ps = page_src(p, sh, I);
     const uint32_t g0 = g;
@@ -574,7 +589,14 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
               pf.gp = gg;
               pf.ps = ps;
             }
-            while (!px::mbar_test(&empty[slot], ph ^ 1u) && pf_step(p, sh, q, pf, gg, li, nl)) {
+            // paced: at most one page per kPfGapNs per loader, so that the
+            // look-ahead uses spare HBM bandwidth without queueing ahead of
+            // the activation exchanges
+            while (!px::mbar_test(&empty[slot], ph ^ 1u)) {
+              const uint64_t now = px::gtimer();
+              if (now - pf_last < kPfGapNs) continue;
+              if (!pf_step(p, sh, q, pf, gg, li, nl)) break;
+              pf_last = now;
             }
           }
         }
@@ -817,7 +839,7 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
     float t = 0.f;
 #pragma unroll
     for (int w = 0; w < kComputeWarps; ++w) t += c.sh->red[w][b];
-    inv[b] = 1.0f / sqrtf(t / (float)H + p.eps);
+    inv[b] = __frsqrt_rn(t * p.inv_H + p.eps);  // one rounding; t * (1/H) == t / H for H = 2^k
   }
 #pragma unroll
   for (int b = 0; b < NB; ++b) {

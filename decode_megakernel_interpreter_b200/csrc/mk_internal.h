@@ -96,6 +96,7 @@ struct KParams {
   int S;        // kv splits
   int max_seq;
   float eps, attn_scale;
+  float inv_H;                     // 1 / hidden (exact: hidden is a power of two)
   // weights
   const LayerDev *layers;
   const LayerRaw *layers_raw;  // only read by the raw-layout kernel variant

@@ -238,6 +238,7 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   k.S = p.S;
   k.max_seq = cfg->max_seq;
   k.eps = cfg->rms_eps;
+  k.inv_H = 1.0f / (float)s.H;
   k.attn_scale = (float)(1.0 / std::sqrt((double)s.d));
   k.layers = reinterpret_cast<const LayerDev *>(base + o_layers);
   k.layers_raw = reinterpret_cast<const LayerRaw *>(base + o_raw);
