@@ -1,29 +1,30 @@
 // The decode interpreter: one persistent CTA per SM runs a queue of
-// instructions (fetch -> wait for dependency counters -> stage the input
-// vector -> stream weight pages -> compute -> store -> signal), after the
-// on-GPU interpreter of the "Hazy megakernel summary" page (section 四(二))
-// and the task loop of the "Mirage Persistent Kernel" article (Part 2).
+// instructions (fetch -> stage the input vector -> stream weight pages ->
+// compute -> store -> signal), after the on-GPU interpreter of the "Hazy
+// megakernel summary" page (section 四(二)) and the task loop of the
+// "Mirage Persistent Kernel" article (Part 2).
 //
 // Warp roles (this build's design for sm_100a):
-//   warp 0, lane 0  loader: walks the same queue ahead of the compute warps and
-//                   streams every weight / KV page of every instruction into a
-//                   ring of 16 KiB shared-memory pages with 1-D bulk copies
-//                   (cp.async.bulk, mbarrier completion).  Weights never depend
-//                   on activations, so the next instructions' pages load while
-//                   the current one is still waiting or storing (the paged
-//                   shared memory of the same section, whose freed pages go to
-//                   the next instruction).  Optionally it also runs an L2
-//                   prefetch cursor further ahead (cp.async.bulk.prefetch.L2).
-//   warps 1..8      compute: CUDA-core fp32 FMA matrix-vector products over
+//   warps 0, 1 (lane 0 of each)  loaders: walk the same queue ahead of the
+//                   compute warps and stream every weight / KV page of every
+//                   instruction into a ring of 16 KiB shared-memory pages
+//                   with 1-D bulk copies (cp.async.bulk, mbarrier
+//                   completion); loader i owns the pages g with g % 2 == i.
+//                   Weights never depend on activations, so the next
+//                   instructions' pages load while the current one is still
+//                   waiting or storing (the paged shared memory of the same
+//                   section, whose freed pages go to the next instruction).
+//   warps 2..9      compute: CUDA-core fp32 FMA matrix-vector products over
 //                   bf16 pages (batch 1 is a matrix-vector product; tensor
 //                   cores do not help there, section 五(二)), warp-shuffle
-//                   reductions, fused epilogues, and the counter protocol.
-// Synchronisation between instructions: an array of counters in global memory
-// (section 四(二) "同步"): a producer adds 1 (release) when done, a consumer
-// waits (acquire) until the counter reaches epoch * producers.  Counters are
-// never reset; `epoch` is the step number.  Every wait is bounded by a
-// global-timer deadline; a timeout records MK_ERR_TIMEOUT and makes every CTA
-// leave cleanly.
+//                   reductions, fused epilogues, and the signalling.
+// Synchronisation between instructions: activations are tagged words that
+// carry the step number (epoch), so a reader tells this step's value from a
+// stale one by itself; completion counters in global memory (section 四(二)
+// "同步") are relaxed hints telling a waiting CTA when to look again.
+// Counters are never reset: targets are epoch * producers.  Every wait is
+// bounded by a global-timer deadline; a timeout records MK_ERR_TIMEOUT and
+// makes every CTA leave cleanly.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
