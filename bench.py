@@ -150,15 +150,19 @@ class ClockSampler:
 
 
 def step_bytes(shape, weight_bytes: int, positions, logits: bool) -> float:
-    """Algorithmic HBM bytes of one step: weights streamed once (+ norm
-    vectors and one embedding row per sequence), the KV cache read over
-    positions 0..pos, the new K/V row written, fp32 logits written."""
+    """Algorithmic HBM bytes of one step, averaged over the timed steps:
+    weights streamed once for all sequences (+ norm vectors), and per sequence
+    one embedding row, the KV cache read over positions 0..pos, the new K/V
+    row written and fp32 logits written.  positions[i][b]: position of
+    sequence b at step i."""
     L, H, d, nkv = shape.n_layers, shape.hidden, shape.head_dim, shape.n_kv_heads
     norms = (2 * L + 1) * H * 2
     per_pos = L * nkv * d * 2 * 2
     tot = 0.0
-    for p in positions:
-        tot += weight_bytes + norms + H * 2 + per_pos * (p + 1) + per_pos + (shape.vocab * 4 if logits else 0)
+    for row in positions:
+        tot += weight_bytes + norms
+        for p in row:
+            tot += H * 2 + per_pos * (p + 1) + per_pos + (shape.vocab * 4 if logits else 0)
     return tot / len(positions)
 
 
@@ -237,8 +241,7 @@ def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
     import numpy as np
     import torch
     eng.plan(**{**eng.plan_kw, "trace": True})
-    pos = torch.tensor([pos0], dtype=torch.int32, device="cuda")
-    eng.decode_step(tokens, pos, logits, nxt)
+    eng.decode_step(tokens, pos0, logits, nxt)
     torch.cuda.synchronize()
     tr = eng.trace().astype(np.int64)
     eng.plan(**eng.plan_kw)
@@ -291,8 +294,9 @@ def main():
     s = w.shape
     B = w.batch
     K, W = args.steps, args.warmup
-    ctx = int(w.lengths()[0])
-    max_seq = ctx + K + W + 2
+    lengths = [int(x) for x in w.lengths()]
+    ctx = lengths[0]
+    max_seq = max(lengths) + K + W + 2
     model = synth.make_model(s)
     dev = harness.upload_model(model, s.tied)
     k, v = synth.alloc_kv(s, B, max_seq)
@@ -307,12 +311,14 @@ def main():
     stream = torch.cuda.current_stream()
     first = torch.tensor(synth.first_tokens(w), dtype=torch.int32, device="cuda")
     tokens = first.clone()  # next_tokens_out aliases tokens: device-to-device feedback
-    pos_all = torch.arange(ctx, ctx + max(K, W) + 1, dtype=torch.int32, device="cuda")
+    # positions of every sequence at every step (row i: step i)
+    pos_host = torch.tensor([[n + i for n in lengths] for i in range(max(K, W) + 1)], dtype=torch.int32)
+    pos_all = pos_host.to("cuda")
     logits = None if args.no_logits else torch.empty(B, s.vocab, dtype=torch.float32, device="cuda")
     lptr = logits.data_ptr() if logits is not None else None
 
     def step(i):
-        rc = mk.mk_decode_step(eng.h, tokens.data_ptr(), pos_all.data_ptr() + 4 * i, lptr, tokens.data_ptr(),
+        rc = mk.mk_decode_step(eng.h, tokens.data_ptr(), pos_all[i].data_ptr(), lptr, tokens.data_ptr(),
                                stream.cuda_stream)
         if rc != mk.MK_OK:
             raise mk.MkError(rc, "mk_decode_step")
@@ -365,7 +371,7 @@ def main():
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(K):
-            h_pos.fill_(ctx + i)
+            h_pos.copy_(pos_host[i])
             d_tok.copy_(h_tok, non_blocking=True)
             d_pos.copy_(h_pos, non_blocking=True)
             rc = mk.mk_decode_step(eng.h, d_tok.data_ptr(), d_pos.data_ptr(), lptr, d_next.data_ptr(),
@@ -385,13 +391,13 @@ def main():
         e2e = {"value": world * K / (ems / 1e3), "unit": "steps/s", "h2d_bytes_per_step": 8 * B,
                "d2h_bytes_per_step": 4 * B, "us_per_step": 1e3 * ems / K}
 
-    bd = breakdown(eng, mk, info, tokens, ctx, logits, torch.empty_like(tokens)) if args.breakdown else None
+    bd = breakdown(eng, mk, info, tokens, pos_all[0], logits, torch.empty_like(tokens)) if args.breakdown else None
     eng.close()
 
     if rank == 0:
         peak, peak_kind = peaks()
-        positions = [ctx + i for i in range(K)]
-        bytes_step = step_bytes(s, info.weight_bytes_per_step, positions, logits is not None) * B
+        positions = [[n + i for n in lengths] for i in range(K)]
+        bytes_step = step_bytes(s, info.weight_bytes_per_step, positions, logits is not None)
         achieved = bytes_step / (us_step * 1e-6) / 1e9
         out = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": W,

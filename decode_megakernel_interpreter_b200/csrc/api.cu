@@ -255,8 +255,10 @@ int check_cfg(const mk_config *c, std::string *why) {
 
 size_t act_floats_for(const mk_config &c, const Plan &p, int nb) {
   const int G = c.n_q_heads / c.n_kv_heads;
-  // input vector (+ the O projection's residual rows after it)
-  size_t vec = (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim + c.hidden, p.KCd});
+  // input vector per sequence (batch 1: + the O projection's residual rows
+  // after it)
+  size_t vec = nb == 1 ? (size_t)std::max({c.hidden, c.n_q_heads * c.head_dim + c.hidden, p.KCd})
+                       : (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim, p.KCd});
   size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim;  // + cur K/V rows (bf16)
   size_t f = std::max(vec, attn);
   return (f + 31) / 32 * 32;
@@ -374,7 +376,6 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   const bool one_launch = o.exec_mode == MK_EXEC_MEGAKERNEL || o.exec_mode == MK_EXEC_MEGAKERNEL_GENERIC;
   if (!one_launch && o.sched_mode == MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
   if (o.kv_splits < 0 || o.num_sms < 0 || o.wait_timeout_ns < 0) return MK_ERR_INVALID_ARG;
-  if (o.batch > 1) return MK_ERR_UNSUPPORTED_SHAPE;  // batched instructions: not in this build yet
   cudaError_t ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) {
     cudaGetLastError();
@@ -390,7 +391,8 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
     fprintf(stderr, "mk_plan: %s\n", err.c_str());
     return MK_ERR_UNSUPPORTED_SHAPE;
   }
-  const int nb = 1;
+  // batched plans run the kernel instantiated for up to kMaxBatch sequences
+  const int nb = o.batch > 1 ? kMaxBatch : 1;
   const size_t act_floats = act_floats_for(h->cfg, p, nb);
   const int fixed = shared_bytes_fixed(0, act_floats);
   int num_pages = (h->smem_optin - fixed) / (kPageBytes + 16);
@@ -412,7 +414,8 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   sel.Ro = p.Ro;
   sel.Rd = p.Rd;
   int variant = 0;
-  const void *kernel = interp_kernel_for(sel, o.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC, &variant);
+  const void *kernel = interp_kernel_for(sel, o.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC, nb, &variant);
+  if (!kernel) return MK_ERR_UNSUPPORTED_SHAPE;  // batch > 1 without a batched build for this shape
   int per_sm = 0;
   cudaError_t e = interp_prepare(kernel, smem, &per_sm);
   if (e != cudaSuccess) {

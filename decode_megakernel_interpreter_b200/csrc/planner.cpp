@@ -98,11 +98,15 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   if (req.S > 0) {
     p.S = std::min(req.S, 256);
   } else {
-    // one attention item per CTA, but keep at least ~32 positions per split
+    // one attention item per CTA, but keep at least ~32 positions per split;
+    // when the sequences alone fill the CTAs (batched plans), still split
+    // long contexts up to ~4 items per CTA with >= 256 positions each, so
+    // that the longest sequence does not run on one CTA alone
     int items = req.B * s.nkv;
     int S = std::max(1, req.num_ctas / items);
     S = std::min(S, std::max(1, req.assumed_context / 32));
-    p.S = std::min(S, 64);
+    if (req.B > 1) S = std::max(S, std::min(4 * req.num_ctas / items, req.assumed_context / 256));
+    p.S = std::max(1, std::min(S, 64));
   }
   p.P_qkv = (s.nq + 2 * s.nkv) * s.d / p.Rh;
   p.P_o = s.H / p.Ro;
