@@ -259,7 +259,8 @@ size_t act_floats_for(const mk_config &c, const Plan &p, int nb) {
   // after it)
   size_t vec = nb == 1 ? (size_t)std::max({c.hidden, c.n_q_heads * c.head_dim + c.hidden, p.KCd})
                        : (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim, p.KCd});
-  size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim;  // + cur K/V rows (bf16)
+  // warps' partials + the current K/V rows (bf16) + the warps' merge weights
+  size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim + (size_t)G * (kComputeWarps + 2);
   size_t f = std::max(vec, attn);
   return (f + 31) / 32 * 32;
 }

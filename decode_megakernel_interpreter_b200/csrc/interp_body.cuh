@@ -192,6 +192,11 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
@@ -1467,25 +1472,39 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
     }
   }
   px::cbar();
+  // per head: the warps' weights exp(m_w - M) once (one thread per (head,
+  // warp), 8-lane groups of warp 0), then every output element sums the
+  // warps' contributions with them
+  float *fac = reinterpret_cast<float *>(cur + 2 * D);  // [G][warps] weights, then [G] M and [G] L
+  if (c.ctid < G * kComputeWarps) {
+    constexpr unsigned fm = (G * kComputeWarps >= 32) ? 0xffffffffu : ((1u << (G * kComputeWarps)) - 1u);
+    const int h = c.ctid / kComputeWarps, w = c.ctid % kComputeWarps;
+    const float *ws = scr + ((size_t)w * G + h) * (D + 2);
+    const float mw = ws[D];
+    float M = mw;
+#pragma unroll
+    for (int off = kComputeWarps / 2; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(fm, M, off));
+    const float f = (mw == -INFINITY) ? 0.f : expf(mw - M);
+    float L = f * ws[D + 1];
+#pragma unroll
+    for (int off = kComputeWarps / 2; off; off >>= 1) L += __shfl_xor_sync(fm, L, off);
+    fac[h * kComputeWarps + w] = f;
+    if (w == 0) {
+      fac[G * kComputeWarps + h] = M;
+      fac[G * kComputeWarps + G + h] = L;
+    }
+  }
+  px::cbar();
   const size_t hbase = ((size_t)l * p.B + b) * p.nq + (size_t)g * G;  // [l][b][head]
   for (int e = c.ctid; e < G * D; e += kComputeThreads) {
     const int h = e / D, dd = e % D;
-    float M = -INFINITY;
-    for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, scr[((size_t)w * G + h) * (D + 2) + D]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int w = 0; w < kComputeWarps; ++w) {
-        const float *ws = scr + ((size_t)w * G + h) * (D + 2);
-        const float mw = ws[D];
-        const float f = (mw == -INFINITY) ? 0.f : expf(mw - M);
-        L += f * ws[D + 1];
-        O += f * ws[dd];
-      }
-    }
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < kComputeWarps; ++w) O += fac[h * kComputeWarps + w] * scr[((size_t)w * G + h) * (D + 2) + dd];
     px::st_tf(p.part_o + ((hbase + h) * p.S + s) * D + dd, O, tag);
     if (dd == 0) {
-      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 0, M, tag);
-      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 1, L, tag);
+      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 0, fac[G * kComputeWarps + h], tag);
+      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 1, fac[G * kComputeWarps + G + h], tag);
     }
   }
   px::cbar();
@@ -1523,18 +1542,20 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
       for (int j = 0; j < SB; ++j) ov[e][j] = (idx < NE && j < S) ? px::ld_tf(p.part_o + ((hbase + h) * S + j) * D + dd) : 0u;
     }
     px::cbar();
-    if (c.ctid < G) {  // per head: max, weights exp(m_s - M), and the total weight L
-      const int h = c.ctid;
+    if (c.cw < G) {  // warp h: head h's max, weights exp(m_s - M) and total weight L, lanes over splits
+      const int h = c.cw;
       float M = -INFINITY;
-      for (int sp = 0; sp < S; ++sp) M = fmaxf(M, sml[2 * (h * S + sp)]);
+      for (int sp = c.lane; sp < S; sp += 32) M = fmaxf(M, sml[2 * (h * S + sp)]);
+      M = px::warp_max(M);
       float L = 0.f;
-      for (int sp = 0; sp < S; ++sp) {
+      for (int sp = c.lane; sp < S; sp += 32) {
         const float ms = sml[2 * (h * S + sp)];
         const float wgt = (ms == -INFINITY) ? 0.f : expf(ms - M);
         L += wgt * sml[2 * (h * S + sp) + 1];
         sml[2 * (h * S + sp)] = wgt;
       }
-      c.sh->red[h % kComputeWarps][h / kComputeWarps] = L;
+      L = px::warp_sum(L);
+      if (c.lane == 0) c.sh->red[h % kComputeWarps][h / kComputeWarps] = L;
     }
     px::cbar();
 #pragma unroll

@@ -150,7 +150,7 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   // shared memory geometry (as mk_plan)
   const int G = s.nq / s.nkv;
   size_t act = std::max(std::max((size_t)s.H, qd + (size_t)s.H), (size_t)p.KCd);
-  act = std::max(act, (size_t)kComputeWarps * G * (s.d + 2) + s.d);
+  act = std::max(act, (size_t)kComputeWarps * G * (s.d + 2) + s.d + (size_t)G * (kComputeWarps + 2));
   act = (act + 31) / 32 * 32;
   int num_pages = std::min(16, (slot->smem_optin - shared_bytes_fixed(0, act)) / (kPageBytes + 16));
   num_pages = num_pages / kLoaders * kLoaders;  // as mk_plan: unambiguous mbarrier phases
