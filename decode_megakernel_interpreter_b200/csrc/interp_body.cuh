@@ -928,6 +928,51 @@ __device__ __forceinline__ void mv_page(const uint8_t *page, const float *act, i
   for (int b = 0; b < NB; ++b)
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[b][r] = 0.f;
+  if constexpr (NB > 4) {
+    // many sequences: one pass over the page per group of 4 sequences, so
+    // that the running sums of a pass stay in registers (the page is read
+    // from shared memory once per group)
+#pragma unroll
+    for (int b0 = 0; b0 < NB; b0 += 4) {
+      if (b0 >= B) break;
+      float part[4][R];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int r = 0; r < R; ++r) part[i][r] = 0.f;
+#pragma unroll 1
+      for (int j = 0; j < CH / 32; ++j) {
+        const int ch = lane + 32 * j;
+        uint4 w[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) w[r] = pg[r * CH + ch];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (b0 + i >= B) break;
+          const float4 *a = reinterpret_cast<const float4 *>(act + (size_t)(b0 + i) * act_stride);
+          const float4 a0 = a[ch], a1 = a[CH + ch];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            float t = part[i][r];
+            t = fmaf(px::bf_lo(w[r].x), a0.x, t);
+            t = fmaf(px::bf_hi(w[r].x), a0.y, t);
+            t = fmaf(px::bf_lo(w[r].y), a0.z, t);
+            t = fmaf(px::bf_hi(w[r].y), a0.w, t);
+            t = fmaf(px::bf_lo(w[r].z), a1.x, t);
+            t = fmaf(px::bf_hi(w[r].z), a1.y, t);
+            t = fmaf(px::bf_lo(w[r].w), a1.z, t);
+            t = fmaf(px::bf_hi(w[r].w), a1.w, t);
+            part[i][r] = t;
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[b0 + i][r] = px::warp_sum(part[i][r]);
+    }
+    return;
+  }
 #pragma unroll(CH / 32 > 2 ? 2 : CH / 32)
   for (int j = 0; j < CH / 32; ++j) {
     const int ch = lane + 32 * j;
@@ -1647,6 +1692,10 @@ constexpr unsigned kSpeculativeOps = MK_SPECULATIVE_OPS;
 template <int NB, class S>
 __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile int *dyn_tail,
                             volatile int *dyn_head) {
+  // op bodies inline in the loop for the batch-1 shape builds; a batched
+  // build calls them (each body alone fits the register budget, the loop
+  // holding all six would spill)
+  constexpr bool kInline = S::fixed && NB == 1;
   const KParams &p = c.p;
   const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
   const bool trace = (p.mode & MODE_TRACE) != 0;
@@ -1703,27 +1752,33 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
     c.tr = tr;
     switch (I.op) {
       case OP_QKV:
-        if constexpr (S::fixed) c.g = qkv_body<NB, S::RH>(c, I);
+        if constexpr (kInline) c.g = qkv_body<NB, S::RH>(c, I);
+        else if constexpr (S::fixed) c.g = op_qkv<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_qkv, NB, p.Rh, c, I);
         break;
       case OP_ATTN:
-        if constexpr (S::fixed) c.g = attn_body<S::G, S::DPL>(c, I);
+        if constexpr (kInline) c.g = attn_body<S::G, S::DPL>(c, I);
+        else if constexpr (S::fixed) c.g = op_attn_t<S::G, S::DPL>(c, I);
         else c.g = op_attn(c, I);
         break;
       case OP_OPROJ:
-        if constexpr (S::fixed) c.g = oproj_body<NB, S::RO>(c, I);
+        if constexpr (kInline) c.g = oproj_body<NB, S::RO>(c, I);
+        else if constexpr (S::fixed) c.g = op_oproj<NB, S::RO>(c, I);
         else MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);
         break;
       case OP_GATEUP:
-        if constexpr (S::fixed) c.g = gateup_body<NB, S::RH>(c, I);
+        if constexpr (kInline) c.g = gateup_body<NB, S::RH>(c, I);
+        else if constexpr (S::fixed) c.g = op_gateup<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_gateup, NB, p.Rh, c, I);
         break;
       case OP_DOWN:
-        if constexpr (S::fixed) c.g = down_body<NB, S::RD>(c, I);
+        if constexpr (kInline) c.g = down_body<NB, S::RD>(c, I);
+        else if constexpr (S::fixed) c.g = op_down<NB, S::RD>(c, I);
         else MK_DISPATCH_R(op_down, NB, p.Rd, c, I);
         break;
       case OP_LMHEAD:
-        if constexpr (S::fixed) c.g = lmhead_body<NB, S::RH>(c, I);
+        if constexpr (kInline) c.g = lmhead_body<NB, S::RH>(c, I);
+        else if constexpr (S::fixed) c.g = op_lmhead<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I);
         break;
       default: break;
