@@ -806,12 +806,15 @@ __device__ __forceinline__ float4 ll_load4(uint32_t tag, const float *a, bool &o
   return tf_chk4(px::ld_tf4(a), tag, ok);
 }
 
-// Stage rms(x)*gamma for every sequence, x = layer_input(l) (l == L: final norm).
-// Contains two compute barriers.
+// Stage x*gamma for every sequence, x = layer_input(l) (l == L: final norm),
+// and return inv[b] = 1 / rms(x_b): the consumer scales its dot products,
+// since W (x*gamma*inv) == (W (x*gamma)) * inv, so the matrix-vector pages
+// need not wait for a second pass over the staged vector.  One compute
+// barrier.
 // IT = float4 loads per thread (H / 4 / 256, at least 1), fixed by the caller's
 // rows-per-page so that every load is issued before the first one is used.
 template <int NB, int IT>
-__device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only) {
+__device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only, float (&inv)[NB]) {
   const KParams &p = c.p;
   const int H = p.H, n4 = H / 4;
   float ss[NB];
@@ -840,8 +843,10 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
       const int e4 = c.ctid + it * kComputeThreads;
       if (e4 < n4) {
         const float4 x = xs[it];
+        const uint2 gw = gws[it];
         ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-        dst[stage_slot4(e4, H)] = x;
+        dst[stage_slot4(e4, H)] =
+            make_float4(x.x * px::bf_lo(gw.x), x.y * px::bf_hi(gw.x), x.z * px::bf_lo(gw.y), x.w * px::bf_hi(gw.y));
       }
     }
   }
@@ -851,7 +856,6 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
     if (c.lane == 0) c.sh->red[c.cw][b] = v;
   }
   px::cbar();
-  float inv[NB];
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     float t = 0.f;
@@ -859,24 +863,6 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
     for (int w = 0; w < kComputeWarps; ++w) t += c.sh->red[w][b];
     inv[b] = __frsqrt_rn(t * p.inv_H + p.eps);  // one rounding; t * (1/H) == t / H for H = 2^k
   }
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    if (b >= p.B) break;
-    float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
-#pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      const int e4 = c.ctid + it * kComputeThreads;
-      if (e4 >= n4) break;
-      const uint2 gw = gws[it];
-      float4 x = dst[stage_slot4(e4, H)];
-      x.x = x.x * inv[b] * px::bf_lo(gw.x);
-      x.y = x.y * inv[b] * px::bf_hi(gw.x);
-      x.z = x.z * inv[b] * px::bf_lo(gw.y);
-      x.w = x.w * inv[b] * px::bf_hi(gw.y);
-      dst[stage_slot4(e4, H)] = x;
-    }
-  }
-  px::cbar();
   if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
 }
 
@@ -1052,7 +1038,8 @@ __device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
   const int l = I.layer;
   const int half = R / 2, pph = p.d / R, hd = p.d / 2;
   const int pos0 = read_pos(c.sh, 0);
-  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].attn_norm, false);
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].attn_norm, false, inv);
   const int nq = p.nq, nkv = p.nkv, d = p.d, lane = c.lane, Bn = p.B, kvdim = p.kvdim;
   const uint32_t tag = c.epoch;
   float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
@@ -1069,7 +1056,7 @@ __device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       if (NB > 1 && b >= Bn) break;
-      float u = pick<R>(acc[b], lane), w = pick<R>(acc[b], lane + half);
+      float u = pick<R>(acc[b], lane) * inv[b], w = pick<R>(acc[b], lane + half) * inv[b];
       const int pos = NB == 1 ? pos0 : read_pos(c.sh, b);
       if (head < nq + nkv) {
         const float2 cs = NB == 1 ? rope_s[i] : __ldg(rope_g + (size_t)pos * hd + i);
@@ -1132,7 +1119,8 @@ template <int NB, int R>
 __device__ __forceinline__ uint32_t gateup_body(CCtx c, const Instr I) {
   const KParams &p = c.p;
   const int l = I.layer;
-  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].ffn_norm, true);
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].ffn_norm, true, inv);
   const int half = R / 2, lane = c.lane, Bn = p.B, F = p.F;
   const uint32_t tag = c.epoch;
   float *const aout = p.actb + (size_t)l * Bn * F;
@@ -1142,7 +1130,7 @@ __device__ __forceinline__ uint32_t gateup_body(CCtx c, const Instr I) {
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       if (NB > 1 && b >= Bn) break;
-      const float gt = pick<R>(acc[b], lane), up = pick<R>(acc[b], lane + half);
+      const float gt = pick<R>(acc[b], lane) * inv[b], up = pick<R>(acc[b], lane + half) * inv[b];
       const float silu = gt / (1.0f + expf(-gt));
       px::st_tf(aout + (size_t)b * F + row, silu * up, tag);
     }
@@ -1181,7 +1169,8 @@ __device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi) {
 template <int NB, int R>
 __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
   const KParams &p = c.p;
-  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false);
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false, inv);
   float bv[NB];
   int bi[NB];
 #pragma unroll
@@ -1197,7 +1186,7 @@ __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       if (NB > 1 && b >= Bn) break;
-      const float v = pick<R>(acc[b], lane);
+      const float v = pick<R>(acc[b], lane) * inv[b];
       if (valid) {
         if (logits) logits[(size_t)b * V + row] = v;
         if (arg_better(v, row, bv[b], bi[b])) {
