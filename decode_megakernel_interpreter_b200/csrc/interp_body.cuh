@@ -1418,7 +1418,11 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   // split holding the current position, that position's K and V rows (this
   // step's QKV wrote them as tagged words): one group of loads
   const uint32_t tag = c.epoch;
-  const bool load_cur = r.has_cur && c.cw == 0;
+  // the current position's row goes to the first warp with less than a full
+  // share of the last cached page (often none), not to an already loaded warp
+  const int last_cnt = npg > 0 ? (r.pref_end - r.start) - (npg - 1) * PPP : 0;
+  const int cur_warp = min(kComputeWarps - 1, last_cnt / PW);
+  const bool load_cur = r.has_cur && c.cw == cur_warp;
   const float *kcur = p.kvcur + (((size_t)l * p.B + b) * 2) * p.kvdim + (size_t)g * D;
   const float *vcur = kcur + p.kvdim;
   const float *qb = p.qbuf + ((size_t)l * p.B + b) * p.qdim + (size_t)g * G * D;
@@ -1490,7 +1494,7 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   }
   c.g += npg;
   __syncwarp();
-  if (r.has_cur && c.cw == 0 && !c.sh->abort) {
+  if (load_cur && !c.sh->abort) {
     // one valid position; the block reads PW rows, rows past the first are masked
     attn_block<G, DPL, PB>(q, cur, cur + D, 1, c.lane, m, lsum, o);
   }
