@@ -166,6 +166,22 @@ def step_bytes(shape, weight_bytes: int, positions, logits: bool) -> float:
     return tot / len(positions)
 
 
+def max_over_ranks(ms: float, pg, device: str) -> float:
+    """The job's time: the slowest rank's (every rank takes part; `pg` is
+    torch.distributed or None for a single process)."""
+    if pg is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank's steps over the job's time."""
+    return world * steps / (ms / 1e3)
+
+
 def dist_setup(n):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -346,12 +362,9 @@ def main():
     rc = eng.status()
     if rc != mk.MK_OK:
         raise mk.MkError(rc, "timed steps")
-    if pg:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, pg, "cuda")
     us_step = 1e3 * ms / K
-    value = world * K / (ms / 1e3)
+    value = job_rate(world, K, ms)
     launches_per_step = 1 if args.exec_mode.startswith("megakernel") else s.n_layers * 5 + 1
 
     # end to end through the C ABI with host buffers: per step copy the token
@@ -384,11 +397,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1)
-        if pg:
-            t = torch.tensor([ems], dtype=torch.float64, device="cuda")
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * K / (ems / 1e3), "unit": "steps/s", "h2d_bytes_per_step": 8 * B,
+        ems = max_over_ranks(ems, pg, "cuda")
+        e2e = {"value": job_rate(world, K, ems), "unit": "steps/s", "h2d_bytes_per_step": 8 * B,
                "d2h_bytes_per_step": 4 * B, "us_per_step": 1e3 * ems / K}
 
     bd = breakdown(eng, mk, info, tokens, pos_all[0], logits, torch.empty_like(tokens)) if args.breakdown else None
