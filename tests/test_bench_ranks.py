@@ -68,9 +68,8 @@ def test_gpus_flag_must_match_the_launcher(monkeypatch):
 def test_reference_arm_runs_on_rank_0_only(capsys):
     """Under torchrun the CPU reference runs once: ranks other than 0 return
     at once and print nothing."""
-    b = _bench()
-    args = b.parse.__wrapped__() if hasattr(b.parse, "__wrapped__") else None
     import argparse
+    b = _bench()
     ns = argparse.Namespace(workload="tiny", steps=1, warmup=0, gpus=2)
     assert b.run_reference(ns, 2, 1) is None
     assert capsys.readouterr().out == ""
