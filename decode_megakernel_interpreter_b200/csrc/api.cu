@@ -114,6 +114,37 @@ __global__ void gather_rows_kernel(uint16_t *dst, const unsigned long long *src_
   }
 }
 
+// The LM head as 128-row tiles for the tensor cores: tile (block, kb) is one
+// 16 KiB page of 64 columns, stored as 8 column chunks of 128 rows x 8 bf16
+// (16-byte rows); rows past the vocabulary are zero.
+__global__ void tile_lm_kernel(uint16_t *dst, const uint16_t *src, int V, int H, long long n16) {
+  const int kpb = H / 64;
+  const bool aligned = ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n16; u += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(u % 128);
+    long long t = u / 128;
+    const int ch = (int)(t % 8);
+    t /= 8;
+    const int kb = (int)(t % kpb);
+    const long long blk = t / kpb;
+    const long long row = blk * 128 + r;
+    const long long col = (long long)kb * 64 + ch * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < V) {
+      const uint16_t *sp = src + row * H + col;
+      if (aligned) {
+        v = *reinterpret_cast<const uint4 *>(sp);
+      } else {
+        uint16_t e[8];
+        for (int i = 0; i < 8; ++i) e[i] = sp[i];
+        v = make_uint4(e[0] | ((uint32_t)e[1] << 16), e[2] | ((uint32_t)e[3] << 16), e[4] | ((uint32_t)e[5] << 16),
+                       e[6] | ((uint32_t)e[7] << 16));
+      }
+    }
+    reinterpret_cast<uint4 *>(dst)[u] = v;
+  }
+}
+
 int gather_rows(uint16_t *dst, const std::vector<unsigned long long> &src, int row_elems) {
   if (src.empty()) return MK_OK;
   unsigned long long *d_src = nullptr;
@@ -229,6 +260,7 @@ PlanRequest make_request(const mk_config &c, const mk_plan_opts &o, int num_ctas
   r.dynamic = o.sched_mode == MK_SCHED_DYNAMIC;
   r.assumed_context = std::max(1, c.max_seq);
   r.drop_producer = o.debug_drop_producer != 0;
+  r.lm_tensor = o.batch > 1;  // batched plans run the LM head on the tensor cores
   return r;
 }
 
@@ -486,6 +518,20 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   k.layers = h->d_layers;
   k.embed = h->embed;
   k.lm_head = h->lm_head;
+  k.lm_tc = nullptr;
+  k.lm_ppb = s.H / 64;
+  if (p.lm_tensor) {
+    // the tensor-core LM head reads a tiled copy (plan-owned)
+    const long long blocks = (s.V + 127) / 128, n16 = blocks * 128 * (s.H / 8);
+    uint16_t *tiles = nullptr;
+    if ((rc = dalloc(h->plan_allocs, &tiles, (size_t)n16 * 8, false))) return rc;
+    tile_lm_kernel<<<4 * h->sm_count, 256>>>(tiles, h->lm_head, s.V, s.H, n16);
+    if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
+    k.lm_tc = tiles;
+  }
   k.final_norm = h->final_norm;
   k.kc = h->kc;
   k.vc = h->vc;

@@ -80,6 +80,44 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       "l"(src), "r"(bytes), "r"(sa(bar)), "l"(policy)
       : "memory");
 }
+// ---- 5th-generation tensor cores (tcgen05): MMA with the accumulator in
+// tensor memory.  Shared-memory operands use the K-major layout without
+// swizzle: 16-byte rows of 8 bf16, 8-row groups `sbo` bytes apart, the two
+// 8-element K chunks of one MMA `lbo` bytes apart.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);  // version 1, no swizzle
+}
+// D (f32) += A (bf16, M x 16, K-major) * B (bf16, N x 16, K-major)^T; one thread issues.
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+// arrive on `bar` once every MMA this thread issued so far has completed
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(sa(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// 16 consecutive f32 columns of this warp's 32 tensor-memory lanes
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -220,6 +258,11 @@ struct Shared {
   uint32_t dep_ctr, dep_target;
   int dep_seq;
   int dep_state;   // 0: not checked, 1: a thread is polling, 2: met, 3: failed
+  // tensor-core LM head (batched builds): tensor-memory columns, the MMA
+  // completion barrier and how many times it has completed
+  uint32_t tmem_base;
+  uint32_t mma_phase;
+  unsigned long long mma_bar;
   uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
   float red[kComputeWarps][kMaxBatch];
   float argv[kComputeWarps][kMaxBatch];
@@ -451,6 +494,11 @@ __device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, 
     case OP_GATEUP: s.a = p.layers[I.layer].wgu + (size_t)I.a * kPageElems; break;
     case OP_DOWN: s.a = p.layers[I.layer].wd + ((size_t)I.c * (p.H / p.Rd) + I.a) * kPageElems; break;
     case OP_LMHEAD: {
+      if (p.lm_tc) {  // whole 128-row tiles, ppb pages each
+        s.a = p.lm_tc + (size_t)I.a * p.lm_ppb * kPageElems;
+        s.npg = (int)I.b * p.lm_ppb;
+        break;
+      }
       s.a = p.lm_head + (size_t)I.a * p.Rh * p.H;
       const int r_last = (int)(I.a + I.b - 1) * p.Rh;
       s.last = (uint32_t)min(p.Rh, p.V - r_last) * p.H * 2;
@@ -813,7 +861,20 @@ __device__ __forceinline__ float4 ll_load4(uint32_t tag, const float *a, bool &o
 // barrier.
 // IT = float4 loads per thread (H / 4 / 256, at least 1), fixed by the caller's
 // rows-per-page so that every load is issued before the first one is used.
-template <int NB, int IT>
+// bf16 pair (hi, lo) with hi + lo == x to about 16 significant bits: the
+// tensor-core path multiplies bf16 weights by both halves of each activation
+__device__ __forceinline__ void split_bf16x4(float4 x, uint16_t *hi, uint16_t *lo) {
+  const uint16_t h0 = px::f2bf(x.x), h1 = px::f2bf(x.y), h2 = px::f2bf(x.z), h3 = px::f2bf(x.w);
+  const uint16_t l0 = px::f2bf(x.x - px::bf16f(h0)), l1 = px::f2bf(x.y - px::bf16f(h1)),
+                 l2 = px::f2bf(x.z - px::bf16f(h2)), l3 = px::f2bf(x.w - px::bf16f(h3));
+  *reinterpret_cast<uint2 *>(hi) = make_uint2((uint32_t)h0 | ((uint32_t)h1 << 16), (uint32_t)h2 | ((uint32_t)h3 << 16));
+  *reinterpret_cast<uint2 *>(lo) = make_uint2((uint32_t)l0 | ((uint32_t)l1 << 16), (uint32_t)l2 | ((uint32_t)l3 << 16));
+}
+
+// TC: stage x*gamma as bf16 (hi, lo) in the tensor cores' K-major layout
+// instead: 8-element chunk ch of sequence b at byte ((ch * 16) + b) * 16 of
+// the hi block (H * 32 bytes), the lo block right after it.
+template <int NB, int IT, bool TC = false>
 __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only, float (&inv)[NB]) {
   const KParams &p = c.p;
   const int H = p.H, n4 = H / 4;
@@ -845,8 +906,15 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
         const float4 x = xs[it];
         const uint2 gw = gws[it];
         ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-        dst[stage_slot4(e4, H)] =
+        const float4 xg =
             make_float4(x.x * px::bf_lo(gw.x), x.y * px::bf_hi(gw.x), x.z * px::bf_lo(gw.y), x.w * px::bf_hi(gw.y));
+        if constexpr (TC) {
+          uint16_t *hi = reinterpret_cast<uint16_t *>(c.act);
+          const size_t o = ((size_t)(e4 >> 1) * 16 + b) * 8 + (e4 & 1) * 4;
+          split_bf16x4(xg, hi + o, hi + (size_t)H * 16 + o);
+        } else {
+          dst[stage_slot4(e4, H)] = xg;
+        }
       }
     }
   }
@@ -1166,36 +1234,12 @@ __device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-template <int NB, int R>
-__device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
+// The LM-head instruction's argmax: per thread (bv, bi) of each sequence ->
+// per warp -> per CTA (the instruction's tagged slot); the last LM instruction
+// to finish merges every slot and writes the next tokens.
+template <int NB>
+__device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&bv)[NB], int (&bi)[NB]) {
   const KParams &p = c.p;
-  float inv[NB];
-  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false, inv);
-  float bv[NB];
-  int bi[NB];
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    bv[b] = -INFINITY;
-    bi[b] = 0x7fffffff;
-  }
-  const int lane = c.lane, Bn = p.B, V = p.V;
-  float *const logits = p.logits;
-  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    const int row = j * R + lane;
-    const bool valid = lane < R && row < V;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      if (NB > 1 && b >= Bn) break;
-      const float v = pick<R>(acc[b], lane) * inv[b];
-      if (valid) {
-        if (logits) logits[(size_t)b * V + row] = v;
-        if (arg_better(v, row, bv[b], bi[b])) {
-          bv[b] = v;
-          bi[b] = row;
-        }
-      }
-    }
-  });
   // CTA-wide argmax of this instruction
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
@@ -1285,8 +1329,131 @@ __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
       p.next_tokens[b] = (i == 0x7fffffff) ? 0 : i;
     }
   }
+}
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false, inv);
+  float bv[NB];
+  int bi[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    bv[b] = -INFINITY;
+    bi[b] = 0x7fffffff;
+  }
+  const int lane = c.lane, Bn = p.B, V = p.V;
+  float *const logits = p.logits;
+  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    const int row = j * R + lane;
+    const bool valid = lane < R && row < V;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (NB > 1 && b >= Bn) break;
+      const float v = pick<R>(acc[b], lane) * inv[b];
+      if (valid) {
+        if (logits) logits[(size_t)b * V + row] = v;
+        if (arg_better(v, row, bv[b], bi[b])) {
+          bv[b] = v;
+          bi[b] = row;
+        }
+      }
+    }
+  });
+  lm_argmax_tail<NB>(c, I, bv, bi);
   return c.g;
 }
+
+// LM head on the tensor cores (batched builds): the weight is in 128-row
+// tiles of 64 columns per 16 KiB page (K-major, no swizzle), an instruction
+// covers whole 128-row blocks, and every block accumulates
+// D[128 rows][16 sequences] (f32, tensor memory) over the block's pages with
+// two MMAs per 16 columns (the activations' bf16 hi and lo halves).  One
+// thread issues the MMAs and recycles each page once its MMAs completed;
+// four warps (one per quarter of the tensor-memory lanes) read the block's
+// logits.  A dense contraction at 16 sequences: about 16 flops per weight
+// byte.
+template <int NB, int R>
+__device__ __forceinline__ uint32_t lmhead_tc_body(CCtx c, const Instr I) {
+  static_assert(NB == 16, "the MMA's N is the batch slot count");
+  const KParams &p = c.p;
+  const int H = p.H, V = p.V, Bn = p.B, ppb = p.lm_ppb;
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v, true>(c, p.L, p.final_norm, false, inv);
+  px::fence_proxy_async_smem();  // the staged operand, written by the generic proxy, is read by the MMAs
+  px::cbar();
+  const uint32_t hi_s = px::sa(c.act), lo_s = hi_s + (uint32_t)H * 32u;
+  // D f32, A and B bf16, both K-major, N = 16, M = 128
+  constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+  const uint32_t tmem = c.sh->tmem_base;
+  const Ring rg = ring_of(c);
+  // the warps whose tensor-memory lane quarter is (warp % 4)
+  const int warp = c.cw + kLoaders, quarter = warp & 3;
+  const bool reader = c.cw >= 2 && c.cw < 6;
+  float bv[NB];
+  int bi[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    bv[b] = -INFINITY;
+    bi[b] = 0x7fffffff;
+  }
+  const int nblk = (int)I.b;
+  for (int blk = 0; blk < nblk; ++blk) {
+    if (c.ctid == 0) {
+      for (int kb = 0; kb < ppb; ++kb) {
+        const uint32_t g = c.g + (uint32_t)(blk * ppb + kb);
+        if (!ring_wait(p, rg, g)) break;
+        const uint32_t pg = px::sa(ring_page(rg, g));
+        px::tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t a = px::umma_desc(pg + ks * 4096u, 2048u, 128u);
+          const uint32_t boff = (uint32_t)(kb * 8 + 2 * ks) * 256u;
+          px::umma_bf16(tmem, a, px::umma_desc(hi_s + boff, 256u, 128u), kIdesc, kb > 0 || ks > 0);
+          px::umma_bf16(tmem, a, px::umma_desc(lo_s + boff, 256u, 128u), kIdesc, true);
+        }
+        // the page is free once its MMAs have read it
+        px::umma_commit(reinterpret_cast<uint64_t *>(&c.sh->mma_bar));
+        const uint32_t ph = c.sh->mma_phase & 1u;
+        c.sh->mma_phase += 1u;
+        if (!wait_bar(p, c.sh, reinterpret_cast<uint64_t *>(&c.sh->mma_bar), ph, 6)) {
+          c.sh->abort = 1;
+          break;
+        }
+        ring_release(rg, g, kComputeWarps);
+      }
+      px::tc_fence_before();
+    }
+    // every MMA of the block has completed (thread 0 waited for each page's)
+    if (px::cbar_or(px::ld_volatile(&c.sh->abort) != 0)) break;
+    px::tc_fence_after();
+    if (reader) {
+      float v[16];
+      px::tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16), v);
+      const int row = ((int)I.a + blk) * 128 + quarter * 32 + c.lane;
+      if (row < V) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= Bn) break;
+          const float x = v[b] * inv[b];
+          if (p.logits) p.logits[(size_t)b * V + row] = x;
+          if (arg_better(x, row, bv[b], bi[b])) {
+            bv[b] = x;
+            bi[b] = row;
+          }
+        }
+      }
+    }
+    px::tc_fence_before();
+    px::cbar();  // the block's logits are read before the next block's MMAs overwrite them
+  }
+  c.g += (uint32_t)(nblk * ppb);
+  lm_argmax_tail<NB>(c, I, bv, bi);
+  return c.g;
+}
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_lmhead_tc(CCtx c, const Instr I) { return lmhead_tc_body<NB, R>(c, I); }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_lmhead(CCtx c, const Instr I) { return lmhead_body<NB, R>(c, I); }
 
@@ -1770,6 +1937,12 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         else MK_DISPATCH_R(op_down, NB, p.Rd, c, I);
         break;
       case OP_LMHEAD:
+        if constexpr (NB > 1 && S::fixed) {
+          if (p.lm_tc) {
+            c.g = op_lmhead_tc<NB, S::RH>(c, I);
+            break;
+          }
+        }
         if constexpr (kInline) c.g = lmhead_body<NB, S::RH>(c, I);
         else if constexpr (S::fixed) c.g = op_lmhead<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I);
@@ -1816,6 +1989,8 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
       px::mbar_init(&full[i], 1);
       px::mbar_init(&empty[i], kComputeWarps);
     }
+    px::mbar_init(reinterpret_cast<uint64_t *>(&sh->mma_bar), 1);
+    sh->mma_phase = 0;
     px::fence_mbar_init();
     sh->abort = 0;
     sh->flag = 0;
@@ -1835,7 +2010,17 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   }
   __syncthreads();
   if (threadIdx.x < (unsigned)(p.d / 2)) sh->rope[threadIdx.x] = __ldg(p.rope + (size_t)sh->pos[0] * (p.d / 2) + threadIdx.x);
+  if constexpr (NB > 1) {
+    // tensor memory for the LM head's accumulators (32 columns: 16 used)
+    if (warp == kLoaders) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 32;" ::"r"(px::sa(&sh->tmem_base))
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    px::tc_fence_before();
+  }
   __syncthreads();
+  if constexpr (NB > 1) px::tc_fence_after();
   const unsigned epoch = *reinterpret_cast<volatile unsigned *>(p.epoch);
   Queue q;
   q.base = p.instrs + p.q_off[blockIdx.x];
@@ -1850,7 +2035,13 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
            (int)threadIdx.x - 32 * kLoaders, 0u, nullptr};
     run_compute<NB, S>(c, q, dyn_fifo, dyn_tail, dyn_head);
   }
+  if constexpr (NB > 1) px::tc_fence_before();
   __syncthreads();
+  if constexpr (NB > 1) {
+    px::tc_fence_after();
+    if (warp == kLoaders)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 32;" ::"r"(sh->tmem_base) : "memory");
+  }
   if (threadIdx.x == 0) {
     // every bulk copy must land before the CTA exits: after an abort the
     // compute warps stop consuming pages, so wait on each slot's latest use

@@ -97,6 +97,10 @@ struct KParams {
   int max_seq;
   float eps, attn_scale;
   float inv_H;                     // 1 / hidden (exact: hidden is a power of two)
+  // batched plans: the LM head in 128-row tensor-core tiles (64 columns per
+  // page, K-major without swizzle) and the pages per tile; null otherwise
+  const uint16_t *lm_tc;
+  int lm_ppb;
   // weights
   const LayerDev *layers;
   const LayerRaw *layers_raw;  // only read by the raw-layout kernel variant

@@ -220,8 +220,12 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
     }
     (void)total;
   }
-  // final RMSNorm + LM head + argmax
-  auto cl = split_even(p.P_lm, parts);
+  // final RMSNorm + LM head + argmax (units: pages of R rows, or 128-row
+  // blocks of H / 64 pages on the tensor-core path)
+  p.lm_tensor = req.lm_tensor;
+  const int lm_units = p.lm_tensor ? (s.V + 127) / 128 : p.P_lm;
+  const int64_t lm_unit_bytes = p.lm_tensor ? (int64_t)(s.H / 64) * kPageBytes : kPageBytes;
+  auto cl = split_even(lm_units, parts);
   p.n_lm = (int)cl.size();
   for (size_t i = 0; i < cl.size(); ++i) {
     Instr I = mk_instr(OP_LMHEAD, s.L);
@@ -230,7 +234,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
     I.c = (uint32_t)i;
     I.wait_ctr = p.ctr_dn(s.L - 1);
     I.wait_cnt = n_down[s.L - 1];
-    all.push_back({I, (int64_t)cl[i].count * kPageBytes, s.L * 8 + ST_QKV + 0, (int)i});
+    all.push_back({I, (int64_t)cl[i].count * lm_unit_bytes, s.L * 8 + ST_QKV + 0, (int)i});
   }
   // the LM head sorts after every layer
   for (auto &x : all)
@@ -244,11 +248,11 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   for (size_t i = 0; i < all.size(); ++i) all[i].ins.seq = (uint16_t)i;
   for (auto &x : all) {
     if (x.ins.op >= OP_QKV && x.ins.op <= OP_LMHEAD && x.ins.op != OP_ATTN)
-      p.weight_bytes += (int64_t)x.ins.b * kPageBytes;
+      p.weight_bytes += (int64_t)x.ins.b * (x.ins.op == OP_LMHEAD ? lm_unit_bytes : kPageBytes);
   }
-  // the last LM page may be partial
+  // the last LM page (or block) may be partial
   {
-    int64_t full = (int64_t)p.P_lm * kPageBytes, real = (int64_t)s.V * s.H * 2;
+    int64_t full = (int64_t)lm_units * lm_unit_bytes, real = (int64_t)s.V * s.H * 2;
     p.weight_bytes -= full - real;
   }
 

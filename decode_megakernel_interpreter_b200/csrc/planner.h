@@ -25,11 +25,15 @@ struct PlanRequest {
   int dyn_chunks_per_cta = 2;  // dynamic mode: instructions per CTA per matvec stage
   int assumed_context = 1024;  // for the automatic split count
   bool drop_producer = false;  // test hook (see mk_plan_opts)
+  // LM head on the tensor cores (batched plans): instructions cover whole
+  // 128-row blocks of a tiled copy of the LM head, H / 64 pages per block
+  bool lm_tensor = false;
 };
 
 struct Plan {
   // geometry
   int Rh = 0, Ro = 0, Rd = 0, KCd = 0, ndp = 0, S = 0;
+  bool lm_tensor = false;  // see PlanRequest
   int P_qkv = 0, P_o = 0, P_gu = 0, P_dp = 0, P_lm = 0;  // pages per layer / piece / head
   // instructions: static mode = per-CTA queues back to back; dynamic = global order
   std::vector<Instr> instrs;
