@@ -145,6 +145,51 @@ __global__ void tile_lm_kernel(uint16_t *dst, const uint16_t *src, int V, int H,
   }
 }
 
+// One 16-byte unit of a tensor-core tile copy (row `row` of a matrix with
+// row stride ld elements, columns col..col+7), zero past `rows`.
+__device__ __forceinline__ uint4 tile_unit(const uint16_t *src, long long row, long long rows, long long ld,
+                                           long long col) {
+  if (row >= rows) return make_uint4(0, 0, 0, 0);
+  const uint16_t *sp = src + row * ld + col;
+  if ((reinterpret_cast<uintptr_t>(sp) & 15) == 0) return *reinterpret_cast<const uint4 *>(sp);
+  uint16_t e[8];
+  for (int i = 0; i < 8; ++i) e[i] = sp[i];
+  return make_uint4(e[0] | ((uint32_t)e[1] << 16), e[2] | ((uint32_t)e[3] << 16), e[4] | ((uint32_t)e[5] << 16),
+                    e[6] | ((uint32_t)e[7] << 16));
+}
+// gate/up tiles: tile t = gate rows 64t..64t+63 then up rows 64t..64t+63;
+// page kb = columns 64kb..64kb+63 as 8 chunks of 128 rows x 8 bf16
+__global__ void tile_gu_kernel(uint16_t *dst, const uint16_t *gate, const uint16_t *up, int F, int H, long long n16) {
+  const int kpt = H / 64;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n16; u += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(u % 128);
+    long long t = u / 128;
+    const int ch = (int)(t % 8);
+    t /= 8;
+    const int kb = (int)(t % kpt);
+    const long long tile = t / kpt;
+    const long long col = (long long)kb * 64 + ch * 8;
+    reinterpret_cast<uint4 *>(dst)[u] =
+        r < 64 ? tile_unit(gate, tile * 64 + r, F, H, col) : tile_unit(up, tile * 64 + r - 64, F, H, col);
+  }
+}
+// down tiles: piece k (columns k*KCd..), row tile rt (rows 128rt..), page kb
+__global__ void tile_down_kernel(uint16_t *dst, const uint16_t *wd, int H, int F, int KCd, long long n16) {
+  const int kpt = KCd / 64, rts = H / 128;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n16; u += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(u % 128);
+    long long t = u / 128;
+    const int ch = (int)(t % 8);
+    t /= 8;
+    const int kb = (int)(t % kpt);
+    t /= kpt;
+    const int rt = (int)(t % rts);
+    const long long k = t / rts;
+    reinterpret_cast<uint4 *>(dst)[u] =
+        tile_unit(wd, (long long)rt * 128 + r, H, F, k * KCd + (long long)kb * 64 + ch * 8);
+  }
+}
+
 int gather_rows(uint16_t *dst, const std::vector<unsigned long long> &src, int row_elems) {
   if (src.empty()) return MK_OK;
   unsigned long long *d_src = nullptr;
@@ -260,7 +305,7 @@ PlanRequest make_request(const mk_config &c, const mk_plan_opts &o, int num_ctas
   r.dynamic = o.sched_mode == MK_SCHED_DYNAMIC;
   r.assumed_context = std::max(1, c.max_seq);
   r.drop_producer = o.debug_drop_producer != 0;
-  r.lm_tensor = o.batch > 1;  // batched plans run the LM head on the tensor cores
+  r.tensor = o.batch > 1;  // batched plans run gate/up, down and the LM head on the tensor cores
   return r;
 }
 
@@ -519,18 +564,37 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   k.embed = h->embed;
   k.lm_head = h->lm_head;
   k.lm_tc = nullptr;
-  k.lm_ppb = s.H / 64;
-  if (p.lm_tensor) {
-    // the tensor-core LM head reads a tiled copy (plan-owned)
-    const long long blocks = (s.V + 127) / 128, n16 = blocks * 128 * (s.H / 8);
-    uint16_t *tiles = nullptr;
-    if ((rc = dalloc(h->plan_allocs, &tiles, (size_t)n16 * 8, false))) return rc;
-    tile_lm_kernel<<<4 * h->sm_count, 256>>>(tiles, h->lm_head, s.V, s.H, n16);
+  if (p.tensor) {
+    // the tensor-core instructions read tiled copies (plan-owned): LM head,
+    // and per layer gate/up and down, with a plan-owned layer table
+    const int grid = 4 * h->sm_count;
+    const long long lm16 = (long long)((s.V + 127) / 128) * 128 * (s.H / 8);
+    const long long gu16 = (long long)(s.F / 64) * 128 * (s.H / 8);
+    const long long dn16 = (long long)s.H * (s.F / 8);
+    uint16_t *lm_t = nullptr, *gu_t = nullptr, *dn_t = nullptr;
+    if ((rc = dalloc(h->plan_allocs, &lm_t, (size_t)lm16 * 8, false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &gu_t, (size_t)gu16 * 8 * s.L, false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &dn_t, (size_t)dn16 * 8 * s.L, false))) return rc;
+    tile_lm_kernel<<<grid, 256>>>(lm_t, h->lm_head, s.V, s.H, lm16);
+    std::vector<LayerDev> ld(s.L);
+    MK_CUDA(cudaMemcpy(ld.data(), h->d_layers, sizeof(LayerDev) * s.L, cudaMemcpyDeviceToHost));
+    for (int l = 0; l < s.L; ++l) {
+      const mk_layer_weights &W = h->lw[l];
+      uint16_t *gl = gu_t + (size_t)gu16 * 8 * l, *dl = dn_t + (size_t)dn16 * 8 * l;
+      tile_gu_kernel<<<grid, 256>>>(gl, (const uint16_t *)W.w_gate, (const uint16_t *)W.w_up, s.F, s.H, gu16);
+      tile_down_kernel<<<grid, 256>>>(dl, (const uint16_t *)W.w_down, s.H, s.F, p.KCd, dn16);
+      ld[l].wgu_tc = gl;
+      ld[l].wd_tc = dl;
+    }
     if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
       cudaGetLastError();
       return MK_ERR_CUDA;
     }
-    k.lm_tc = tiles;
+    LayerDev *d_ld = nullptr;
+    if ((rc = dalloc(h->plan_allocs, &d_ld, s.L, false))) return rc;
+    MK_CUDA(cudaMemcpy(d_ld, ld.data(), sizeof(LayerDev) * s.L, cudaMemcpyHostToDevice));
+    k.layers = d_ld;
+    k.lm_tc = lm_t;
   }
   k.final_norm = h->final_norm;
   k.kc = h->kc;

@@ -263,6 +263,7 @@ struct Shared {
   uint32_t tmem_base;
   uint32_t mma_phase;
   unsigned long long mma_bar;
+  float tc_xch[64 * 16];  // gate/up on the tensor cores: up rows handed to the gate rows' warps
   uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
   float red[kComputeWarps][kMaxBatch];
   float argv[kComputeWarps][kMaxBatch];
@@ -491,12 +492,26 @@ __device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, 
   switch (I.op) {
     case OP_QKV: s.a = p.layers[I.layer].wqkv + (size_t)I.a * kPageElems; break;
     case OP_OPROJ: s.a = p.layers[I.layer].wo + (size_t)I.a * kPageElems; break;
-    case OP_GATEUP: s.a = p.layers[I.layer].wgu + (size_t)I.a * kPageElems; break;
-    case OP_DOWN: s.a = p.layers[I.layer].wd + ((size_t)I.c * (p.H / p.Rd) + I.a) * kPageElems; break;
+    case OP_GATEUP:
+      if (p.layers[I.layer].wgu_tc) {  // 128-row tiles (64 gate + 64 up rows) of H / 64 pages
+        s.a = p.layers[I.layer].wgu_tc + (size_t)I.a * (p.H / 64) * kPageElems;
+        s.npg = (int)I.b * (p.H / 64);
+      } else {
+        s.a = p.layers[I.layer].wgu + (size_t)I.a * kPageElems;
+      }
+      break;
+    case OP_DOWN:
+      if (p.layers[I.layer].wd_tc) {  // per K piece: 128-row tiles of KCd / 64 pages
+        s.a = p.layers[I.layer].wd_tc + ((size_t)I.c * (p.H / 128) + I.a) * (p.KCd / 64) * kPageElems;
+        s.npg = (int)I.b * (p.KCd / 64);
+      } else {
+        s.a = p.layers[I.layer].wd + ((size_t)I.c * (p.H / p.Rd) + I.a) * kPageElems;
+      }
+      break;
     case OP_LMHEAD: {
-      if (p.lm_tc) {  // whole 128-row tiles, ppb pages each
-        s.a = p.lm_tc + (size_t)I.a * p.lm_ppb * kPageElems;
-        s.npg = (int)I.b * p.lm_ppb;
+      if (p.lm_tc) {  // whole 128-row tiles of H / 64 pages
+        s.a = p.lm_tc + (size_t)I.a * (p.H / 64) * kPageElems;
+        s.npg = (int)I.b * (p.H / 64);
         break;
       }
       s.a = p.lm_head + (size_t)I.a * p.Rh * p.H;
@@ -1365,41 +1380,31 @@ __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
   return c.g;
 }
 
-// LM head on the tensor cores (batched builds): the weight is in 128-row
+// Tensor-core matrix product for batched builds: the matrix is in 128-row
 // tiles of 64 columns per 16 KiB page (K-major, no swizzle), an instruction
-// covers whole 128-row blocks, and every block accumulates
-// D[128 rows][16 sequences] (f32, tensor memory) over the block's pages with
-// two MMAs per 16 columns (the activations' bf16 hi and lo halves).  One
-// thread issues the MMAs and recycles each page once its MMAs completed;
-// four warps (one per quarter of the tensor-memory lanes) read the block's
-// logits.  A dense contraction at 16 sequences: about 16 flops per weight
-// byte.
-template <int NB, int R>
-__device__ __forceinline__ uint32_t lmhead_tc_body(CCtx c, const Instr I) {
+// covers whole tiles, and every tile accumulates D[128 rows][16 sequences]
+// (f32, tensor memory) over the tile's pages with two MMAs per 16 columns
+// (the staged activations' bf16 hi and lo halves, staged by stage_norm /
+// stage_copy_tc).  One thread issues the MMAs and recycles each page once
+// its MMAs completed; then the four warps of the tensor-memory lane quarters
+// read the tile (row = 32 * quarter + lane, 16 sequences) and run
+// epi(tile, quarter, v).  At 16 sequences the product is a dense contraction
+// (about 16 flops per weight byte).
+__device__ __forceinline__ bool tc_reader(const CCtx &c) { return c.cw >= 2 && c.cw < 6; }
+__device__ __forceinline__ int tc_quarter(const CCtx &c) { return (c.cw + kLoaders) & 3; }
+// barrier of the four reader warps only
+__device__ __forceinline__ void tc_readers_sync() { asm volatile("barrier.cta.sync 3, 128;" ::: "memory"); }
+
+template <int NB, class Epi>
+__device__ __forceinline__ bool tc_tiles(CCtx &c, int ntiles, int ppb, int K, Epi &&epi) {
   static_assert(NB == 16, "the MMA's N is the batch slot count");
   const KParams &p = c.p;
-  const int H = p.H, V = p.V, Bn = p.B, ppb = p.lm_ppb;
-  float inv[NB];
-  stage_norm<NB, StageIt<R>::v, true>(c, p.L, p.final_norm, false, inv);
-  px::fence_proxy_async_smem();  // the staged operand, written by the generic proxy, is read by the MMAs
-  px::cbar();
-  const uint32_t hi_s = px::sa(c.act), lo_s = hi_s + (uint32_t)H * 32u;
+  const uint32_t hi_s = px::sa(c.act), lo_s = hi_s + (uint32_t)K * 32u;  // K staged columns
   // D f32, A and B bf16, both K-major, N = 16, M = 128
   constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
   const uint32_t tmem = c.sh->tmem_base;
   const Ring rg = ring_of(c);
-  // the warps whose tensor-memory lane quarter is (warp % 4)
-  const int warp = c.cw + kLoaders, quarter = warp & 3;
-  const bool reader = c.cw >= 2 && c.cw < 6;
-  float bv[NB];
-  int bi[NB];
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    bv[b] = -INFINITY;
-    bi[b] = 0x7fffffff;
-  }
-  const int nblk = (int)I.b;
-  for (int blk = 0; blk < nblk; ++blk) {
+  for (int blk = 0; blk < ntiles; ++blk) {
     if (c.ctid == 0) {
       for (int kb = 0; kb < ppb; ++kb) {
         const uint32_t g = c.g + (uint32_t)(blk * ppb + kb);
@@ -1425,33 +1430,142 @@ __device__ __forceinline__ uint32_t lmhead_tc_body(CCtx c, const Instr I) {
       }
       px::tc_fence_before();
     }
-    // every MMA of the block has completed (thread 0 waited for each page's)
-    if (px::cbar_or(px::ld_volatile(&c.sh->abort) != 0)) break;
+    // every MMA of the tile has completed (thread 0 waited for each page's)
+    if (px::cbar_or(px::ld_volatile(&c.sh->abort) != 0)) return false;
     px::tc_fence_after();
-    if (reader) {
+    if (tc_reader(c)) {
+      const int q = tc_quarter(c);
       float v[16];
-      px::tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16), v);
-      const int row = ((int)I.a + blk) * 128 + quarter * 32 + c.lane;
-      if (row < V) {
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          if (b >= Bn) break;
-          const float x = v[b] * inv[b];
-          if (p.logits) p.logits[(size_t)b * V + row] = x;
-          if (arg_better(x, row, bv[b], bi[b])) {
-            bv[b] = x;
-            bi[b] = row;
-          }
-        }
-      }
+      px::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16), v);
+      epi(blk, q, v);
     }
     px::tc_fence_before();
-    px::cbar();  // the block's logits are read before the next block's MMAs overwrite them
+    px::cbar();  // the tile is read before the next tile's MMAs overwrite it
   }
-  c.g += (uint32_t)(nblk * ppb);
+  c.g += (uint32_t)(ntiles * ppb);
+  return true;
+}
+
+template <int NB, int R>
+__device__ __forceinline__ uint32_t lmhead_tc_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int V = p.V, Bn = p.B;
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v, true>(c, p.L, p.final_norm, false, inv);
+  px::fence_proxy_async_smem();  // the staged operand, written by the generic proxy, is read by the MMAs
+  px::cbar();
+  float bv[NB];
+  int bi[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    bv[b] = -INFINITY;
+    bi[b] = 0x7fffffff;
+  }
+  const bool ok = tc_tiles<NB>(c, (int)I.b, p.H / 64, p.H, [&](int blk, int q, const float (&v)[16]) {
+    const int row = ((int)I.a + blk) * 128 + q * 32 + c.lane;
+    if (row >= V) return;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= Bn) break;
+      const float x = v[b] * inv[b];
+      if (p.logits) p.logits[(size_t)b * V + row] = x;
+      if (arg_better(x, row, bv[b], bi[b])) {
+        bv[b] = x;
+        bi[b] = row;
+      }
+    }
+  });
+  if (!ok) return c.g;
   lm_argmax_tail<NB>(c, I, bv, bi);
   return c.g;
 }
+
+// gate/up on the tensor cores: a tile holds 64 gate rows then the same 64 up
+// rows, so quarters 0-1 pair their gate rows with the up rows quarters 2-3 read
+template <int NB, int R>
+__device__ __forceinline__ uint32_t gateup_tc_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, Bn = p.B, F = p.F;
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v, true>(c, l, p.layers[l].ffn_norm, true, inv);
+  px::fence_proxy_async_smem();
+  px::cbar();
+  const uint32_t tag = c.epoch;
+  float *const aout = p.actb + (size_t)l * Bn * F;
+  float *xch = reinterpret_cast<float *>(c.sh->tc_xch);  // [64 rows][16 sequences]
+  tc_tiles<NB>(c, (int)I.b, p.H / 64, p.H, [&](int blk, int q, const float (&v)[16]) {
+    const int r = (q & 1) * 32 + c.lane;  // row inside the tile's 64 gate / up rows
+    if (q >= 2) {
+#pragma unroll
+      for (int b = 0; b < 16; ++b) xch[r * 16 + b] = v[b];
+    }
+    tc_readers_sync();
+    if (q < 2) {
+      const int row = ((int)I.a + blk) * 64 + r;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b >= Bn) break;
+        const float gt = v[b] * inv[b], up = xch[r * 16 + b] * inv[b];
+        const float silu = gt / (1.0f + expf(-gt));
+        px::st_tf(aout + (size_t)b * F + row, silu * up, tag);
+      }
+    }
+    tc_readers_sync();  // the exchange buffer is reused by the next tile
+  });
+  return c.g;
+}
+
+// down projection on the tensor cores: K piece I.c (KCd columns of act,
+// staged as bf16 hi / lo), tiles of 128 output rows
+template <int NB>
+__device__ __forceinline__ void stage_copy_tc(CCtx &c, const float *src, size_t src_stride, int K) {
+  const KParams &p = c.p;
+  uint16_t *hi = reinterpret_cast<uint16_t *>(c.act);
+  const int n4 = K / 4;
+  for (int b0 = 0; b0 < NB; b0 += 4) {
+    if (b0 >= p.B) break;
+    settle(c, 8, [&](bool &ok) {
+      for (int e4 = c.ctid; e4 < n4; e4 += kComputeThreads) {
+        float4 x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (b0 + i < p.B) x[i] = ll_load4(c.epoch, src + (size_t)(b0 + i) * src_stride + e4 * 4, ok);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (b0 + i < p.B) {
+            const size_t o = ((size_t)(e4 >> 1) * 16 + b0 + i) * 8 + (e4 & 1) * 4;
+            split_bf16x4(x[i], hi + o, hi + (size_t)K * 16 + o);
+          }
+      }
+    });
+  }
+  px::fence_proxy_async_smem();
+  px::cbar();
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+}
+
+template <int NB>
+__device__ __forceinline__ uint32_t down_tc_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, k = I.c, Bn = p.B, H = p.H;
+  stage_copy_tc<NB>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
+  const uint32_t tag = c.epoch;
+  float *const dout = p.dpart + ((size_t)l * p.ndp + k) * Bn * H;
+  tc_tiles<NB>(c, (int)I.b, p.KCd / 64, p.KCd, [&](int blk, int q, const float (&v)[16]) {
+    const int row = ((int)I.a + blk) * 128 + q * 32 + c.lane;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= Bn) break;
+      px::st_tf(dout + (size_t)b * H + row, v[b], tag);
+    }
+  });
+  return c.g;
+}
+
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_gateup_tc(CCtx c, const Instr I) { return gateup_tc_body<NB, R>(c, I); }
+template <int NB>
+__device__ __noinline__ uint32_t op_down_tc(CCtx c, const Instr I) { return down_tc_body<NB>(c, I); }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_lmhead_tc(CCtx c, const Instr I) { return lmhead_tc_body<NB, R>(c, I); }
 template <int NB, int R>
@@ -1927,11 +2041,23 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         else MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);
         break;
       case OP_GATEUP:
+        if constexpr (NB > 1 && S::fixed) {
+          if (p.layers[I.layer].wgu_tc) {
+            c.g = op_gateup_tc<NB, S::RH>(c, I);
+            break;
+          }
+        }
         if constexpr (kInline) c.g = gateup_body<NB, S::RH>(c, I);
         else if constexpr (S::fixed) c.g = op_gateup<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_gateup, NB, p.Rh, c, I);
         break;
       case OP_DOWN:
+        if constexpr (NB > 1 && S::fixed) {
+          if (p.layers[I.layer].wd_tc) {
+            c.g = op_down_tc<NB>(c, I);
+            break;
+          }
+        }
         if constexpr (kInline) c.g = down_body<NB, S::RD>(c, I);
         else if constexpr (S::fixed) c.g = op_down<NB, S::RD>(c, I);
         else MK_DISPATCH_R(op_down, NB, p.Rd, c, I);

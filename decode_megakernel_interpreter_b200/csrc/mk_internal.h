@@ -67,6 +67,10 @@ struct LayerDev {
   const uint16_t *wd;       // packed [F/KCd pieces][H/Rd pages][Rd][KCd]
   const uint16_t *attn_norm;
   const uint16_t *ffn_norm;
+  // batched plans: gate/up and down in 128-row tensor-core tiles (64 columns
+  // per page, K-major without swizzle); null otherwise
+  const uint16_t *wgu_tc;   // [F/64 tiles: 64 gate + 64 up rows][H/64 pages]
+  const uint16_t *wd_tc;    // [F/KCd pieces][H/128 tiles][KCd/64 pages]
 };
 
 // Per-layer pointers to the caller's weights in their own [out][in] layout
@@ -98,9 +102,8 @@ struct KParams {
   float eps, attn_scale;
   float inv_H;                     // 1 / hidden (exact: hidden is a power of two)
   // batched plans: the LM head in 128-row tensor-core tiles (64 columns per
-  // page, K-major without swizzle) and the pages per tile; null otherwise
+  // page, K-major without swizzle); null otherwise
   const uint16_t *lm_tc;
-  int lm_ppb;
   // weights
   const LayerDev *layers;
   const LayerRaw *layers_raw;  // only read by the raw-layout kernel variant

@@ -136,6 +136,13 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
     return I;
   };
   std::vector<int> n_down(s.L, 0), n_qkv(s.L, 0), n_o(s.L, 0);
+  p.tensor = req.tensor;
+  p.gu_rows_unit = p.tensor ? 64 : p.Rh / 2;
+  p.dn_rows_unit = p.tensor ? 128 : p.Rd;
+  const int gu_units = p.tensor ? s.F / 64 : p.P_gu;
+  const int dn_units = p.tensor ? s.H / 128 : p.P_dp;
+  const int64_t gu_unit_bytes = p.tensor ? (int64_t)(s.H / 64) * kPageBytes : kPageBytes;
+  const int64_t dn_unit_bytes = p.tensor ? (int64_t)(p.KCd / 64) * kPageBytes : kPageBytes;
   for (int l = 0; l < s.L; ++l) {
     // fused RMSNorm + QKV + RoPE
     auto cq = split_even(p.P_qkv, parts);
@@ -182,9 +189,11 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       all.push_back({I, (int64_t)co[i].count * kPageBytes, l * 8 + ST_OPROJ, (int)i});
     }
     // RMSNorm + gate/up + SiLU; signals the down-projection K pieces it feeds
-    auto cg = split_even(p.P_gu, parts);
+    // (units: pages of R/2 gate + R/2 up rows, or 128-row tensor-core tiles
+    // of 64 gate + 64 up rows)
+    auto cg = split_even(gu_units, parts);
     std::vector<int> gu_per_piece(p.ndp, 0);
-    const int half = p.Rh / 2;
+    const int half = p.gu_rows_unit;
     for (size_t i = 0; i < cg.size(); ++i) {
       Instr I = mk_instr(OP_GATEUP, l);
       I.a = cg[i].first;
@@ -196,7 +205,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       I.sig_ctr = p.ctr_gu(l, k0);
       I.sig_n = (uint16_t)(k1 - k0 + 1);
       for (int k = k0; k <= k1; ++k) gu_per_piece[k]++;
-      all.push_back({I, (int64_t)cg[i].count * kPageBytes, l * 8 + ST_GATEUP, (int)i});
+      all.push_back({I, (int64_t)cg[i].count * gu_unit_bytes, l * 8 + ST_GATEUP, (int)i});
     }
     // down projection, K-split into pieces; each piece waits only for the
     // gate/up instructions that produce its K range
@@ -204,7 +213,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
     int ord2 = 0;
     for (int k = 0; k < p.ndp; ++k) {
       int ck = (int)((int64_t)parts * (k + 1) / p.ndp - (int64_t)parts * k / p.ndp);
-      auto cd = split_even(p.P_dp, std::max(1, ck));
+      auto cd = split_even(dn_units, std::max(1, ck));
       for (auto &c : cd) {
         Instr I = mk_instr(OP_DOWN, l);
         I.a = c.first;
@@ -215,16 +224,15 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
         I.sig_ctr = p.ctr_dn(l);
         I.sig_n = 1;
         n_down[l]++;
-        all.push_back({I, (int64_t)c.count * kPageBytes, l * 8 + ST_DOWN, ord2++});
+        all.push_back({I, (int64_t)c.count * dn_unit_bytes, l * 8 + ST_DOWN, ord2++});
       }
     }
     (void)total;
   }
   // final RMSNorm + LM head + argmax (units: pages of R rows, or 128-row
   // blocks of H / 64 pages on the tensor-core path)
-  p.lm_tensor = req.lm_tensor;
-  const int lm_units = p.lm_tensor ? (s.V + 127) / 128 : p.P_lm;
-  const int64_t lm_unit_bytes = p.lm_tensor ? (int64_t)(s.H / 64) * kPageBytes : kPageBytes;
+  const int lm_units = p.tensor ? (s.V + 127) / 128 : p.P_lm;
+  const int64_t lm_unit_bytes = p.tensor ? (int64_t)(s.H / 64) * kPageBytes : kPageBytes;
   auto cl = split_even(lm_units, parts);
   p.n_lm = (int)cl.size();
   for (size_t i = 0; i < cl.size(); ++i) {
@@ -248,7 +256,10 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   for (size_t i = 0; i < all.size(); ++i) all[i].ins.seq = (uint16_t)i;
   for (auto &x : all) {
     if (x.ins.op >= OP_QKV && x.ins.op <= OP_LMHEAD && x.ins.op != OP_ATTN)
-      p.weight_bytes += (int64_t)x.ins.b * (x.ins.op == OP_LMHEAD ? lm_unit_bytes : kPageBytes);
+      p.weight_bytes += (int64_t)x.ins.b * (x.ins.op == OP_LMHEAD   ? lm_unit_bytes
+                                           : x.ins.op == OP_GATEUP ? gu_unit_bytes
+                                           : x.ins.op == OP_DOWN   ? dn_unit_bytes
+                                                                   : (int64_t)kPageBytes);
   }
   // the last LM page (or block) may be partial
   {
@@ -391,7 +402,7 @@ void rw_sets(const PlanRequest &req, const Plan &p, const Instr &I, std::vector<
     }
     case OP_GATEUP: {
       rd.push_back({B_XRES, (int64_t)l * s.H, (int64_t)(l + 1) * s.H});
-      int half = p.Rh / 2;
+      int half = p.gu_rows_unit;
       wr.push_back({B_ACT, (int64_t)l * s.F + (int64_t)I.a * half,
                     (int64_t)l * s.F + (int64_t)(I.a + I.b) * half});
       break;
@@ -400,7 +411,7 @@ void rw_sets(const PlanRequest &req, const Plan &p, const Instr &I, std::vector<
       rd.push_back({B_ACT, (int64_t)l * s.F + (int64_t)I.c * p.KCd,
                     (int64_t)l * s.F + (int64_t)(I.c + 1) * p.KCd});
       int64_t base = ((int64_t)l * p.ndp + I.c) * s.H;
-      wr.push_back({B_DPART, base + (int64_t)I.a * p.Rd, base + (int64_t)(I.a + I.b) * p.Rd});
+      wr.push_back({B_DPART, base + (int64_t)I.a * p.dn_rows_unit, base + (int64_t)(I.a + I.b) * p.dn_rows_unit});
       break;
     }
     case OP_LMHEAD:

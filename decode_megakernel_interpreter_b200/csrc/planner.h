@@ -25,15 +25,17 @@ struct PlanRequest {
   int dyn_chunks_per_cta = 2;  // dynamic mode: instructions per CTA per matvec stage
   int assumed_context = 1024;  // for the automatic split count
   bool drop_producer = false;  // test hook (see mk_plan_opts)
-  // LM head on the tensor cores (batched plans): instructions cover whole
-  // 128-row blocks of a tiled copy of the LM head, H / 64 pages per block
-  bool lm_tensor = false;
+  // tensor cores (batched plans): gate/up, down and LM-head instructions
+  // cover whole 128-row tiles of tiled weight copies (64 columns per page)
+  bool tensor = false;
 };
 
 struct Plan {
   // geometry
   int Rh = 0, Ro = 0, Rd = 0, KCd = 0, ndp = 0, S = 0;
-  bool lm_tensor = false;  // see PlanRequest
+  bool tensor = false;  // see PlanRequest
+  int gu_rows_unit = 0;  // act rows per gate/up unit (page, or 64 on the tensor cores)
+  int dn_rows_unit = 0;  // output rows per down unit (page, or 128 on the tensor cores)
   int P_qkv = 0, P_o = 0, P_gu = 0, P_dp = 0, P_lm = 0;  // pages per layer / piece / head
   // instructions: static mode = per-CTA queues back to back; dynamic = global order
   std::vector<Instr> instrs;
