@@ -897,38 +897,50 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
   uint2 gws[IT];
 #pragma unroll
   for (int b = 0; b < NB; ++b) ss[b] = 0.f;
+  // sequences in groups of GB: one group's loads are in flight together
+  constexpr int GB = NB == 1 ? 1 : 4;
 #pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    if (b >= p.B) break;
-    const int tok = (l == 0 && !from_xres_only) ? read_tok(c.sh, b) : 0;
-    float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
-    float4 xs[IT];
+  for (int b0 = 0; b0 < NB; b0 += GB) {
+    if (b0 >= p.B) break;
+    float4 xs[GB][IT];
     settle(c, 2, [&](bool &ok) {
 #pragma unroll
-      for (int it = 0; it < IT; ++it) {
-        const int e4 = c.ctid + it * kComputeThreads;
-        if (e4 < n4) {
-          if (b == 0) gws[it] = __ldg(reinterpret_cast<const uint2 *>(gamma) + e4);  // with x: one round trip
-          xs[it] = from_xres_only ? ll_load4(c.epoch, p.xres + ((size_t)l * p.B + b) * H + e4 * 4, ok)
-                                  : layer_input4(p, c.epoch, l, b, tok, e4, ok);
+      for (int i = 0; i < GB; ++i) {
+        const int b = b0 + i;
+        if (b >= p.B) break;
+        const int tok = (l == 0 && !from_xres_only) ? read_tok(c.sh, b) : 0;
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+          const int e4 = c.ctid + it * kComputeThreads;
+          if (e4 < n4) {
+            if (b == 0) gws[it] = __ldg(reinterpret_cast<const uint2 *>(gamma) + e4);  // with x: one round trip
+            xs[i][it] = from_xres_only ? ll_load4(c.epoch, p.xres + ((size_t)l * p.B + b) * H + e4 * 4, ok)
+                                       : layer_input4(p, c.epoch, l, b, tok, e4, ok);
+          }
         }
       }
     });
 #pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      const int e4 = c.ctid + it * kComputeThreads;
-      if (e4 < n4) {
-        const float4 x = xs[it];
-        const uint2 gw = gws[it];
-        ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
-        const float4 xg =
-            make_float4(x.x * px::bf_lo(gw.x), x.y * px::bf_hi(gw.x), x.z * px::bf_lo(gw.y), x.w * px::bf_hi(gw.y));
-        if constexpr (TC) {
-          uint16_t *hi = reinterpret_cast<uint16_t *>(c.act);
-          const size_t o = ((size_t)(e4 >> 1) * 16 + b) * 8 + (e4 & 1) * 4;
-          split_bf16x4(xg, hi + o, hi + (size_t)H * 16 + o);
-        } else {
-          dst[stage_slot4(e4, H)] = xg;
+    for (int i = 0; i < GB; ++i) {
+      const int b = b0 + i;
+      if (b >= p.B) break;
+      float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int e4 = c.ctid + it * kComputeThreads;
+        if (e4 < n4) {
+          const float4 x = xs[i][it];
+          const uint2 gw = gws[it];
+          ss[b] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+          const float4 xg =
+              make_float4(x.x * px::bf_lo(gw.x), x.y * px::bf_hi(gw.x), x.z * px::bf_lo(gw.y), x.w * px::bf_hi(gw.y));
+          if constexpr (TC) {
+            uint16_t *hi = reinterpret_cast<uint16_t *>(c.act);
+            const size_t o = ((size_t)(e4 >> 1) * 16 + b) * 8 + (e4 & 1) * 4;
+            split_bf16x4(xg, hi + o, hi + (size_t)H * 16 + o);
+          } else {
+            dst[stage_slot4(e4, H)] = xg;
+          }
         }
       }
     }
@@ -960,23 +972,32 @@ __device__ void stage_copy(CCtx &c, const float *src, size_t src_stride, int K, 
   float xr = 0.f;
   const bool has_row = c.ctid < nrows;
   const int tok0 = l == 0 ? read_tok(c.sh, 0) : 0;
+  constexpr int GB = NB == 1 ? 1 : 4;  // sequences whose loads are in flight together
 #pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    if (b >= p.B) break;
-    float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)b * c.act_stride);
-    float4 vs[IT];
+  for (int b0 = 0; b0 < NB; b0 += GB) {
+    if (b0 >= p.B) break;
+    float4 vs[GB][IT];
     settle(c, 3, [&](bool &ok) {  // the row of x_in rides along with sequence 0's vector
-      if (b == 0 && has_row) xr = layer_input1(p, c.epoch, l, 0, tok0, row0 + c.ctid, ok);
+      if (b0 == 0 && has_row) xr = layer_input1(p, c.epoch, l, 0, tok0, row0 + c.ctid, ok);
 #pragma unroll
-      for (int it = 0; it < IT; ++it) {
-        const int e4 = c.ctid + it * kComputeThreads;
-        if (e4 < n4) vs[it] = ll_load4(c.epoch, src + (size_t)b * src_stride + e4 * 4, ok);
+      for (int i = 0; i < GB; ++i) {
+        if (b0 + i >= p.B) break;
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+          const int e4 = c.ctid + it * kComputeThreads;
+          if (e4 < n4) vs[i][it] = ll_load4(c.epoch, src + (size_t)(b0 + i) * src_stride + e4 * 4, ok);
+        }
       }
     });
 #pragma unroll
-    for (int it = 0; it < IT; ++it) {
-      const int e4 = c.ctid + it * kComputeThreads;
-      if (e4 < n4) dst[stage_slot4(e4, K)] = vs[it];
+    for (int i = 0; i < GB; ++i) {
+      if (b0 + i >= p.B) break;
+      float4 *dst = reinterpret_cast<float4 *>(c.act + (size_t)(b0 + i) * c.act_stride);
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int e4 = c.ctid + it * kComputeThreads;
+        if (e4 < n4) dst[stage_slot4(e4, K)] = vs[i][it];
+      }
     }
   }
   for (int r = c.ctid; r < nrows; r += kComputeThreads)
@@ -1184,13 +1205,23 @@ __device__ __forceinline__ uint32_t oproj_body(CCtx c, const Instr I) {
   matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
     if (lane >= R) return;
     const int row = j * R + lane;
+    if constexpr (NB == 1) {
+      px::st_tf(xout + row, xrows[row] + pick<R>(acc[0], lane), tag);
+    } else {
+      // the residual row of every sequence: one group of loads (retried as a whole)
+      float xin[NB];
+      for (LLRetry r;;) {
+        bool ok = true;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      if (NB > 1 && b >= Bn) break;
-      const float v = pick<R>(acc[b], lane);
-      const float xin =
-          NB == 1 ? xrows[row] : layer_input1_settled(p, c.sh, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row);
-      px::st_tf(xout + (size_t)b * H + row, xin + v, tag);
+        for (int b = 0; b < NB; ++b)
+          if (b < Bn) xin[b] = layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
+        if (ok || !ll_retry(p, c.sh, r, 9)) break;
+      }
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b >= Bn) break;
+        px::st_tf(xout + (size_t)b * H + row, xin[b] + pick<R>(acc[b], lane), tag);
+      }
     }
   });
   return c.g;
@@ -1524,20 +1555,29 @@ __device__ __forceinline__ void stage_copy_tc(CCtx &c, const float *src, size_t 
   const int n4 = K / 4;
   for (int b0 = 0; b0 < NB; b0 += 4) {
     if (b0 >= p.B) break;
+    constexpr int IT = 2;  // K <= 2048: two float4 per thread and sequence
+    float4 x[4][IT];
     settle(c, 8, [&](bool &ok) {
-      for (int e4 = c.ctid; e4 < n4; e4 += kComputeThreads) {
-        float4 x[4];
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int e4 = c.ctid + it * kComputeThreads;
+        if (e4 >= n4) break;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          if (b0 + i < p.B) x[i] = ll_load4(c.epoch, src + (size_t)(b0 + i) * src_stride + e4 * 4, ok);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (b0 + i < p.B) {
-            const size_t o = ((size_t)(e4 >> 1) * 16 + b0 + i) * 8 + (e4 & 1) * 4;
-            split_bf16x4(x[i], hi + o, hi + (size_t)K * 16 + o);
-          }
+          if (b0 + i < p.B) x[i][it] = ll_load4(c.epoch, src + (size_t)(b0 + i) * src_stride + e4 * 4, ok);
       }
     });
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 >= n4) break;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (b0 + i < p.B) {
+          const size_t o = ((size_t)(e4 >> 1) * 16 + b0 + i) * 8 + (e4 & 1) * 4;
+          split_bf16x4(x[i][it], hi + o, hi + (size_t)K * 16 + o);
+        }
+    }
   }
   px::fence_proxy_async_smem();
   px::cbar();
