@@ -148,3 +148,26 @@ def test_plan_rejects_bad_options():
         mk.mk_host_plan(cfg, mk.plan_opts(batch=2), 8)
     with pytest.raises(mk.MkError):
         mk.mk_host_plan(cfg, mk.plan_opts(batch=0), 8)
+
+
+def test_batched_plan_uses_tensor_core_tiles():
+    """Batched plans cover gate/up, down and the LM head in 128-row tiles
+    (64 gate + 64 up rows for gate/up) and stream the same weight bytes as
+    the batch-1 plan."""
+    cfg1 = cfg_for("llama1b")
+    *_, info1 = mk.mk_host_plan(cfg1, mk.plan_opts(batch=1), 148)
+    cfg = cfg_for("llama1b_b16", max_batch=16)
+    instrs, off, ln, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=16), 148)
+    assert info.weight_bytes_per_step == info1.weight_bytes_per_step
+    F, H, V = cfg.ffn, cfg.hidden, cfg.vocab
+    for l in (0, cfg.n_layers - 1):
+        gu = [i for i in instrs if i.op == OP["gateup"] and i.layer == l]
+        assert sorted((i.a, i.a + i.b) for i in gu)[0][0] == 0
+        assert sum(i.b for i in gu) == F // 64
+        for k in range(F // 2048):
+            dn = [i for i in instrs if i.op == OP["down"] and i.layer == l and i.c == k]
+            assert sum(i.b for i in dn) == H // 128
+    lm = [i for i in instrs if i.op == OP["lmhead"]]
+    assert sum(i.b for i in lm) == -(-V // 128)
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=16), 148, steps=1, seed=5, timeout_ms=20000)
+    assert err == ""
