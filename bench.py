@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--l2-prefetch-kb", type=int, default=0)
     ap.add_argument("--inflight", type=int, default=0, help="bulk-copy pages in flight per CTA (0 = default)")
+    ap.add_argument("--tensor-qkv-o", action="store_true",
+                    help="batched plans: QKV and O projection on the tensor cores too")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="add a per-instruction-class time breakdown")
@@ -321,7 +323,8 @@ def main():
     del k, v
     eng = harness.make_engine(s, dev, kc, vc, B, max_seq)
     plan_kw = dict(batch=B, kv_splits=args.kv_splits, sched=args.sched, exec_mode=args.exec_mode,
-                   l2_prefetch_kb=args.l2_prefetch_kb, max_inflight_pages=args.inflight)
+                   l2_prefetch_kb=args.l2_prefetch_kb, max_inflight_pages=args.inflight,
+                   tensor_qkv_o=args.tensor_qkv_o)
     eng.plan_kw = plan_kw
     info = eng.plan(**plan_kw)
     stream = torch.cuda.current_stream()

@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["api.cu", "interp.cu", "interp_spec_llama1b.cu", "interp_spec_llama1b_batched.cu", "interp_spec_llama8b.cu",
+SOURCES = ["api.cu", "interp.cu", "interp_spec_llama1b.cu", "interp_spec_llama1b_batched.cu",
+           "interp_spec_llama1b_batched_tqo.cu", "interp_spec_llama8b.cu",
            "noalloc.cu", "planner.cpp"]
 HEADERS = ["mk_internal.h", "planner.h", "interp_body.cuh", "interp_launch.h"]
 PUBLIC = [os.path.join(ROOT, "include", h) for h in ("mk.h", "mk_host.h")]

@@ -173,6 +173,25 @@ __global__ void tile_gu_kernel(uint16_t *dst, const uint16_t *gate, const uint16
         r < 64 ? tile_unit(gate, tile * 64 + r, F, H, col) : tile_unit(up, tile * 64 + r - 64, F, H, col);
   }
 }
+// fused QKV tiles: rows of [q; k; v] (wq, wk, wv stacked), 128 per tile
+__global__ void tile_qkv_kernel(uint16_t *dst, const uint16_t *wq, const uint16_t *wk, const uint16_t *wv, int qdim,
+                                int kvdim, int H, long long n16) {
+  const int kpt = H / 64;
+  for (long long u = blockIdx.x * (long long)blockDim.x + threadIdx.x; u < n16; u += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(u % 128);
+    long long t = u / 128;
+    const int ch = (int)(t % 8);
+    t /= 8;
+    const int kb = (int)(t % kpt);
+    const long long row = (t / kpt) * 128 + r;
+    const long long col = (long long)kb * 64 + ch * 8;
+    uint4 v;
+    if (row < qdim) v = tile_unit(wq, row, qdim, H, col);
+    else if (row < qdim + kvdim) v = tile_unit(wk, row - qdim, kvdim, H, col);
+    else v = tile_unit(wv, row - qdim - kvdim, kvdim, H, col);
+    reinterpret_cast<uint4 *>(dst)[u] = v;
+  }
+}
 // down tiles: piece k (columns k*KCd..), row tile rt (rows 128rt..), page kb
 __global__ void tile_down_kernel(uint16_t *dst, const uint16_t *wd, int H, int F, int KCd, long long n16) {
   const int kpt = KCd / 64, rts = H / 128;
@@ -306,6 +325,7 @@ PlanRequest make_request(const mk_config &c, const mk_plan_opts &o, int num_ctas
   r.assumed_context = std::max(1, c.max_seq);
   r.drop_producer = o.debug_drop_producer != 0;
   r.tensor = o.batch > 1;  // batched plans run gate/up, down and the LM head on the tensor cores
+  r.tensor_qkv_o = o.tensor_qkv_o != 0;
   return r;
 }
 
@@ -492,7 +512,8 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   sel.Ro = p.Ro;
   sel.Rd = p.Rd;
   int variant = 0;
-  const void *kernel = interp_kernel_for(sel, o.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC, nb, &variant);
+  const void *kernel =
+      interp_kernel_for(sel, o.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC, nb, p.tensor_qkv_o, &variant);
   if (!kernel) return MK_ERR_UNSUPPORTED_SHAPE;  // batch > 1 without a batched build for this shape
   int per_sm = 0;
   cudaError_t e = interp_prepare(kernel, smem, &per_sm);
@@ -571,10 +592,16 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
     const long long lm16 = (long long)((s.V + 127) / 128) * 128 * (s.H / 8);
     const long long gu16 = (long long)(s.F / 64) * 128 * (s.H / 8);
     const long long dn16 = (long long)s.H * (s.F / 8);
-    uint16_t *lm_t = nullptr, *gu_t = nullptr, *dn_t = nullptr;
+    const int qdim = s.nq * s.d, kvdim = s.nkv * s.d;
+    const long long qkv16 = (long long)(qdim + 2 * kvdim) * (s.H / 8), o16 = (long long)s.H * (qdim / 8);
+    uint16_t *lm_t = nullptr, *gu_t = nullptr, *dn_t = nullptr, *qkv_t = nullptr, *o_t = nullptr;
     if ((rc = dalloc(h->plan_allocs, &lm_t, (size_t)lm16 * 8, false))) return rc;
     if ((rc = dalloc(h->plan_allocs, &gu_t, (size_t)gu16 * 8 * s.L, false))) return rc;
     if ((rc = dalloc(h->plan_allocs, &dn_t, (size_t)dn16 * 8 * s.L, false))) return rc;
+    if (p.tensor_qkv_o) {
+      if ((rc = dalloc(h->plan_allocs, &qkv_t, (size_t)qkv16 * 8 * s.L, false))) return rc;
+      if ((rc = dalloc(h->plan_allocs, &o_t, (size_t)o16 * 8 * s.L, false))) return rc;
+    }
     tile_lm_kernel<<<grid, 256>>>(lm_t, h->lm_head, s.V, s.H, lm16);
     std::vector<LayerDev> ld(s.L);
     MK_CUDA(cudaMemcpy(ld.data(), h->d_layers, sizeof(LayerDev) * s.L, cudaMemcpyDeviceToHost));
@@ -585,6 +612,14 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
       tile_down_kernel<<<grid, 256>>>(dl, (const uint16_t *)W.w_down, s.H, s.F, p.KCd, dn16);
       ld[l].wgu_tc = gl;
       ld[l].wd_tc = dl;
+      if (p.tensor_qkv_o) {
+        uint16_t *ql = qkv_t + (size_t)qkv16 * 8 * l, *ol = o_t + (size_t)o16 * 8 * l;
+        tile_qkv_kernel<<<grid, 256>>>(ql, (const uint16_t *)W.wq, (const uint16_t *)W.wk, (const uint16_t *)W.wv,
+                                       qdim, kvdim, s.H, qkv16);
+        tile_lm_kernel<<<grid, 256>>>(ol, (const uint16_t *)W.wo, s.H, qdim, o16);  // rows H, K = q_dim
+        ld[l].wqkv_tc = ql;
+        ld[l].wo_tc = ol;
+      }
     }
     if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaDeviceSynchronize()) != cudaSuccess) {
       cudaGetLastError();

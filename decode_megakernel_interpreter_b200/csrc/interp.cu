@@ -15,24 +15,26 @@ struct SpecEntry {
   int rh, ro, rd, g, dpl;
   const void *(*kernel)();          // one sequence per instruction
   const void *(*kernel_batched)();  // up to kMaxBatch sequences (or null)
+  const void *(*kernel_batched_tqo)();  // the same with tensor-core QKV / O (or null)
 };
 // Shapes with a specialised build: Llama-3.2-1B (hidden 2048, 32/8 heads of
 // 64; also batched) and Llama-3.1-8B (hidden 4096, 32/8 heads of 128).
 const SpecEntry kSpecs[] = {
-    {4, 4, 4, 4, 2, spec_kernel_llama1b, spec_kernel_llama1b_batched},
-    {2, 2, 4, 4, 4, spec_kernel_llama8b, nullptr},
+    {4, 4, 4, 4, 2, spec_kernel_llama1b, spec_kernel_llama1b_batched, spec_kernel_llama1b_batched_tqo},
+    {2, 2, 4, 4, 4, spec_kernel_llama8b, nullptr, nullptr},
 };
 }  // namespace
 
-const void *interp_kernel_for(const KParams &p, bool specialised, int nb, int *variant) {
+const void *interp_kernel_for(const KParams &p, bool specialised, int nb, bool tqo, int *variant) {
   if (variant) *variant = 0;
   if (specialised && p.nkv > 0) {
     const int g = p.nq / p.nkv, dpl = p.d / 32;
     for (const SpecEntry &e : kSpecs)
       if (e.rh == p.Rh && e.ro == p.Ro && e.rd == p.Rd && e.g == g && e.dpl == dpl) {
-        if (nb > 1 && !e.kernel_batched) return nullptr;
+        const auto batched = tqo ? e.kernel_batched_tqo : e.kernel_batched;
+        if (nb > 1 && !batched) return nullptr;
         if (variant) *variant = 1;
-        return nb > 1 ? e.kernel_batched() : e.kernel();
+        return nb > 1 ? batched() : e.kernel();
       }
   }
   if (nb > 1) return nullptr;

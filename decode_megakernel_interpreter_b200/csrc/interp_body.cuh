@@ -263,7 +263,7 @@ struct Shared {
   uint32_t tmem_base;
   uint32_t mma_phase;
   unsigned long long mma_bar;
-  float tc_xch[64 * 16];  // gate/up on the tensor cores: up rows handed to the gate rows' warps
+  float tc_xch[128 * 16];  // tensor-core epilogues: rows handed between lane quarters
   uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
   float red[kComputeWarps][kMaxBatch];
   float argv[kComputeWarps][kMaxBatch];
@@ -490,8 +490,22 @@ __device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, 
   s.bytes = s.last = kPageBytes;
   s.npg = (int)I.b;
   switch (I.op) {
-    case OP_QKV: s.a = p.layers[I.layer].wqkv + (size_t)I.a * kPageElems; break;
-    case OP_OPROJ: s.a = p.layers[I.layer].wo + (size_t)I.a * kPageElems; break;
+    case OP_QKV:
+      if (p.layers[I.layer].wqkv_tc) {  // 128-row tiles of [q; k; v], H / 64 pages
+        s.a = p.layers[I.layer].wqkv_tc + (size_t)I.a * (p.H / 64) * kPageElems;
+        s.npg = (int)I.b * (p.H / 64);
+      } else {
+        s.a = p.layers[I.layer].wqkv + (size_t)I.a * kPageElems;
+      }
+      break;
+    case OP_OPROJ:
+      if (p.layers[I.layer].wo_tc) {  // 128-row tiles, q_dim / 64 pages
+        s.a = p.layers[I.layer].wo_tc + (size_t)I.a * (p.qdim / 64) * kPageElems;
+        s.npg = (int)I.b * (p.qdim / 64);
+      } else {
+        s.a = p.layers[I.layer].wo + (size_t)I.a * kPageElems;
+      }
+      break;
     case OP_GATEUP:
       if (p.layers[I.layer].wgu_tc) {  // 128-row tiles (64 gate + 64 up rows) of H / 64 pages
         s.a = p.layers[I.layer].wgu_tc + (size_t)I.a * (p.H / 64) * kPageElems;
@@ -1602,6 +1616,88 @@ __device__ __forceinline__ uint32_t down_tc_body(CCtx c, const Instr I) {
   return c.g;
 }
 
+// fused QKV on the tensor cores: a tile is 128 rows of [q; k; v] (two heads
+// of 64 or one of 128); RoPE pairs rows i and i + d/2, which sit in lane
+// quarters q and q ^ 1 (d = 64) or q ^ 2 (d = 128), so the quarters swap
+// their values through shared memory first
+template <int NB, int R>
+__device__ __forceinline__ uint32_t qkv_tc_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, Bn = p.B, d = p.d, hd = d / 2, nq = p.nq, nkv = p.nkv, kvdim = p.kvdim;
+  float inv[NB];
+  stage_norm<NB, StageIt<R>::v, true>(c, l, p.layers[l].attn_norm, false, inv);
+  px::fence_proxy_async_smem();
+  px::cbar();
+  const uint32_t tag = c.epoch;
+  float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
+  float *const kvc = p.kvcur + (size_t)l * Bn * 2 * kvdim;
+  uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
+  float *xch = c.sh->tc_xch;  // [128 rows][16 sequences]
+  tc_tiles<NB>(c, (int)I.b, p.H / 64, p.H, [&](int blk, int q, const float (&v)[16]) {
+    const int rr = q * 32 + c.lane, row = ((int)I.a + blk) * 128 + rr;
+    const int head = row / d, i = row % d;
+#pragma unroll
+    for (int b = 0; b < 16; ++b) xch[rr * 16 + b] = v[b];
+    tc_readers_sync();
+    const int partner = i < hd ? rr + hd : rr - hd;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= Bn) break;
+      const int pos = read_pos(c.sh, b);
+      const float mine = v[b] * inv[b], other = xch[partner * 16 + b] * inv[b];
+      float out = mine;
+      if (head < nq + nkv) {  // q and k heads are rotated
+        const float2 cs = __ldg(p.rope + (size_t)pos * hd + (i < hd ? i : i - hd));
+        out = i < hd ? mine * cs.x - other * cs.y : other * cs.y + mine * cs.x;
+      }
+      if (head < nq) {
+        px::st_tf(qrow + (size_t)b * p.qdim + row, out, tag);
+      } else {
+        const bool isk = head < nq + nkv;
+        const int gk = isk ? head - nq : head - nq - nkv;
+        const uint16_t bo = px::f2bf(out);
+        uint16_t *dst = (isk ? kl : vl) + (size_t)b * p.kv_bs + (size_t)gk * p.kv_hs + (size_t)pos * d;
+        dst[i] = bo;
+        px::st_tf(kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + (size_t)gk * d + i, px::bf16f(bo), tag);
+      }
+    }
+    tc_readers_sync();  // the exchange buffer is reused by the next tile
+  });
+  return c.g;
+}
+
+// output projection + residual on the tensor cores (attention output staged
+// as bf16 hi / lo; the residual rows of every sequence in one load group)
+template <int NB>
+__device__ __forceinline__ uint32_t oproj_tc_body(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, Bn = p.B, H = p.H;
+  stage_copy_tc<NB>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim);
+  const uint32_t tag = c.epoch;
+  float *const xout = p.xres + (size_t)l * Bn * H;
+  tc_tiles<NB>(c, (int)I.b, p.qdim / 64, p.qdim, [&](int blk, int q, const float (&v)[16]) {
+    const int row = ((int)I.a + blk) * 128 + q * 32 + c.lane;
+    float xin[NB];
+    for (LLRetry r;;) {
+      bool ok = true;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+        if (b < Bn) xin[b] = layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
+      if (ok || !ll_retry(p, c.sh, r, 9)) break;
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if (b >= Bn) break;
+      px::st_tf(xout + (size_t)b * H + row, xin[b] + v[b], tag);
+    }
+  });
+  return c.g;
+}
+
+template <int NB, int R>
+__device__ __noinline__ uint32_t op_qkv_tc(CCtx c, const Instr I) { return qkv_tc_body<NB, R>(c, I); }
+template <int NB>
+__device__ __noinline__ uint32_t op_oproj_tc(CCtx c, const Instr I) { return oproj_tc_body<NB>(c, I); }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_gateup_tc(CCtx c, const Instr I) { return gateup_tc_body<NB, R>(c, I); }
 template <int NB>
@@ -1987,10 +2083,13 @@ __device__ __forceinline__ int &sh_stat(CCtx &c) { return c.sh->stat_cwait; }
 // down-projection pages (RD), the query heads per KV head (G) and head_dim / 32
 // (DPL).  With every value fixed, each op body is inlined into the interpreter
 // loop (no call, no spills across a call boundary); the shape-generic build
-// (all zero) reaches the bodies through calls selected at run time.
-template <int RH_, int RO_, int RD_, int G_, int DPL_>
+// (all zero) reaches the bodies through calls selected at run time.  TQO
+// (batched builds): QKV and the O projection may run as tensor-core tiles; a
+// build of its own, since the extra op bodies raise every body's spills.
+template <int RH_, int RO_, int RD_, int G_, int DPL_, bool TQO_ = false>
 struct Spec {
   static constexpr bool fixed = RH_ > 0;
+  static constexpr bool TQO = TQO_;
   static constexpr int RH = RH_, RO = RO_, RD = RD_, G = G_, DPL = DPL_;
 };
 using SpecGeneric = Spec<0, 0, 0, 0, 0>;
@@ -2066,6 +2165,12 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
     c.tr = tr;
     switch (I.op) {
       case OP_QKV:
+        if constexpr (NB > 1 && S::fixed && S::TQO) {
+          if (p.layers[I.layer].wqkv_tc) {
+            c.g = op_qkv_tc<NB, S::RH>(c, I);
+            break;
+          }
+        }
         if constexpr (kInline) c.g = qkv_body<NB, S::RH>(c, I);
         else if constexpr (S::fixed) c.g = op_qkv<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_qkv, NB, p.Rh, c, I);
@@ -2076,6 +2181,12 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         else c.g = op_attn(c, I);
         break;
       case OP_OPROJ:
+        if constexpr (NB > 1 && S::fixed && S::TQO) {
+          if (p.layers[I.layer].wo_tc) {
+            c.g = op_oproj_tc<NB>(c, I);
+            break;
+          }
+        }
         if constexpr (kInline) c.g = oproj_body<NB, S::RO>(c, I);
         else if constexpr (S::fixed) c.g = op_oproj<NB, S::RO>(c, I);
         else MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);

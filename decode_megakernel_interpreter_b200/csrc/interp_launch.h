@@ -16,8 +16,9 @@ int shared_bytes_fixed(int num_pages, size_t act_floats);
 // instruction (1, or kMaxBatch for batched plans): a shape-specialised build
 // when one exists and `specialised` is set (*variant = 1), else the
 // shape-generic one (*variant = 0).  Batched plans have specialised builds
-// only; nullptr when the shape has none.
-const void *interp_kernel_for(const KParams &p, bool specialised, int nb, int *variant);
+// only (`tqo`: the build with QKV and the O projection on the tensor cores);
+// nullptr when the shape has none.
+const void *interp_kernel_for(const KParams &p, bool specialised, int nb, bool tqo, int *variant);
 // The raw-layout variant (weights read in the caller's layout).
 const void *interp_kernel_raw();
 // Allow `smem` bytes of dynamic shared memory for fn and report how many of
@@ -29,5 +30,6 @@ cudaError_t launch_interp(const void *fn, const KParams &p, int grid, int smem, 
 // shape-specialised kernels (interp_spec_*.cu)
 const void *spec_kernel_llama1b();
 const void *spec_kernel_llama1b_batched();
+const void *spec_kernel_llama1b_batched_tqo();
 const void *spec_kernel_llama8b();
 }  // namespace mk

@@ -71,6 +71,8 @@ struct LayerDev {
   // per page, K-major without swizzle); null otherwise
   const uint16_t *wgu_tc;   // [F/64 tiles: 64 gate + 64 up rows][H/64 pages]
   const uint16_t *wd_tc;    // [F/KCd pieces][H/128 tiles][KCd/64 pages]
+  const uint16_t *wqkv_tc;  // [(q_dim + 2 kv_dim)/128 tiles of [q; k; v] rows][H/64 pages]
+  const uint16_t *wo_tc;    // [H/128 tiles][q_dim/64 pages]
 };
 
 // Per-layer pointers to the caller's weights in their own [out][in] layout

@@ -137,15 +137,25 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   };
   std::vector<int> n_down(s.L, 0), n_qkv(s.L, 0), n_o(s.L, 0);
   p.tensor = req.tensor;
+  p.tensor_qkv_o = req.tensor && req.tensor_qkv_o;
   p.gu_rows_unit = p.tensor ? 64 : p.Rh / 2;
   p.dn_rows_unit = p.tensor ? 128 : p.Rd;
   const int gu_units = p.tensor ? s.F / 64 : p.P_gu;
   const int dn_units = p.tensor ? s.H / 128 : p.P_dp;
   const int64_t gu_unit_bytes = p.tensor ? (int64_t)(s.H / 64) * kPageBytes : kPageBytes;
+  // QKV: pages, or 128-row tiles of [q; k; v] (128 / Rh pages of the batch-1
+  // page numbering each); O projection: pages, or 128-row tiles
+  const int qdim = s.nq * s.d, kvdim = s.nkv * s.d;
+  const int qkv_units = p.tensor_qkv_o ? (qdim + 2 * kvdim) / 128 : p.P_qkv;
+  const int o_units = p.tensor_qkv_o ? s.H / 128 : p.P_o;
+  const int64_t qkv_unit_bytes = p.tensor_qkv_o ? (int64_t)(s.H / 64) * kPageBytes : kPageBytes;
+  const int64_t o_unit_bytes = p.tensor_qkv_o ? (int64_t)(qdim / 64) * kPageBytes : kPageBytes;
+  p.qkv_pages_unit = p.tensor_qkv_o ? 128 / p.Rh : 1;
+  p.o_rows_unit = p.tensor_qkv_o ? 128 : p.Ro;
   const int64_t dn_unit_bytes = p.tensor ? (int64_t)(p.KCd / 64) * kPageBytes : kPageBytes;
   for (int l = 0; l < s.L; ++l) {
     // fused RMSNorm + QKV + RoPE
-    auto cq = split_even(p.P_qkv, parts);
+    auto cq = split_even(qkv_units, parts);
     n_qkv[l] = (int)cq.size();
     for (size_t i = 0; i < cq.size(); ++i) {
       Instr I = mk_instr(OP_QKV, l);
@@ -157,7 +167,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       }
       I.sig_ctr = p.ctr_qkv(l);
       I.sig_n = 1;
-      all.push_back({I, (int64_t)cq[i].count * kPageBytes, l * 8 + ST_QKV, (int)i});
+      all.push_back({I, (int64_t)cq[i].count * qkv_unit_bytes, l * 8 + ST_QKV, (int)i});
     }
     // split-KV attention
     int ord = 0;
@@ -176,7 +186,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
           all.push_back({I, bytes, l * 8 + ST_ATTN, ord++});
         }
     // O projection + residual
-    auto co = split_even(p.P_o, parts);
+    auto co = split_even(o_units, parts);
     n_o[l] = (int)co.size();
     for (size_t i = 0; i < co.size(); ++i) {
       Instr I = mk_instr(OP_OPROJ, l);
@@ -186,7 +196,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       I.wait_cnt = req.B * s.nkv;
       I.sig_ctr = p.ctr_o(l);
       I.sig_n = 1;
-      all.push_back({I, (int64_t)co[i].count * kPageBytes, l * 8 + ST_OPROJ, (int)i});
+      all.push_back({I, (int64_t)co[i].count * o_unit_bytes, l * 8 + ST_OPROJ, (int)i});
     }
     // RMSNorm + gate/up + SiLU; signals the down-projection K pieces it feeds
     // (units: pages of R/2 gate + R/2 up rows, or 128-row tensor-core tiles
@@ -259,6 +269,8 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       p.weight_bytes += (int64_t)x.ins.b * (x.ins.op == OP_LMHEAD   ? lm_unit_bytes
                                            : x.ins.op == OP_GATEUP ? gu_unit_bytes
                                            : x.ins.op == OP_DOWN   ? dn_unit_bytes
+                                           : x.ins.op == OP_QKV    ? qkv_unit_bytes
+                                           : x.ins.op == OP_OPROJ  ? o_unit_bytes
                                                                    : (int64_t)kPageBytes);
   }
   // the last LM page (or block) may be partial
@@ -376,7 +388,8 @@ void rw_sets(const PlanRequest &req, const Plan &p, const Instr &I, std::vector<
   switch (I.op) {
     case OP_QKV:
       layer_input_reads(req, p, l, 0, s.H, rd);
-      wr.push_back({B_QKV, (int64_t)l * p.P_qkv + I.a, (int64_t)l * p.P_qkv + I.a + I.b});
+      wr.push_back({B_QKV, (int64_t)l * p.P_qkv + (int64_t)I.a * p.qkv_pages_unit,
+                    (int64_t)l * p.P_qkv + (int64_t)(I.a + I.b) * p.qkv_pages_unit});
       break;
     case OP_ATTN: {
       const int pph = s.d / p.Rh;  // pages per head
@@ -395,7 +408,7 @@ void rw_sets(const PlanRequest &req, const Plan &p, const Instr &I, std::vector<
     }
     case OP_OPROJ: {
       rd.push_back({B_O, (int64_t)l * req.B * s.nkv, (int64_t)(l + 1) * req.B * s.nkv});
-      int64_t r0 = (int64_t)I.a * p.Ro, r1 = (int64_t)(I.a + I.b) * p.Ro;
+      int64_t r0 = (int64_t)I.a * p.o_rows_unit, r1 = (int64_t)(I.a + I.b) * p.o_rows_unit;
       layer_input_reads(req, p, l, r0, r1, rd);
       wr.push_back({B_XRES, (int64_t)l * s.H + r0, (int64_t)l * s.H + r1});
       break;

@@ -28,14 +28,19 @@ struct PlanRequest {
   // tensor cores (batched plans): gate/up, down and LM-head instructions
   // cover whole 128-row tiles of tiled weight copies (64 columns per page)
   bool tensor = false;
+  // with `tensor`: QKV and O-projection instructions as tensor-core tiles too
+  bool tensor_qkv_o = false;
 };
 
 struct Plan {
   // geometry
   int Rh = 0, Ro = 0, Rd = 0, KCd = 0, ndp = 0, S = 0;
   bool tensor = false;  // see PlanRequest
+  bool tensor_qkv_o = false;
   int gu_rows_unit = 0;  // act rows per gate/up unit (page, or 64 on the tensor cores)
   int dn_rows_unit = 0;  // output rows per down unit (page, or 128 on the tensor cores)
+  int qkv_pages_unit = 1;  // batch-1 QKV pages per QKV unit (1, or 128 / Rh for a tile)
+  int o_rows_unit = 0;     // output rows per O-projection unit (page, or 128)
   int P_qkv = 0, P_o = 0, P_gu = 0, P_dp = 0, P_lm = 0;  // pages per layer / piece / head
   // instructions: static mode = per-CTA queues back to back; dynamic = global order
   std::vector<Instr> instrs;

@@ -148,6 +148,12 @@ typedef struct {
                              (the rest of its page ring only buffers landed
                              pages); 0 = automatic (4), -1 = no cap; rounded
                              down to a multiple of the loader count (2) */
+  int32_t tensor_qkv_o;   /* batched plans (batch > 1): 1 = QKV and the O
+                             projection run on the tensor cores as well, as
+                             whole 128-row tiles (fewer, larger instructions:
+                             on 148 SMs the Llama-1B shape then has 24 QKV and
+                             16 O tiles per layer, and the step is slower);
+                             0 = on CUDA cores (default).  Ignored at batch 1 */
 } mk_plan_opts;
 
 /*

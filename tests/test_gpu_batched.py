@@ -92,6 +92,17 @@ def test_llama1b_batch16_modes_agree(b16):
             np.testing.assert_array_equal(a, b)
 
 
+def test_llama1b_batch16_tensor_qkv_o_matches_oracle(b16):
+    """QKV (with RoPE and the K/V append) and the O projection as tensor-core
+    tiles: every sequence against the oracle, and the per-op path agrees bit
+    for bit."""
+    w, lengths, model = b16
+    ref = _run(w, lengths, model, 2, dict(tensor_qkv_o=True), check_oracle=True)
+    got = _run(w, lengths, model, 2, dict(tensor_qkv_o=True, exec_mode="per_op"), check_oracle=False)
+    for a, b in zip(ref, got):
+        np.testing.assert_array_equal(a, b)
+
+
 def test_batched_plan_needs_a_batched_build():
     """Shapes without a batched build refuse batch > 1 (the tiny shape)."""
     s = synth.TINY

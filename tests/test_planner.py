@@ -171,3 +171,26 @@ def test_batched_plan_uses_tensor_core_tiles():
     assert sum(i.b for i in lm) == -(-V // 128)
     err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=16), 148, steps=1, seed=5, timeout_ms=20000)
     assert err == ""
+
+
+def test_batched_plan_tensor_qkv_o_tiles():
+    """With tensor_qkv_o, QKV covers the [q; k; v] rows and the O projection
+    the hidden rows in 128-row tiles, each tile once per layer; the weight
+    bytes stay those of the batch-1 plan and the counter protocol holds."""
+    cfg1 = cfg_for("llama1b")
+    *_, info1 = mk.mk_host_plan(cfg1, mk.plan_opts(batch=1), 148)
+    cfg = cfg_for("llama1b_b16", max_batch=16)
+    opts = mk.plan_opts(batch=16, tensor_qkv_o=True)
+    instrs, off, ln, info = mk.mk_host_plan(cfg, opts, 148)
+    assert info.weight_bytes_per_step == info1.weight_bytes_per_step
+    rows_qkv = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    for l in range(cfg.n_layers):
+        for op, n in (("qkv", rows_qkv // 128), ("oproj", cfg.hidden // 128)):
+            spans = sorted((i.a, i.a + i.b) for i in instrs if i.op == OP[op] and i.layer == l)
+            covered = [u for a, e in spans for u in range(a, e)]
+            assert covered == list(range(n)), (op, l)
+    # the default keeps them on CUDA cores, one page per unit
+    instrs0, *_ = mk.mk_host_plan(cfg, mk.plan_opts(batch=16), 148)
+    assert sum(i.b for i in instrs0 if i.op == OP["qkv"] and i.layer == 0) == rows_qkv * cfg.hidden * 2 // 16384
+    err = mk.mk_host_plan_simulate(cfg, opts, 148, steps=1, seed=7, timeout_ms=20000)
+    assert err == ""
