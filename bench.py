@@ -193,66 +193,99 @@ def dist_setup(n):
     return world, rank, local
 
 
-def run_reference(args, world, rank):
-    """The CPU oracle (fp64) on this host's cores: the workload's decode steps,
-    a bounded sample of them."""
-    if rank != 0:
-        return
+def workload_config(w) -> dict:
+    """The config keys both arms report for a workload."""
+    s = w.shape
+    lengths = [int(x) for x in w.lengths()]
+    family = {4096: "Llama-3.1-8B", 2048: "Llama-3.2-1B"}.get(s.hidden)
+    desc = w.name
+    if family:
+        desc += (f": {family} shape ({s.n_layers} layers, hidden {s.hidden}, {s.n_q_heads}/{s.n_kv_heads} heads, "
+                 f"head_dim {s.head_dim}, ffn {s.ffn}, vocab {s.vocab}, {'tied' if s.tied else 'untied'})")
+    if w.ragged is None:
+        ctx = lengths[0]
+        desc += f", batch {w.batch}, KV pre-filled to {ctx}"
+    else:
+        ctx = f"U[{w.ragged[0]}, {w.ragged[1]}] per sequence (mean {sum(lengths) / len(lengths):.0f})"
+        desc += f", batch {w.batch}, KV pre-filled to {ctx}"
+    return {"workload": desc, "batch": w.batch, "context": ctx}
+
+
+def host_cores() -> int:
+    """Threads the OpenMP oracle runs with on this host."""
+    if os.environ.get("OMP_NUM_THREADS"):
+        return int(os.environ["OMP_NUM_THREADS"])
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_steps(w, model, steps: int, warmup: int, budget_s: float):
+    """Greedy decode steps of the whole batch (every sequence at its own
+    context length) with the fp64 oracle: `warmup` untimed steps, then up to
+    `steps` timed ones, stopping early once `budget_s` seconds are spent.
+    Returns (timed steps, seconds, warm-up steps done)."""
     import numpy as np
     import oracle
     import synth
-    w = synth.WORKLOADS[args.workload]
     s = w.shape
-    model = synth.make_model(s)
-    k, v = synth.alloc_kv(s, 1, w.context + args.steps + args.warmup + 2)
-    synth.fill_kv_prefix(s, k, v, [w.context])
+    lengths = [int(x) for x in w.lengths()]
+    k, v = synth.alloc_kv(s, w.batch, max(lengths) + steps + warmup + 2)
+    synth.fill_kv_prefix(s, k, v, lengths)
     orc = oracle.Oracle(s, model, "f64")
-    tok = int(synth.first_tokens(w)[0])
-    pos = w.context
+    tok = [int(t) for t in synth.first_tokens(w)]
+    pos = list(lengths)
+
+    def step():
+        for b in range(w.batch):
+            lg = orc.decode_step(k, v, b, tok[b], pos[b])
+            tok[b], pos[b] = int(np.argmax(lg)), pos[b] + 1
+
     t0 = time.perf_counter()
-    lg = orc.decode_step(k, v, 0, tok, pos)
-    t_step = time.perf_counter() - t0
-    tok, pos = int(np.argmax(lg)), pos + 1
-    budget = 150.0
-    n = max(1, min(args.steps, int(budget / max(t_step, 1e-3))))
-    t0 = time.perf_counter()
-    for _ in range(n):
-        lg = orc.decode_step(k, v, 0, tok, pos)
-        tok, pos = int(np.argmax(lg)), pos + 1
-    el = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    done_w = 0
+    for _ in range(warmup):  # untimed, bounded like the timed part
+        step()
+        done_w += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    n, t0 = 0, time.perf_counter()
+    while n < steps:
+        step()
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return n, time.perf_counter() - t0, done_w
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle (fp64) on this host's cores: the workload's decode steps
+    (all of its sequences), a bounded sample of them."""
+    if rank != 0:
+        return
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    model = synth.make_model(w.shape)
+    n, el, done_w = oracle_steps(w, model, args.steps, args.warmup, budget_s=150.0)
     val = n / el
-    sample = f"{n} of the {args.steps} requested decode steps of {args.workload} (1 untimed warm-up), fp64 oracle"
-    out = {"metric": METRIC, "value": val, "unit": "steps/s", "n_gpus": world, "steps": n, "warmup": 1,
+    sample = (f"{n} of the {args.steps} requested decode steps of {args.workload} "
+              f"({w.batch} sequence{'s' if w.batch > 1 else ''} each; {done_w} untimed warm-up), fp64 oracle")
+    out = {"metric": METRIC, "value": val, "unit": "steps/s", "n_gpus": world, "steps": n, "warmup": done_w,
            "ms_per_step": 1e3 * el / n, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "f64", "data": "synthetic (seeded bf16 weights ~N(0,0.02), KV ~N(0,1))",
-           "config": {"workload": args.workload, "batch": 1, "context": w.context},
+           "config": workload_config(w),
            "impl": "reference",
-           "cpu_baseline": {"value": val, "unit": "steps/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "cpu_baseline": {"value": val, "unit": "steps/s", "cores": host_cores(), "kind": "oracle",
+                            "sample": sample},
            "e2e": {"value": val, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
-def cpu_baseline(model, w, s, seconds=15.0):
-    import numpy as np
-    import oracle
-    import synth
-    k, v = synth.alloc_kv(s, 1, w.context + 64)
-    synth.fill_kv_prefix(s, k, v, [w.context])
-    orc = oracle.Oracle(s, model, "f64")
-    tok, pos = int(synth.first_tokens(w)[0]), w.context
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        lg = orc.decode_step(k, v, 0, tok, pos)
-        tok, pos, n = int(np.argmax(lg)), pos + 1, n + 1
-        el = time.perf_counter() - t0
-        if el >= seconds or n >= 60:
-            break
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": n / el, "unit": "steps/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} consecutive decode steps of {w.name} (context {w.context}+), fp64 oracle, "
-                      f"{el:.1f} s of host time"}
+def cpu_baseline(model, w, seconds=15.0):
+    n, el, _ = oracle_steps(w, model, 60, 0, budget_s=seconds)
+    return {"value": n / el, "unit": "steps/s", "cores": host_cores(), "kind": "oracle",
+            "sample": f"{n} consecutive decode steps of {w.name} ({w.batch} sequence{'s' if w.batch > 1 else ''} "
+                      f"each, at the workload's context lengths), fp64 oracle, {el:.1f} s of host time"}
 
 
 def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
@@ -313,7 +346,6 @@ def main():
     B = w.batch
     K, W = args.steps, args.warmup
     lengths = [int(x) for x in w.lengths()]
-    ctx = lengths[0]
     max_seq = max(lengths) + K + W + 2
     model = synth.make_model(s)
     dev = harness.upload_model(model, s.tied)
@@ -416,10 +448,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": us_step / 1e3, "us_per_step": us_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 weights, fp32 arithmetic", "data": "synthetic",
-            "config": {"workload": f"{w.name}: Llama-3.2-1B shape (16 layers, hidden 2048, 32/8 heads, head_dim 64, "
-                                   f"ffn 8192, vocab 128256, tied), batch {B}, KV pre-filled to {ctx}, "
-                                   f"{K} greedy steps" if w.name == "llama1b" else w.name,
-                       "batch": B, "context": ctx, "exec_mode": args.exec_mode, "sched": args.sched,
+            "config": {**workload_config(w), "exec_mode": args.exec_mode, "sched": args.sched,
                        "kv_splits": info.kv_splits, "ctas": info.num_ctas, "smem_pages": info.num_pages,
                        "interpreter": "shape-specialised" if info.kernel_variant == 1 else "shape-generic",
                        "parallelism": "replicas only" if world > 1 else "single GPU",
@@ -436,7 +465,7 @@ def main():
         if bd:
             out["breakdown"] = bd
         if world == 1 and not args.no_cpu_baseline:
-            out["cpu_baseline"] = cpu_baseline(model, w, s)
+            out["cpu_baseline"] = cpu_baseline(model, w)
         print(json.dumps(out), flush=True)
     if pg:
         pg.barrier()

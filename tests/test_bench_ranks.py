@@ -73,3 +73,23 @@ def test_reference_arm_runs_on_rank_0_only(capsys):
     ns = argparse.Namespace(workload="tiny", steps=1, warmup=0, gpus=2)
     assert b.run_reference(ns, 2, 1) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line(capsys):
+    """Rank 0 prints one JSON line with the workload's config, the warm-up it
+    ran, and an e2e block without host-device bytes (the oracle runs on the
+    host)."""
+    import argparse
+    import json
+    import synth
+    b = _bench()
+    ns = argparse.Namespace(workload="tiny", steps=3, warmup=3, gpus=1)
+    b.run_reference(ns, 1, 0)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 3 and d["warmup"] == 3
+    assert d["config"] == b.workload_config(synth.WORKLOADS["tiny"])
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"] > 0
+    assert d["unit"] == "steps/s" and d["higher_is_better"] is True
