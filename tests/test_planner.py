@@ -194,3 +194,30 @@ def test_batched_plan_tensor_qkv_o_tiles():
     assert sum(i.b for i in instrs0 if i.op == OP["qkv"] and i.layer == 0) == rows_qkv * cfg.hidden * 2 // 16384
     err = mk.mk_host_plan_simulate(cfg, opts, 148, steps=1, seed=7, timeout_ms=20000)
     assert err == ""
+
+
+@pytest.mark.parametrize("tqo", [False, True])
+@pytest.mark.parametrize("sched,num_ctas", [("static", 37), ("dynamic", 148), ("dynamic", 16)])
+def test_batched_plan_other_grids(tqo, sched, num_ctas):
+    """Batched plans on smaller grids and with the dynamic queue: every
+    matrix row of every layer is covered exactly once, and the host
+    simulation of the counter protocol completes."""
+    cfg = cfg_for("llama1b_b16", max_batch=16)
+    opts = mk.plan_opts(batch=16, sched=sched, tensor_qkv_o=tqo)
+    instrs, off, ln, info = mk.mk_host_plan(cfg, opts, num_ctas)
+    assert [i.seq for i in sorted(instrs, key=lambda i: i.seq)] == list(range(len(instrs)))
+    H, F = cfg.hidden, cfg.ffn
+    qkv_rows = (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    rows_per_unit = {"qkv": 128 if tqo else 8192 // H, "oproj": 128 if tqo else 8192 // (cfg.n_q_heads * cfg.head_dim),
+                     "gateup": 64}
+    total = {"qkv": qkv_rows, "oproj": H, "gateup": F}
+    for l in (0, cfg.n_layers // 2, cfg.n_layers - 1):
+        for op, n in total.items():
+            units = sorted(u for i in instrs if i.op == OP[op] and i.layer == l for u in range(i.a, i.a + i.b))
+            assert units == list(range(n // rows_per_unit[op])), (op, l)
+        for k in range(F // 2048):
+            units = sorted(u for i in instrs if i.op == OP["down"] and i.layer == l and i.c == k
+                           for u in range(i.a, i.a + i.b))
+            assert units == list(range(H // 128)), ("down", l, k)
+    err = mk.mk_host_plan_simulate(cfg, opts, num_ctas, steps=1, seed=11, timeout_ms=30000)
+    assert err == ""
