@@ -27,8 +27,11 @@ typedef struct {
   uint8_t op;      /* 0 nop, 1 qkv, 2 attention, 3 o-proj, 4 gate/up, 5 down, 6 lm-head */
   uint8_t pad;
   uint16_t layer;  /* n_layers for the LM head */
-  uint32_t a;      /* matvec ops: first 16 KiB weight page; attention: kv head */
-  uint32_t b;      /* matvec ops: number of pages; attention: split index */
+  uint32_t a;      /* matvec ops: first unit (a 16 KiB weight page; in batched
+                      plans a 128-row tensor-core tile for gate/up (64 gate +
+                      64 up rows), down, LM head, and QKV / O projection with
+                      tensor_qkv_o); attention: kv head */
+  uint32_t b;      /* matvec ops: number of units; attention: split index */
   uint32_t c;      /* down: K piece; attention: sequence; lm-head: argmax slot */
   uint32_t wait_ctr, wait_cnt; /* wait until counter[wait_ctr] >= step * wait_cnt
                                   (wait_ctr = 0xFFFFFFFF: no wait) */

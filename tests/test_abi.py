@@ -73,3 +73,44 @@ def test_struct_layouts_match_headers():
     assert ctypes.sizeof(mk.mk_instr_desc) == 32
     assert ctypes.sizeof(mk.mk_config) == 56
     assert ctypes.sizeof(mk.mk_plan_opts) == 48
+
+
+C_TYPES = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "uint32_t": ctypes.c_uint32,
+           "uint16_t": ctypes.c_uint16, "uint8_t": ctypes.c_uint8, "float": ctypes.c_float,
+           "double": ctypes.c_double}
+
+
+def header_struct(name):
+    """(field, C type) of `typedef struct { ... } name;` in the public headers
+    (pointer fields typed "ptr")."""
+    for h in ("mk.h", "mk_host.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        m = re.search(r"typedef struct \{([^}]*)\}\s*" + name + r"\s*;", src)
+        if m:
+            out = []
+            for decl in m.group(1).split(";"):
+                decl = decl.strip()
+                if not decl:
+                    continue
+                f = re.match(r"(?:const\s+)?(\w+)\s*(\*?)\s*(\w+(?:\s*,\s*\w+)*)$", decl)
+                assert f, decl
+                for fld in f.group(3).split(","):
+                    out.append((fld.strip(), "ptr" if f.group(2) else f.group(1)))
+            return out
+    raise AssertionError(name)
+
+
+@pytest.mark.parametrize("name", ["mk_config", "mk_plan_opts", "mk_plan_info", "mk_instr_desc", "mk_layer_weights",
+                                  "mk_weights", "mk_kv_cache"])
+def test_binding_structs_follow_the_headers(name):
+    """Field names, order and types of the ctypes mirrors equal the C
+    declarations (a field added on one side only fails here)."""
+    want = header_struct(name)
+    got = getattr(mk, name)._fields_
+    assert [n for n, _ in got] == [n for n, _ in want]
+    for (n, ct), (_, hc) in zip(got, want):
+        if hc == "ptr":
+            assert ct in (ctypes.c_void_p,) or issubclass(ct, ctypes._Pointer), n
+        else:
+            assert ct is C_TYPES[hc], (n, ct, hc)
