@@ -114,3 +114,23 @@ def test_binding_structs_follow_the_headers(name):
             assert ct in (ctypes.c_void_p,) or issubclass(ct, ctypes._Pointer), n
         else:
             assert ct is C_TYPES[hc], (n, ct, hc)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """Without libmk.so there is no fallback: loading raises."""
+    monkeypatch.setattr(mk, "_lib", None)
+    with pytest.raises(ImportError):
+        mk.load(str(tmp_path / "libmk.so"))
+
+
+def test_product_code_never_imports_the_oracle():
+    """The engine package and its sources name neither the oracle package nor
+    its library (only tests, the smoke entry and the bench's CPU legs may)."""
+    pkg = os.path.join(ROOT, "decode_megakernel_interpreter_b200")
+    for dirpath, _, files in os.walk(pkg):
+        if "_build" in dirpath:
+            continue
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert not re.search(r"\bimport oracle\b|from oracle\b|liboracle|llama_oracle", src), f
