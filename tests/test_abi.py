@@ -134,3 +134,44 @@ def test_product_code_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 src = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert not re.search(r"\bimport oracle\b|from oracle\b|liboracle|llama_oracle", src), f
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "mk.h"
+#include "mk_host.h"
+
+int main(void) {
+  mk_handle *h = (mk_handle *)1;
+  mk_config cfg;
+  memset(&cfg, 0, sizeof cfg);
+  if (mk_create(NULL, NULL, NULL, &h) != MK_ERR_INVALID_ARG || h != NULL) return 1;
+  if (mk_plan(NULL, NULL) != MK_ERR_INVALID_ARG) return 2;
+  if (mk_decode_step(NULL, NULL, NULL, NULL, NULL, NULL) != MK_ERR_INVALID_ARG) return 3;
+  if (strcmp(mk_status_string(MK_OK), "ok") != 0) return 4;
+  mk_destroy(NULL);
+  printf("%zu %zu %zu\n", sizeof(mk_config), sizeof(mk_plan_opts), sizeof(mk_instr_desc));
+  return 0;
+}
+"""
+
+
+def test_headers_compile_as_c_and_link(tmp_path):
+    """include/*.h are plain C: a C99 program includes them, links libmk.so
+    and calls the argument checks (no GPU needed); struct sizes agree with
+    the binding's."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    lib = mk.LIB_PATH
+    src = tmp_path / "abi_check.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi_check"
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe), lib, "-Wl,-rpath," + os.path.dirname(lib)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    sizes = [int(x) for x in out.stdout.split()]
+    assert sizes == [ctypes.sizeof(mk.mk_config), ctypes.sizeof(mk.mk_plan_opts), ctypes.sizeof(mk.mk_instr_desc)]
