@@ -102,9 +102,12 @@ typedef struct {
  *    and reads embed / wo / lm_head / norm weights in place.  The KV cache is
  *    written only at row positions[b] of sequence b by mk_decode_step.
  *  - Shapes implemented: head_dim in {64, 128}, hidden and n_q_heads*head_dim
- *    in {256, 512, 1024, 2048, 4096}, ffn a multiple of 256 (and of 2048 when
- *    above 2048), vocab >= 1, max_batch in [1, 16], max_seq >= 1.  Others give
- *    MK_ERR_UNSUPPORTED_SHAPE.
+ *    in {256, 512, 1024, 2048, 4096}, n_q_heads a multiple of n_kv_heads with
+ *    at most 8 query heads per KV head, ffn in {256, 512, 1024, 2048} or a
+ *    multiple of 2048 up to 16384 (the down projection's K pieces divide a
+ *    16 KiB page), vocab >= 1, max_batch in [1, 16], max_seq >= 1.  Others
+ *    give MK_ERR_UNSUPPORTED_SHAPE.  Batch > 1 is planned only for shapes with
+ *    a batched build (the Llama-3.2-1B shape).
  *  - Uses the current CUDA device.  Synchronous (returns when set-up is done).
  *  - Errors: MK_ERR_INVALID_ARG (NULL pointer, non-positive size),
  *    MK_ERR_UNSUPPORTED_SHAPE, MK_ERR_OUT_OF_MEMORY, MK_ERR_CUDA.

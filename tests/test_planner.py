@@ -221,3 +221,51 @@ def test_batched_plan_other_grids(tqo, sched, num_ctas):
             assert units == list(range(H // 128)), ("down", l, k)
     err = mk.mk_host_plan_simulate(cfg, opts, num_ctas, steps=1, seed=11, timeout_ms=30000)
     assert err == ""
+
+
+def _shape_grid():
+    """Shapes the engine accepts, beyond the named workloads: every hidden
+    size, both head dims, several GQA groups, FFN widths around the K-piece
+    size and vocabularies that leave a partial LM-head page."""
+    import random
+    rng = random.Random(17)
+    out = []
+    for H in (256, 512, 1024, 2048, 4096):
+        for d in (64, 128):
+            for qd in (256, 1024, 4096):
+                nq = qd // d
+                for g in (1, 2, 4, 8):
+                    if nq % g or (8192 // H) > d or d % (8192 // H):
+                        continue
+                    F = rng.choice([256, 512, 1024, 2048, 6144, 14336, 16384])
+                    if F % max(1, (8192 // H) // 2):
+                        continue
+                    V = rng.choice([1000, 4096, 32003])
+                    out.append((H, d, nq, nq // g, F, V))
+    rng.shuffle(out)
+    return out[:24]
+
+
+@pytest.mark.parametrize("H,d,nq,nkv,F,V", _shape_grid())
+def test_plan_structure_shape_grid(H, d, nq, nkv, F, V):
+    """Page coverage, queue order and counter targets for shapes beyond the
+    named workloads, on a full and a small grid, and the counter protocol on
+    the small grid."""
+    shape = dict(n_layers=2, hidden=H, n_q_heads=nq, n_kv_heads=nkv, head_dim=d, ffn=F, vocab=V,
+                 rms_eps=1e-5, rope_theta=1e4, tied=V == 4096)
+    cfg = mk.make_config(shape, 1, 300)
+    for num_ctas in (148, 13):
+        instrs, off, ln, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1), num_ctas)
+        check_structure(cfg, instrs, off, ln, num_ctas)
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1), 13, steps=1, seed=H + F, timeout_ms=30000)
+    assert err == ""
+
+
+@pytest.mark.parametrize("F", [768, 1280, 3072, 18432])
+def test_unsupported_ffn_widths_rejected(F):
+    """FFN widths outside the documented set are refused by the planner."""
+    shape = dict(n_layers=2, hidden=1024, n_q_heads=16, n_kv_heads=4, head_dim=64, ffn=F, vocab=4096,
+                 rms_eps=1e-5, rope_theta=1e4, tied=True)
+    with pytest.raises(mk.MkError) as e:
+        mk.mk_host_plan(mk.make_config(shape, 1, 64), mk.plan_opts(batch=1), 8)
+    assert e.value.code == mk.MK_ERR_UNSUPPORTED_SHAPE
