@@ -259,6 +259,11 @@ def test_plan_structure_shape_grid(H, d, nq, nkv, F, V):
         check_structure(cfg, instrs, off, ln, num_ctas)
     err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1), 13, steps=1, seed=H + F, timeout_ms=30000)
     assert err == ""
+    instrs, off, ln, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1, sched="dynamic"), 13)
+    check_structure(cfg, instrs, off, ln, 13, dynamic=True)
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched="dynamic"), 13, steps=2, seed=V,
+                                   timeout_ms=30000)
+    assert err == ""
 
 
 @pytest.mark.parametrize("F", [768, 1280, 3072, 18432])
