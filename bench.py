@@ -211,8 +211,20 @@ def workload_config(w) -> dict:
     return {"workload": desc, "batch": w.batch, "context": ctx}
 
 
+def _omp():
+    """The OpenMP runtime the oracle library links (None if not loadable)."""
+    import ctypes
+    try:
+        return ctypes.CDLL("libgomp.so.1")
+    except OSError:
+        return None
+
+
 def host_cores() -> int:
     """Threads the OpenMP oracle runs with on this host."""
+    g = _omp()
+    if g is not None:
+        return int(g.omp_get_max_threads())
     if os.environ.get("OMP_NUM_THREADS"):
         return int(os.environ["OMP_NUM_THREADS"])
     try:
@@ -283,9 +295,21 @@ def run_reference(args, world, rank):
 
 def cpu_baseline(model, w, seconds=15.0):
     n, el, _ = oracle_steps(w, model, 60, 0, budget_s=seconds)
-    return {"value": n / el, "unit": "steps/s", "cores": host_cores(), "kind": "oracle",
-            "sample": f"{n} consecutive decode steps of {w.name} ({w.batch} sequence{'s' if w.batch > 1 else ''} "
-                      f"each, at the workload's context lengths), fp64 oracle, {el:.1f} s of host time"}
+    out = {"value": n / el, "unit": "steps/s", "cores": host_cores(), "kind": "oracle",
+           "sample": f"{n} consecutive decode steps of {w.name} ({w.batch} sequence{'s' if w.batch > 1 else ''} "
+                     f"each, at the workload's context lengths), fp64 oracle, {el:.1f} s of host time"}
+    g = _omp()
+    if g is not None and w.batch == 1:
+        # the same oracle on one thread (a batched step would take minutes there)
+        prev = g.omp_get_max_threads()
+        g.omp_set_num_threads(1)
+        try:
+            n1, el1, _ = oracle_steps(w, model, 60, 0, budget_s=seconds / 2)
+        finally:
+            g.omp_set_num_threads(prev)
+        out["single_thread"] = {"value": n1 / el1, "unit": "steps/s", "cores": 1,
+                                "sample": f"{n1} decode steps of {w.name}, {el1:.1f} s"}
+    return out
 
 
 def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
