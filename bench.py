@@ -471,7 +471,7 @@ def main():
         out = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": us_step / 1e3, "us_per_step": us_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16 weights, fp32 arithmetic", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f32", "operand_dtype": "bf16 weights and KV cache", "data": "synthetic",
             "config": {**workload_config(w), "exec_mode": args.exec_mode, "sched": args.sched,
                        "kv_splits": info.kv_splits, "ctas": info.num_ctas, "smem_pages": info.num_pages,
                        "interpreter": "shape-specialised" if info.kernel_variant == 1 else "shape-generic",
