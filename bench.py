@@ -476,7 +476,8 @@ def main():
                        "kv_splits": info.kv_splits, "ctas": info.num_ctas, "smem_pages": info.num_pages,
                        "interpreter": "shape-specialised" if info.kernel_variant == 1 else "shape-generic",
                        "parallelism": "replicas only" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (weights streamed once per step, 2.5 GB)"},
+                       "l2": f"inputs larger than L2 (weights streamed once per step, "
+                             f"{info.weight_bytes_per_step / 1e9:.2f} GB; L2 126 MB)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "peak_kind": peak_kind, "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                          "traffic": ncu_traffic(args.workload), "algorithmic_bytes_per_step": bytes_step,
