@@ -63,9 +63,12 @@ _lib = None
 
 
 def lib():
+    """The oracle library: liboracle.so (built on first use), or the library
+    named by MK_ORACLE_LIB (the planted-mistake test loads mutated builds of
+    the same source that way)."""
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
+        L = ctypes.CDLL(os.environ.get("MK_ORACLE_LIB") or build())
         vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         for sfx, real in (("_f64", ctypes.c_double), ("_f32", ctypes.c_float)):
             getattr(L, "orc_bf16_to_real" + sfx).restype = real

@@ -358,6 +358,38 @@ def test_position_zero_step_reduces_to_dense_algebra():
     np.testing.assert_allclose(logits, widen(m["lm_head"]) @ f, rtol=1e-11, atol=1e-13)
 
 
+def test_step_rotates_q_and_k_by_the_position_and_leaves_v():
+    """At a position p > 0, the dumped q, k, v of layer 0 against the plain
+    products W a (numpy, a = rms(embed row) * gamma): v is the product itself
+    (not rotated); every (i, i + d/2) pair of q and k keeps its length and is
+    turned by exactly p * theta^(-2i/d); the cache row written at p holds the
+    bf16 rounding of the dumped k and v."""
+    s = synth.ModelShape(1, 128, 4, 2, 32, 256, 300, 1e-5, 1e4, True)
+    m = synth.make_model(s)
+    orc = oracle.Oracle(s, m, "f64")
+    P, tok, d, h2 = 37, 77, s.head_dim, s.head_dim // 2
+    k, v = synth.alloc_kv(s, 1, 48)
+    k[:, 0, :, :P] = synth.normal_bf16((1, s.n_kv_heads, P, d), synth.key(96, 4), 1.0)
+    v[:, 0, :, :P] = synth.normal_bf16((1, s.n_kv_heads, P, d), synth.key(96, 5), 1.0)
+    _, dump = orc.decode_step(k, v, 0, tok, P, dump=True)
+    L = {n: widen(m["layers"][0][n]) for n in synth.LAYER_TENSORS}
+    a = _np_rms(widen(m["embed"][tok]), L["attn_norm"], s.rms_eps)
+    np.testing.assert_allclose(dump["v"][0], L["wv"] @ a, rtol=1e-12, atol=1e-15)
+    want_angle = P * s.rope_theta ** (-2.0 * np.arange(h2) / d)
+    for name, W in (("q", L["wq"]), ("k", L["wk"])):
+        raw = (W @ a).reshape(-1, d)
+        got = dump[name][0].reshape(-1, d)
+        r0, r1, g0, g1 = raw[:, :h2], raw[:, h2:], got[:, :h2], got[:, h2:]
+        np.testing.assert_allclose(np.hypot(g0, g1), np.hypot(r0, r1), rtol=1e-12)
+        turn = np.angle((g0 + 1j * g1) / (r0 + 1j * r1))
+        diff = np.angle(np.exp(1j * (turn - want_angle[None, :])))
+        assert np.max(np.abs(diff)) < 1e-9, name
+    for g in range(s.n_kv_heads):
+        kb = [oracle.real_to_bf16(float(x)) for x in dump["k"][0].reshape(-1, d)[g]]
+        vb = [oracle.real_to_bf16(float(x)) for x in dump["v"][0].reshape(-1, d)[g]]
+        assert list(k[0, 0, g, P]) == kb and list(v[0, 0, g, P]) == vb
+
+
 def test_gqa_contiguous_groups():
     """KV head 0 holds V = +1, KV head 1 holds V = -1 at every earlier
     position; with contiguous grouping query heads 0,1 read head 0 and heads
