@@ -17,7 +17,8 @@ import oracle
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 ODIR = os.path.join(ROOT, "oracle")
 
-# (name, regex, replacement): each must match at least once
+# (name, regex, replacement[, "c" for the wrapper file]): each must match at
+# least once
 MUTANTS = [
     ("gqa_interleaved", r"int gh = h / grp;", "int gh = h % nkv;"),
     ("swiglu_swapped", r"g\[i\] = F\(orc_silu\)\(g\[i\]\) \* u\[i\];", "g[i] = F(orc_silu)(u[i]) * g[i];"),
@@ -42,18 +43,31 @@ MUTANTS = [
     ("no_attention_residual", r"(F\(orc_matvec\)\(L->wo, o, H, qd, t\);\s*for \(int i = 0; i < H; \+\+i\) x\[i\]) \+= t\[i\];",
      r"\1 = t[i];"),
     ("bf16_truncates", r"nearbyint\(ldexp\(m, 8\)\)", "trunc(ldexp(m, 8))"),
+    ("rmsnorm_sum_not_mean", r"\(double\)\(ss / \(R\)n \+ \(R\)eps\)", "(double)(ss + (R)eps)"),
+    ("silu_sign", r"\(R\)exp\(-\(double\)z\)", "(R)exp((double)z)"),
+    ("final_norm_skipped", r"F\(orc_rmsnorm\)\((x|X \+ \(int64_t\)p \* H), m->final_norm, H, sh->rms_eps, a\);",
+     r"for (int i_ = 0; i_ < H; ++i_) a[i_] = (\1)[i_];"),
+    ("no_ffn_residual", r"(F\(orc_matvec\)\(L->w_down, g, H, Fd, t\);\s*for \(int i = 0; i < H; \+\+i\) x\[i\]) \+= t\[i\];",
+     r"\1 = t[i];"),
+    ("embedding_row_shifted", r"m->embed\[\(int64_t\)(token|tokens\[p\]) \* H \+ i\]",
+     r"m->embed[(int64_t)((\1 + 1) % sh->vocab) * H + i]"),
+    ("lm_head_reads_embedding", r"F\(orc_matvec\)\(m->lm_head,", "F(orc_matvec)(m->embed,"),
+    ("argmax_last_maximum", r"if \(x\[i\] > x\[best\]\) best = i;", "if (x[i] >= x[best]) best = i;", "c"),
 ]
 
 
-def _build_mutant(tmp, name, pat, rep):
+def _build_mutant(tmp, name, pat, rep, where="body"):
+    """Copy the oracle source, apply one mutation to the body (or to the
+    wrapper, where = "c") and build it with the oracle's own flags."""
     d = os.path.join(tmp, name)
     os.makedirs(d)
-    for f in ("llama_oracle.c", "llama_oracle.h"):
+    files = {"body": "llama_oracle_body.h", "c": "llama_oracle.c"}
+    for f in ("llama_oracle.c", "llama_oracle.h", "llama_oracle_body.h"):
         shutil.copy(os.path.join(ODIR, f), d)
-    body = open(os.path.join(ODIR, "llama_oracle_body.h")).read()
-    new, n = re.subn(pat, rep, body)
+    target = os.path.join(d, files[where])
+    new, n = re.subn(pat, rep, open(target).read())
     assert n >= 1, f"mutation {name} does not apply"
-    with open(os.path.join(d, "llama_oracle_body.h"), "w") as fh:
+    with open(target, "w") as fh:
         fh.write(new)
     so = os.path.join(d, "liboracle.so")
     subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", so, os.path.join(d, "llama_oracle.c"), "-lm"])
@@ -77,7 +91,7 @@ def test_unmutated_copy_passes(tmp_path):
 def test_every_planted_mistake_fails_a_pin(tmp_path):
     if shutil.which("gcc") is None:
         pytest.skip("no C compiler")
-    libs = [(name, _build_mutant(str(tmp_path), name, pat, rep)) for name, pat, rep in MUTANTS]
+    libs = [(m[0], _build_mutant(str(tmp_path), *m)) for m in MUTANTS]
     with ThreadPoolExecutor(max_workers=4) as ex:
         results = list(ex.map(lambda nl: (nl[0],) + _pins_fail(nl[1]), libs))
     survivors = [name for name, rc, _ in results if rc != 1]
