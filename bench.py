@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--inflight", type=int, default=0, help="bulk-copy pages in flight per CTA (0 = default)")
     ap.add_argument("--tensor-qkv-o", action="store_true",
                     help="batched plans: QKV and O projection on the tensor cores too")
+    ap.add_argument("--compare-modes", action="store_true",
+                    help="single GPU: also time the per-op path (with and without a CUDA graph) and the dynamic "
+                         "queue on the same workload, reported under \"comparison\"")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="add a per-instruction-class time breakdown")
@@ -426,6 +429,37 @@ def main():
     value = job_rate(world, K, ms)
     launches_per_step = 1 if args.exec_mode.startswith("megakernel") else s.n_layers * 5 + 1
 
+    # the comparison paths on the same workload and buffers (opt-in): re-plan,
+    # warm up, time K steps the same way, then restore the measured plan
+    comparison = None
+    if args.compare_modes:
+        if world > 1:
+            raise SystemExit("--compare-modes runs on a single GPU")
+        comparison = {}
+        for label, over in (("per_op", dict(exec_mode="per_op")), ("per_op_graph", dict(exec_mode="per_op_graph")),
+                            ("dynamic_queue", dict(sched="dynamic", exec_mode="megakernel"))):
+            kw = {**plan_kw, **over}
+            if kw == plan_kw:
+                continue
+            eng.plan(**kw)
+            tokens.copy_(first)
+            for i in range(W):
+                step(i)
+            torch.cuda.synchronize()
+            tokens.copy_(first)
+            c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            c0.record(stream)
+            for i in range(K):
+                step(i)
+            c1.record(stream)
+            torch.cuda.synchronize()
+            rc = eng.status()
+            if rc != mk.MK_OK:
+                raise mk.MkError(rc, f"comparison {label}")
+            comparison[label] = {"us_per_step": 1e3 * c0.elapsed_time(c1) / K, "plan": over}
+        info = eng.plan(**plan_kw)
+        tokens.copy_(first)
+
     # end to end through the C ABI with host buffers: per step copy the token
     # and position in from pinned memory, run, read the next token back
     e2e = None
@@ -489,6 +523,8 @@ def main():
             out["e2e"] = e2e
         if bd:
             out["breakdown"] = bd
+        if comparison is not None:
+            out["comparison"] = comparison
         if world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(model, w)
         print(json.dumps(out), flush=True)
