@@ -274,3 +274,16 @@ def test_unsupported_ffn_widths_rejected(F):
     with pytest.raises(mk.MkError) as e:
         mk.mk_host_plan(mk.make_config(shape, 1, 64), mk.plan_opts(batch=1), 8)
     assert e.value.code == mk.MK_ERR_UNSUPPORTED_SHAPE
+
+
+@pytest.mark.parametrize("seed", [101, 202, 303])
+@pytest.mark.parametrize("name,batch,kw", [("llama1b", 1, {}), ("llama1b", 1, {"sched": "dynamic"}),
+                                            ("llama8b", 1, {}), ("llama1b_b16", 16, {}),
+                                            ("llama1b_b16", 16, {"tensor_qkv_o": True})])
+def test_simulation_more_seeds(seed, name, batch, kw):
+    """The counter protocol under other random delay patterns, on the full
+    grid, for the benchmarked plans (two steps, so the epoch targets of a
+    second step are exercised too)."""
+    cfg = cfg_for(name, max_batch=batch)
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=batch, **kw), 148, steps=2, seed=seed, timeout_ms=60000)
+    assert err == ""
