@@ -56,3 +56,23 @@ def test_llama1b_step_bytes_closed_form():
     want = (2 * s.n_params() + 2 * s.hidden) + per_pos * mean_rows + 4 * s.vocab
     assert got == pytest.approx(want, rel=0, abs=1e-3)
     assert round(got) == 2_507_846_656
+
+
+def test_batched_step_bytes_count_every_sequence():
+    """Batch 16: the weights once per step, the K/V of every sequence over its
+    own positions, one embedding row and one row of logits per sequence."""
+    b = _bench()
+    w = synth.WORKLOADS["llama1b_b16"]
+    s = w.shape
+    cfg = mk.make_config(s, 16, w.max_seq())
+    *_, info16 = mk.mk_host_plan(cfg, mk.plan_opts(batch=16), 148)
+    *_, info1 = mk.mk_host_plan(mk.make_config(s, 1, 2048), mk.plan_opts(batch=1), 148)
+    assert info16.weight_bytes_per_step == info1.weight_bytes_per_step
+    lengths = [int(x) for x in w.lengths()]
+    positions = [[n + i for n in lengths] for i in range(3)]
+    got = b.step_bytes(s, info16.weight_bytes_per_step, positions, True)
+    per_pos = s.n_layers * s.n_kv_heads * s.head_dim * 2 * 2
+    norms = (2 * s.n_layers + 1) * s.hidden * 2
+    kv = sum(per_pos * (p + 2) for row in positions for p in row) / len(positions)
+    want = info16.weight_bytes_per_step + norms + 16 * (2 * s.hidden + 4 * s.vocab) + kv
+    assert got == pytest.approx(want, rel=0, abs=1e-3)
