@@ -11,7 +11,11 @@ JSON line.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mk|reference]
 
 N > 1 runs under torchrun: batch-1 decode does not shard, so every rank runs
-an independent replica ("replicas only"); value = all ranks' steps / max time.
+an independent replica ("replicas only", weak scaling); value = all ranks'
+steps / max time.  The batched workload (16 independent sequences) is split
+data-parallel: rank r decodes its own contiguous slice of the sequences, with
+the weights replicated and no collective (strong scaling); value = whole-batch
+steps / max time.
 --impl reference times the CPU oracle (the only reference this build has).
 """
 from __future__ import annotations
@@ -48,12 +52,16 @@ def parse():
     ap.add_argument("--inflight", type=int, default=0, help="bulk-copy pages in flight per CTA (0 = default)")
     ap.add_argument("--tensor-qkv-o", action="store_true",
                     help="batched plans: QKV and O projection on the tensor cores too")
-    ap.add_argument("--compare-modes", action="store_true",
-                    help="single GPU: also time the per-op path (with and without a CUDA graph) and the dynamic "
-                         "queue on the same workload, reported under \"comparison\"")
+    ap.add_argument("--use-tcgen05", type=int, default=0, choices=[-1, 0, 1],
+                    help="batched plans: tensor cores for the matrix instructions (0 = automatic, -1 = off)")
+    ap.add_argument("--no-compare-modes", action="store_true",
+                    help="skip timing the per-op path (with and without a CUDA graph) and the dynamic queue on "
+                         "the same workload after the timed region (single GPU; reported under \"comparison\")")
+    ap.add_argument("--compare-steps", type=int, default=32, help="timed steps of each comparison path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--breakdown", action="store_true", help="add a per-instruction-class time breakdown")
+    ap.add_argument("--no-breakdown", action="store_true",
+                    help="skip the traced step (per-instruction-class time breakdown) after the timed region")
     ap.add_argument("--no-logits", action="store_true", help="do not write logits_out")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: truncate the model to this many layers (not a bench number)")
@@ -183,8 +191,27 @@ def max_over_ranks(ms: float, pg, device: str) -> float:
 
 
 def job_rate(world: int, steps: int, ms: float) -> float:
-    """Whole-job throughput: every rank's steps over the job's time."""
+    """Whole-job throughput of independent replicas: every rank's steps over
+    the job's time."""
     return world * steps / (ms / 1e3)
+
+
+def shard_sequences(batch: int, world: int, rank: int):
+    """Data-parallel split of a batch of independent sequences: rank r decodes
+    the contiguous slice [start, start + count); slices differ by at most one
+    sequence and cover the batch once."""
+    if world > batch:
+        raise SystemExit(f"{world} ranks for {batch} sequences: every rank needs at least one")
+    base, rem = divmod(batch, world)
+    start = rank * base + min(rank, rem)
+    return start, base + (1 if rank < rem else 0)
+
+
+def sharded_rate(steps: int, ms: float) -> float:
+    """Whole-job throughput of a batch split across ranks: every rank advances
+    its slice by `steps` tokens, so the job advances the whole batch `steps`
+    times in the slowest rank's time."""
+    return steps / (ms / 1e3)
 
 
 def dist_setup(n):
@@ -370,24 +397,29 @@ def main():
         w = dataclasses.replace(w, name=f"{w.name}_{args.layers}layers",
                                 shape=dataclasses.replace(w.shape, n_layers=args.layers))
     s = w.shape
-    B = w.batch
     K, W = args.steps, args.warmup
-    lengths = [int(x) for x in w.lengths()]
+    all_lengths = [int(x) for x in w.lengths()]
+    all_first = [int(x) for x in synth.first_tokens(w)]
+    # batched workloads: this rank's slice of the sequences (data parallel);
+    # batch-1 workloads: a full replica per rank
+    sharded = w.batch > 1 and world > 1
+    seq0, B = shard_sequences(w.batch, world, rank) if sharded else (0, w.batch)
+    lengths = all_lengths[seq0:seq0 + B]
     max_seq = max(lengths) + K + W + 2
     model = synth.make_model(s)
     dev = harness.upload_model(model, s.tied)
     k, v = synth.alloc_kv(s, B, max_seq)
-    synth.fill_kv_prefix(s, k, v, w.lengths())
+    synth.fill_kv_prefix(s, k, v, lengths)
     kc, vc = harness.upload_kv(k, v)
     del k, v
     eng = harness.make_engine(s, dev, kc, vc, B, max_seq)
     plan_kw = dict(batch=B, kv_splits=args.kv_splits, sched=args.sched, exec_mode=args.exec_mode,
                    l2_prefetch_kb=args.l2_prefetch_kb, max_inflight_pages=args.inflight,
-                   tensor_qkv_o=args.tensor_qkv_o)
+                   tensor_qkv_o=args.tensor_qkv_o, use_tcgen05=args.use_tcgen05 if B > 1 else 0)
     eng.plan_kw = plan_kw
     info = eng.plan(**plan_kw)
     stream = torch.cuda.current_stream()
-    first = torch.tensor(synth.first_tokens(w), dtype=torch.int32, device="cuda")
+    first = torch.tensor(all_first[seq0:seq0 + B], dtype=torch.int32, device="cuda")
     tokens = first.clone()  # next_tokens_out aliases tokens: device-to-device feedback
     # positions of every sequence at every step (row i: step i)
     pos_host = torch.tensor([[n + i for n in lengths] for i in range(max(K, W) + 1)], dtype=torch.int32)
@@ -426,16 +458,16 @@ def main():
         raise mk.MkError(rc, "timed steps")
     ms = max_over_ranks(ms, pg, "cuda")
     us_step = 1e3 * ms / K
-    value = job_rate(world, K, ms)
+    value = sharded_rate(K, ms) if sharded else job_rate(world, K, ms)
     launches_per_step = 1 if args.exec_mode.startswith("megakernel") else s.n_layers * 5 + 1
 
     # the comparison paths on the same workload and buffers (opt-in): re-plan,
     # warm up, time K steps the same way, then restore the measured plan
     comparison = None
-    if args.compare_modes:
-        if world > 1:
-            raise SystemExit("--compare-modes runs on a single GPU")
-        comparison = {}
+    if not args.no_compare_modes and world == 1:
+        comparison = {"megakernel": {"us_per_step": us_step, "plan": {"exec_mode": args.exec_mode,
+                                                                       "sched": args.sched}}}
+        Kc = max(1, min(K, args.compare_steps))
         for label, over in (("per_op", dict(exec_mode="per_op")), ("per_op_graph", dict(exec_mode="per_op_graph")),
                             ("dynamic_queue", dict(sched="dynamic", exec_mode="megakernel"))):
             kw = {**plan_kw, **over}
@@ -448,15 +480,16 @@ def main():
             torch.cuda.synchronize()
             tokens.copy_(first)
             c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
             c0.record(stream)
-            for i in range(K):
+            for i in range(Kc):
                 step(i)
             c1.record(stream)
             torch.cuda.synchronize()
             rc = eng.status()
             if rc != mk.MK_OK:
                 raise mk.MkError(rc, f"comparison {label}")
-            comparison[label] = {"us_per_step": 1e3 * c0.elapsed_time(c1) / K, "plan": over}
+            comparison[label] = {"us_per_step": 1e3 * c0.elapsed_time(c1) / Kc, "steps": Kc, "plan": over}
         info = eng.plan(**plan_kw)
         tokens.copy_(first)
 
@@ -491,10 +524,13 @@ def main():
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1)
         ems = max_over_ranks(ems, pg, "cuda")
-        e2e = {"value": job_rate(world, K, ems), "unit": "steps/s", "h2d_bytes_per_step": 8 * B,
+        e2e = {"value": sharded_rate(K, ems) if sharded else job_rate(world, K, ems), "unit": "steps/s",
+               "h2d_bytes_per_step": 8 * B,
                "d2h_bytes_per_step": 4 * B, "us_per_step": 1e3 * ems / K}
 
-    bd = breakdown(eng, mk, info, tokens, pos_all[0], logits, torch.empty_like(tokens)) if args.breakdown else None
+    bd = None
+    if not args.no_breakdown:
+        bd = breakdown(eng, mk, info, tokens, pos_all[0], logits, torch.empty_like(tokens))
     eng.close()
 
     if rank == 0:
@@ -504,12 +540,20 @@ def main():
         achieved = bytes_step / (us_step * 1e-6) / 1e9
         out = {
             "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": K, "warmup": W,
-            "ms_per_step": us_step / 1e3, "us_per_step": us_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "operand_dtype": "bf16 weights and KV cache", "data": "synthetic",
+            "ms_per_step": us_step / 1e3, "us_per_step": us_step, "higher_is_better": True,
+            "scaling": "strong" if sharded else "weak",
+            "vs_baseline": None, "dtype": "f32", "operand_dtype": "bf16 weights and KV cache",
+            "exchange": ("fp32 rounded to 22 significant bits with a 2-bit step tag in the low mantissa bits"
+                         + ("; tensor-core operands bf16 hi + lo (about 16 significant bits)"
+                            if B > 1 and args.use_tcgen05 >= 0 else "")),
+            "data": "synthetic",
             "config": {**workload_config(w), "exec_mode": args.exec_mode, "sched": args.sched,
                        "kv_splits": info.kv_splits, "ctas": info.num_ctas, "smem_pages": info.num_pages,
                        "interpreter": "shape-specialised" if info.kernel_variant == 1 else "shape-generic",
-                       "parallelism": "replicas only" if world > 1 else "single GPU",
+                       "parallelism": ("data parallel: sequences split across ranks, weights replicated, "
+                                       "no collective" if sharded else
+                                       "replicas only" if world > 1 else "single GPU"),
+                       **({"sequences_per_rank": B} if sharded else {}),
                        "l2": f"inputs larger than L2 (weights streamed once per step, "
                              f"{info.weight_bytes_per_step / 1e9:.2f} GB; L2 126 MB)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,

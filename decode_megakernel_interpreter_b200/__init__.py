@@ -65,7 +65,7 @@ class mk_plan_opts(ctypes.Structure):
                 ("exec_mode", ctypes.c_int32), ("num_sms", ctypes.c_int32), ("trace", ctypes.c_int32),
                 ("wait_timeout_ns", ctypes.c_int64), ("l2_prefetch_kb", ctypes.c_int32),
                 ("debug_drop_producer", ctypes.c_int32), ("max_inflight_pages", ctypes.c_int32),
-                ("tensor_qkv_o", ctypes.c_int32)]
+                ("tensor_qkv_o", ctypes.c_int32), ("use_tcgen05", ctypes.c_int32)]
 
 
 class mk_plan_info(ctypes.Structure):
@@ -235,11 +235,11 @@ def make_config(shape, max_batch: int, max_seq: int) -> mk_config:
 def plan_opts(batch: int = 1, kv_splits: int = 0, sched: str = "static", exec_mode: str = "megakernel",
               num_sms: int = 0, trace: bool = False, wait_timeout_ns: int = 0, l2_prefetch_kb: int = 0,
               debug_drop_producer: bool = False, max_inflight_pages: int = 0,
-              tensor_qkv_o: bool = False) -> mk_plan_opts:
+              tensor_qkv_o: bool = False, use_tcgen05: int = 0) -> mk_plan_opts:
     return mk_plan_opts(batch, kv_splits, {"static": 0, "dynamic": 1}[sched],
                         {"megakernel": 0, "per_op": 1, "per_op_graph": 2, "megakernel_generic": 3}[exec_mode], num_sms, int(trace),
                         wait_timeout_ns, l2_prefetch_kb, int(debug_drop_producer), max_inflight_pages,
-                        int(tensor_qkv_o))
+                        int(tensor_qkv_o), int(use_tcgen05))
 
 
 class Engine:

@@ -324,9 +324,20 @@ PlanRequest make_request(const mk_config &c, const mk_plan_opts &o, int num_ctas
   r.dynamic = o.sched_mode == MK_SCHED_DYNAMIC;
   r.assumed_context = std::max(1, c.max_seq);
   r.drop_producer = o.debug_drop_producer != 0;
-  r.tensor = o.batch > 1;  // batched plans run gate/up, down and the LM head on the tensor cores
+  // batched plans run gate/up, down and the LM head on the tensor cores
+  // unless asked not to
+  r.tensor = o.batch > 1 && o.use_tcgen05 >= 0;
   r.tensor_qkv_o = o.tensor_qkv_o != 0;
   return r;
+}
+
+// use_tcgen05: -1, 0 or 1; 1 only for batched plans; the tensor-core QKV /
+// O projection only with the tensor cores on
+bool tensor_opts_ok(const mk_plan_opts &o) {
+  if (o.use_tcgen05 < -1 || o.use_tcgen05 > 1) return false;
+  if (o.use_tcgen05 == 1 && o.batch <= 1) return false;
+  if (o.tensor_qkv_o && o.use_tcgen05 < 0) return false;
+  return true;
 }
 
 void set_err(char *err, size_t n, const std::string &m) {
@@ -359,6 +370,8 @@ size_t act_floats_for(const mk_config &c, const Plan &p, int nb) {
   // warps' partials + the current K/V rows (bf16) + the warps' merge weights
   size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim + (size_t)G * (kComputeWarps + 2);
   size_t f = std::max(vec, attn);
+  // batched builds: the tensor-core epilogue exchange follows the staged vectors
+  if (nb > 1) f += kTcXchFloats;
   return (f + 31) / 32 * 32;
 }
 
@@ -474,6 +487,7 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   const bool one_launch = o.exec_mode == MK_EXEC_MEGAKERNEL || o.exec_mode == MK_EXEC_MEGAKERNEL_GENERIC;
   if (!one_launch && o.sched_mode == MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
   if (o.kv_splits < 0 || o.num_sms < 0 || o.wait_timeout_ns < 0) return MK_ERR_INVALID_ARG;
+  if (!tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
   cudaError_t ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) {
     cudaGetLastError();
@@ -850,7 +864,7 @@ extern "C" int mk_host_plan(const mk_config *cfg, const mk_plan_opts *opts, int3
   }
   if (num_ctas < 1) return MK_ERR_INVALID_ARG;
   mk_plan_opts o = opts ? *opts : default_opts(*cfg);
-  if (o.batch < 1 || o.batch > cfg->max_batch) return MK_ERR_INVALID_ARG;
+  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
   PlanRequest req = make_request(*cfg, o, num_ctas);
   Plan p;
   std::string e = build_plan(req, &p);
@@ -893,7 +907,7 @@ extern "C" int mk_host_plan_simulate(const mk_config *cfg, const mk_plan_opts *o
   }
   if (num_ctas < 1 || steps < 1 || timeout_ms < 1) return MK_ERR_INVALID_ARG;
   mk_plan_opts o = opts ? *opts : default_opts(*cfg);
-  if (o.batch < 1 || o.batch > cfg->max_batch) return MK_ERR_INVALID_ARG;
+  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
   PlanRequest req = make_request(*cfg, o, num_ctas);
   Plan p;
   std::string e = build_plan(req, &p);

@@ -179,8 +179,8 @@ __device__ __forceinline__ void ld_ll2(const llw *a, llw &x, llw &y) {
 __device__ __forceinline__ bool ll_fresh(llw w, uint32_t tag) { return (uint32_t)(w >> 32) == tag; }
 __device__ __forceinline__ float ll_f(llw w) { return __uint_as_float((uint32_t)w); }
 // Tagged fp32 activations (the bulk of the exchanged data): the value rounded
-// to 21 significant bits, its two lowest mantissa bits replaced by the step
-// number mod 4.  Every such word is rewritten every step, so the only stale
+// to 22 significant bits (21 stored mantissa bits and the implicit one), its
+// two lowest mantissa bits replaced by the step number mod 4.  Every such word is rewritten every step, so the only stale
 // value a reader can meet is the previous step's (or zero-filled memory
 // before the first step): a 2-bit tag tells them apart, and 4-byte words keep
 // the traffic and registers of plain fp32.
@@ -263,7 +263,6 @@ struct Shared {
   uint32_t tmem_base;
   uint32_t mma_phase;
   unsigned long long mma_bar;
-  float tc_xch[128 * 16];  // tensor-core epilogues: rows handed between lane quarters
   uint32_t slot_last[16];  // 1 + the last page issued into each ring slot (0: never)
   float red[kComputeWarps][kMaxBatch];
   float argv[kComputeWarps][kMaxBatch];
@@ -599,8 +598,8 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
   const uint32_t NP = (uint32_t)p.num_pages;
   const uint32_t cap = (uint32_t)p.max_inflight;
   const bool trace = (p.mode & MODE_TRACE) != 0;
-  uint32_t g = 0, last_issued = 0;
-  bool ok = true, any = false;
+  uint32_t g = 0;
+  bool ok = true;
   const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
   const unsigned dyn_base = dyn ? (epoch - 1u) * (unsigned)(p.n_instr + gridDim.x) : 0u;
   int claimed = 0;
@@ -693,8 +692,6 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
       if constexpr (RAW) {
         if (I.op == OP_QKV || I.op == OP_GATEUP || I.op == OP_DOWN || I.op == OP_OPROJ) {
           issue_page_raw(p, I, t, dst, &full[slot], pol_w, pol_kv, false);
-          any = true;
-          last_issued = gg;
           continue;
         }
       }
@@ -707,17 +704,13 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
         px::mbar_expect_tx(&full[slot], bytes);
         px::bulk_g2s(dst, ps.a + (size_t)t * ps.stride, bytes, &full[slot], pol_w);
       }
-      any = true;
-      last_issued = gg;
     }
     if (ltr) {
       ltr[6] = px::gtimer();
       ltr[9] = lwait;
     }
-    if (!ok) {
-      g = g0;  // not every page of this instruction was issued; drain by last_issued
-      break;
-    }
+    if (!ok) break;  // copies already issued land before the CTA exits: thread 0 waits on
+                     // each ring slot's last issued page (slot_last) at the end of the kernel
     if (px::ld_volatile(&sh->abort) || global_abort(p)) ok = false;
   }
   if (dyn && ok == false) {
@@ -726,8 +719,6 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
     __threadfence_block();
     *dyn_tail = claimed + 1;
   }
-  (void)any;
-  (void)last_issued;
 }
 
 // ============================================================== compute
@@ -742,6 +733,7 @@ struct CCtx {
   int cw, lane, ctid;
   uint32_t g;     // page sequence number (same as the loader's)
   unsigned long long *tr;  // this instruction's trace record (or null)
+  float *xch;     // batched builds: tensor-core epilogue exchange [128 rows][16 sequences]
 };
 
 // Register-resident view of the page ring (copied out of the context once per
@@ -1196,7 +1188,7 @@ __device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
         dst[i] = bu;
         dst[i + hd] = bw;
         float *cur = kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + gk * d;
-        px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 21 bits
+        px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 22 significant bits
         px::st_tf(cur + i + hd, px::bf16f(bw), tag);
       }
     }
@@ -1537,7 +1529,7 @@ __device__ __forceinline__ uint32_t gateup_tc_body(CCtx c, const Instr I) {
   px::cbar();
   const uint32_t tag = c.epoch;
   float *const aout = p.actb + (size_t)l * Bn * F;
-  float *xch = reinterpret_cast<float *>(c.sh->tc_xch);  // [64 rows][16 sequences]
+  float *xch = c.xch;  // [64 rows][16 sequences]
   tc_tiles<NB>(c, (int)I.b, p.H / 64, p.H, [&](int blk, int q, const float (&v)[16]) {
     const int r = (q & 1) * 32 + c.lane;  // row inside the tile's 64 gate / up rows
     if (q >= 2) {
@@ -1632,7 +1624,7 @@ __device__ __forceinline__ uint32_t qkv_tc_body(CCtx c, const Instr I) {
   float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
   float *const kvc = p.kvcur + (size_t)l * Bn * 2 * kvdim;
   uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
-  float *xch = c.sh->tc_xch;  // [128 rows][16 sequences]
+  float *xch = c.xch;  // [128 rows][16 sequences]
   tc_tiles<NB>(c, (int)I.b, p.H / 64, p.H, [&](int blk, int q, const float (&v)[16]) {
     const int rr = q * 32 + c.lane, row = ((int)I.a + blk) * 128 + rr;
     const int head = row / d, i = row % d;
@@ -2251,7 +2243,10 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   extern __shared__ __align__(128) uint8_t smem[];
   const int NP = p.num_pages;
   uint8_t *pages = smem;
-  const int act_stride = (int)(p.act_floats / NB);
+  // batched builds keep the tensor-core epilogue exchange at the end of the
+  // staging region (kTcXchFloats), after the NB staged vectors
+  const long long xch_floats = NB > 1 ? kTcXchFloats : 0;
+  const int act_stride = (int)((p.act_floats - xch_floats) / NB);
   float *act = reinterpret_cast<float *>(smem + (size_t)NP * kPageBytes);
   uint64_t *full = reinterpret_cast<uint64_t *>(act + p.act_floats);
   uint64_t *empty = full + NP;
@@ -2308,8 +2303,8 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
     if (lane == 0 && (!dyn || warp == 0))
       run_loader<RAW>(p, sh, pages, full, empty, q, dyn_fifo, dyn_tail, dyn_head, epoch, warp, dyn ? 1 : kLoaders);
   } else {
-    CCtx c{p, sh, pages, act, act_stride, full, empty, epoch, warp - kLoaders, lane,
-           (int)threadIdx.x - 32 * kLoaders, 0u, nullptr};
+    CCtx c{p,     sh,    pages, act, act_stride, full, empty, epoch, warp - kLoaders, lane, (int)threadIdx.x - 32 * kLoaders,
+           0u,    nullptr, NB > 1 ? act + (p.act_floats - xch_floats) : nullptr};
     run_compute<NB, S>(c, q, dyn_fifo, dyn_tail, dyn_head);
   }
   if constexpr (NB > 1) px::tc_fence_before();

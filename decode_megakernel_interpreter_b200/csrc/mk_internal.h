@@ -21,6 +21,7 @@ constexpr int kMaxKc = 4096;                  // largest K staged in one page ro
 constexpr int kMaxBatch = 16;
 constexpr int kMaxDownPieces = 8;             // ffn / 2048 at most
 constexpr int kDefaultInflight = 4;           // bulk-copy pages in flight per CTA
+constexpr int kTcXchFloats = 128 * 16;        // batched builds: tensor-core epilogue exchange (floats)
 
 // ---------------------------------------------------------------- opcodes
 // The instruction set of the decode step (the fused instructions the
@@ -114,7 +115,7 @@ struct KParams {
   uint16_t *kc, *vc;
   long long kv_ls, kv_bs, kv_hs;   // element strides: layer, batch, head (position stride = d)
   const float2 *rope;              // [max_seq][d/2] (cos, sin)
-  // activations: tagged fp32 words (value rounded to 21 significant bits, the
+  // activations: tagged fp32 words (value rounded to 22 significant bits, the
   // two low mantissa bits = step number mod 4)
   float *qbuf;                  // [L][B][q_dim]
   float *kvcur;                 // [L][B][2][kv_dim]  this step's K and V rows (bf16-rounded)

@@ -172,11 +172,22 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
                      (const uint16_t *)L.wo, (const uint16_t *)L.w_gate, (const uint16_t *)L.w_up,
                      (const uint16_t *)L.w_down};
   }
-  std::vector<unsigned char> key(sizeof(mk_config) + sizeof(int));
-  memcpy(key.data(), cfg, sizeof(mk_config));
-  memcpy(key.data() + sizeof(mk_config), &slot->sm_count, sizeof(int));
-  key.insert(key.end(), (unsigned char *)ld.data(), (unsigned char *)(ld.data() + s.L));
-  key.insert(key.end(), (unsigned char *)lr.data(), (unsigned char *)(lr.data() + s.L));
+  // what the uploaded tables depend on, field by field (a caller's mk_config
+  // may carry indeterminate padding bytes, so the struct is not copied whole)
+  std::vector<unsigned char> key;
+  auto put = [&key](const void *v, size_t n) {
+    key.insert(key.end(), static_cast<const unsigned char *>(v), static_cast<const unsigned char *>(v) + n);
+  };
+  const int32_t ints[] = {cfg->n_layers, cfg->hidden, cfg->n_q_heads, cfg->n_kv_heads, cfg->head_dim, cfg->ffn,
+                          cfg->vocab, cfg->tied_lm_head, cfg->max_batch, cfg->max_seq, slot->sm_count};
+  put(ints, sizeof ints);
+  put(&cfg->rms_eps, sizeof cfg->rms_eps);
+  put(&cfg->rope_theta, sizeof cfg->rope_theta);
+  for (int l = 0; l < s.L; ++l) {
+    const void *ptrs[] = {ld[l].wo, ld[l].attn_norm, ld[l].ffn_norm, lr[l].wq, lr[l].wk, lr[l].wv,
+                          lr[l].wo, lr[l].wg, lr[l].wu, lr[l].wd};
+    put(ptrs, sizeof ptrs);
+  }
   cudaError_t e = cudaSuccess;
   if (key != slot->key) {
     std::vector<float2> rope((size_t)cfg->max_seq * hd);
@@ -208,11 +219,12 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
     slot->key = key;
   }
   // every call starts from zeroed counters, status and tagged activations,
-  // step number 1
-  static const unsigned kOne = 1;
+  // step number 1: the epoch word lies in the zeroed range, so setting its
+  // lowest byte to 1 makes the little-endian word 1 (no host copy per call)
+  static_assert(sizeof(unsigned) == 4, "epoch word");
   e = cudaMemsetAsync(base, 0, sync_end, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(base + tagged_begin, 0, lay.off - tagged_begin, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(base + o_epoch, &kOne, sizeof kOne, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(base + o_epoch, 1, 1, st);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return MK_ERR_CUDA;

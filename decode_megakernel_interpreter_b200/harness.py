@@ -38,3 +38,22 @@ def kv_to_host(t: torch.Tensor) -> np.ndarray:
 
 def make_engine(shape, dev_model: dict, kc: torch.Tensor, vc: torch.Tensor, max_batch: int, max_seq: int) -> Engine:
     return Engine(shape, dev_model, kc, vc, max_batch, max_seq)
+
+
+def kv_row_to_host(t: torch.Tensor, b: int, p: int) -> np.ndarray:
+    """Row p of sequence b of a [L][B][n_kv][max_seq][d] cache: [L][n_kv][d]."""
+    return t[:, b, :, p].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def replace_norms(dev: dict, host: dict, device="cuda") -> dict:
+    """A device model sharing every matrix of `dev`, with the norm vectors
+    uploaded from `host`."""
+    out = dict(dev)
+    out["final_norm"] = to_device_bf16(host["final_norm"], device)
+    out["layers"] = []
+    for Ld, Lh in zip(dev["layers"], host["layers"]):
+        d = dict(Ld)
+        d["attn_norm"] = to_device_bf16(Lh["attn_norm"], device)
+        d["ffn_norm"] = to_device_bf16(Lh["ffn_norm"], device)
+        out["layers"].append(d)
+    return out

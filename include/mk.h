@@ -95,6 +95,8 @@ typedef struct {
 /*
  * mk_create: validate the shape, take the weight and KV pointers, and build the
  * device-side state (repacked weight copies, RoPE table, activation buffers).
+ * ("Hazy megakernel summary", section 四(二): the model's weights streamed
+ * page by page by the interpreter; the repacking makes each page one copy.)
  *  - Ownership: weights and the KV cache are BORROWED; they must stay valid
  *    until mk_destroy and the library never frees them.  The library keeps its
  *    own repacked copy of the fused QKV, gate/up and down-projection weights
@@ -156,11 +158,24 @@ typedef struct {
                              whole 128-row tiles (fewer, larger instructions:
                              on 148 SMs the Llama-1B shape then has 24 QKV and
                              16 O tiles per layer, and the step is slower);
-                             0 = on CUDA cores (default).  Ignored at batch 1 */
+                             0 = on CUDA cores (default).  Ignored at batch 1;
+                             needs the tensor cores (use_tcgen05 not -1) */
+  int32_t use_tcgen05;    /* 5th-generation tensor cores (tcgen05.mma with
+                             tensor-memory accumulators) for the matrix
+                             instructions of batched plans, where a step's
+                             matrix-vector products are dense contractions
+                             over the batch: 0 = automatic (on when
+                             batch > 1), 1 = on (MK_ERR_INVALID_ARG at
+                             batch 1, where every product is a matrix-vector
+                             product and CUDA-core FMAs are used), -1 = off
+                             (CUDA cores for every batch) */
 } mk_plan_opts;
 
 /*
- * mk_plan: build the instruction DAG for this batch size, partition it into
+ * mk_plan ("Hazy megakernel summary", section 四(二): every SM's instruction
+ * sequence is scheduled on the host ahead of time and one schedule serves
+ * many forward passes; "MegaKernel 日志", section on static and dynamic
+ * scheduling): build the instruction DAG for this batch size, partition it into
  * per-SM queues (or one global queue), set the dependency-counter targets,
  * check the plan (every queue follows one global topological order) and upload
  * it.  Call once; the plan is reused by every later mk_decode_step.  Calling it
@@ -174,7 +189,11 @@ int mk_plan(mk_handle *h, const mk_plan_opts *opts);
 
 /* ------------------------------------------------------------------ step */
 /*
- * mk_decode_step: one decode step for sequences b = 0..batch-1.
+ * mk_decode_step ("Hazy megakernel summary", section 四(二): one persistent
+ * kernel whose per-SM interpreter fetches, runs and retires the fused
+ * instructions; "Mirage Persistent Kernel" article, Part 2: the runtime loop
+ * of fetch task -> run -> notify event): one decode step for sequences
+ * b = 0..batch-1.
  *  - tokens          device int32 [batch]: the input token of each sequence.
  *  - positions       device int32 [batch]: its position p_b (0 <= p_b < max_seq).
  *                    The step writes the token's K and V at row p_b of the
@@ -195,7 +214,10 @@ int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions
                    float *logits_out, int32_t *next_tokens_out, void *stream);
 
 /*
- * mk_get_status: synchronise `stream` and return the first device-side error
+ * mk_get_status ("Hazy megakernel summary", section 四(二) 同步: the counters
+ * in global memory that replace kernel boundaries; every wait on them is
+ * bounded here, and a wait that gives up is reported by this call):
+ * synchronise `stream` and return the first device-side error
  * recorded since the last call (MK_ERR_TIMEOUT, MK_ERR_DEVICE_INPUT), or a CUDA
  * error (MK_ERR_CUDA), or MK_OK.  Clears the recorded device error.
  */

@@ -8,7 +8,9 @@ the megakernel pages measure (a Llama-3.2-1B-shaped decoder at batch 1,
 single sequence) plus a tiny model, a long-context, a batched and an 8B-shaped
 variant.  Trained weights are not needed: the shapes and the value
 distributions stand in for them (weights ~N(0, 0.02) in bf16, norm weights
-1.0, KV cache ~N(0, 1), token ids uniform over the vocabulary).
+1.0, KV cache ~N(0, 1), token ids uniform over the vocabulary).  Parity tests
+may also ask for norm weights ~N(1, sigma), one seeded stream per norm vector
+(``make_model(..., norm_sigma=...)``), so that a wrong use of them shows.
 
 Seeds: weights 0, KV cache 1, token ids 2, context lengths 3.
 """
@@ -31,6 +33,7 @@ KV_SIGMA = 1.0
 
 # tensor-kind ids used in stream keys
 K_EMBED, K_LM_HEAD, K_WQ, K_WK, K_WV, K_WO, K_WGATE, K_WUP, K_WDOWN = range(9)
+K_ATTN_NORM, K_FFN_NORM, K_FINAL_NORM = 9, 10, 11
 
 
 def build(force: bool = False) -> str:
@@ -53,6 +56,7 @@ def _L():
         _lib.syn_key.restype = u64
         _lib.syn_key.argtypes = [u64, u64, u64, u64]
         _lib.syn_normal_bf16.argtypes = [vp, u64, u64, dbl, u64]
+        _lib.syn_normal_bf16_mean.argtypes = [vp, u64, u64, dbl, dbl, u64]
         _lib.syn_normal_f32.argtypes = [vp, u64, u64, dbl]
         _lib.syn_uniform_i32.argtypes = [vp, u64, u64, i32, i32]
         _lib.syn_fill_bf16.argtypes = [vp, u64, f32]
@@ -70,6 +74,14 @@ def normal_bf16(shape, k: int, sigma: float, first: int = 0, out: np.ndarray | N
         out = np.empty(shape, dtype=np.uint16)
     assert out.dtype == np.uint16 and out.flags.c_contiguous and out.size == n
     _L().syn_normal_bf16(out.ctypes.data, n, k, sigma, first)
+    return out
+
+
+def normal_bf16_mean(shape, k: int, mean: float, sigma: float) -> np.ndarray:
+    """bf16 bit patterns of ``mean`` + stream ``k`` (the same normal values as
+    ``normal_bf16``, offset before the rounding)."""
+    out = np.empty(shape, dtype=np.uint16)
+    _L().syn_normal_bf16_mean(out.ctypes.data, out.size, k, mean, sigma, 0)
     return out
 
 
@@ -185,10 +197,20 @@ def layer_tensor_shape(s: ModelShape, name: str):
 _KIND = {"wq": K_WQ, "wk": K_WK, "wv": K_WV, "wo": K_WO, "w_gate": K_WGATE, "w_up": K_WUP, "w_down": K_WDOWN}
 
 
-def make_layer_tensor(s: ModelShape, layer: int, name: str, seed: int = SEED_WEIGHTS, out=None) -> np.ndarray:
-    shp = layer_tensor_shape(s, name)
+def make_norm(s: ModelShape, kind: int, layer: int, norm_sigma: float = 0.0, seed: int = SEED_WEIGHTS) -> np.ndarray:
+    """An RMSNorm weight vector: 1.0 everywhere (the workloads), or with
+    ``norm_sigma`` > 0 seeded values ~N(1, norm_sigma) from stream
+    key(seed, kind, layer)."""
+    if norm_sigma <= 0:
+        return fill_bf16((s.hidden,), 1.0)
+    return normal_bf16_mean((s.hidden,), key(seed, kind, layer), 1.0, norm_sigma)
+
+
+def make_layer_tensor(s: ModelShape, layer: int, name: str, seed: int = SEED_WEIGHTS, out=None,
+                      norm_sigma: float = 0.0) -> np.ndarray:
     if name.endswith("norm"):
-        return fill_bf16(shp, 1.0)
+        return make_norm(s, K_ATTN_NORM if name == "attn_norm" else K_FFN_NORM, layer, norm_sigma, seed)
+    shp = layer_tensor_shape(s, name)
     return normal_bf16(shp, key(seed, _KIND[name], layer), WEIGHT_SIGMA, out=out)
 
 
@@ -201,16 +223,35 @@ def make_lm_head(s: ModelShape, seed: int = SEED_WEIGHTS, out=None) -> np.ndarra
     return normal_bf16((s.vocab, s.hidden), key(seed, K_LM_HEAD, 0), WEIGHT_SIGMA, out=out)
 
 
-def make_model(s: ModelShape, seed: int = SEED_WEIGHTS) -> dict:
-    """All weights on the host: {'embed', 'lm_head', 'final_norm', 'layers': [dict]}."""
+def make_model(s: ModelShape, seed: int = SEED_WEIGHTS, norm_sigma: float = 0.0) -> dict:
+    """All weights on the host: {'embed', 'lm_head', 'final_norm', 'layers': [dict]}.
+    Norm weights are 1.0 unless ``norm_sigma`` > 0 (then ~N(1, norm_sigma),
+    a distinct seeded vector per norm and layer)."""
     embed = make_embed(s, seed)
     m = {
         "embed": embed,
         "lm_head": embed if s.tied else make_lm_head(s, seed),
-        "final_norm": fill_bf16((s.hidden,), 1.0),
-        "layers": [{n: make_layer_tensor(s, l, n, seed) for n in LAYER_TENSORS} for l in range(s.n_layers)],
+        "final_norm": make_norm(s, K_FINAL_NORM, 0, norm_sigma, seed),
+        "layers": [{n: make_layer_tensor(s, l, n, seed, norm_sigma=norm_sigma) for n in LAYER_TENSORS}
+                   for l in range(s.n_layers)],
     }
     return m
+
+
+def with_norms(model: dict, s: ModelShape, norm_sigma: float, seed: int = SEED_WEIGHTS) -> dict:
+    """A shallow copy of ``model`` whose norm weights are replaced by the
+    ~N(1, norm_sigma) vectors ``make_model(..., norm_sigma)`` would make (the
+    large matrices are shared, not copied)."""
+    layers = []
+    for l, L in enumerate(model["layers"]):
+        d = dict(L)
+        d["attn_norm"] = make_norm(s, K_ATTN_NORM, l, norm_sigma, seed)
+        d["ffn_norm"] = make_norm(s, K_FFN_NORM, l, norm_sigma, seed)
+        layers.append(d)
+    out = dict(model)
+    out["layers"] = layers
+    out["final_norm"] = make_norm(s, K_FINAL_NORM, 0, norm_sigma, seed)
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -91,6 +91,25 @@ void syn_normal_bf16(uint16_t *out, uint64_t n, uint64_t key, double sigma,
   }
 }
 
+/*
+ * out[j] = bf16 of (mean + element (first + j)) of the normal stream `key`:
+ * the same Box-Muller value as syn_normal_bf16, offset by `mean` in float
+ * before the rounding (norm weights around 1).
+ */
+void syn_normal_bf16_mean(uint16_t *out, uint64_t n, uint64_t key, double mean,
+                          double sigma, uint64_t first) {
+  if (n == 0) return;
+  int64_t lo = (int64_t)(first / 2), hi = (int64_t)((first + n - 1) / 2);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = lo; i <= hi; ++i) {
+    float z0, z1;
+    syn_normal_pair(key, (uint64_t)i, sigma, &z0, &z1);
+    uint64_t e0 = 2 * (uint64_t)i, e1 = e0 + 1;
+    if (e0 >= first && e0 < first + n) out[e0 - first] = syn_f32_to_bf16_rne((float)mean + z0);
+    if (e1 >= first && e1 < first + n) out[e1 - first] = syn_f32_to_bf16_rne((float)mean + z1);
+  }
+}
+
 /* Same stream as syn_normal_bf16 but kept as float (used by the tests of the
  * generator itself). */
 void syn_normal_f32(float *out, uint64_t n, uint64_t key, double sigma) {

@@ -72,7 +72,7 @@ def test_unsupported_shape_rejected_before_any_device_call():
 def test_struct_layouts_match_headers():
     assert ctypes.sizeof(mk.mk_instr_desc) == 32
     assert ctypes.sizeof(mk.mk_config) == 56
-    assert ctypes.sizeof(mk.mk_plan_opts) == 48
+    assert ctypes.sizeof(mk.mk_plan_opts) == 56
 
 
 C_TYPES = {"int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "uint32_t": ctypes.c_uint32,

@@ -93,3 +93,48 @@ def test_reference_arm_line(capsys):
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"] > 0
     assert d["unit"] == "steps/s" and d["higher_is_better"] is True
+
+
+def _shard_rank(rank, world, port, times, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        b = _bench()
+        start, count = b.shard_sequences(16, world, rank)
+        # every rank reports its slice; gather them to check the cover
+        t = torch.tensor([start, count], dtype=torch.int64)
+        got = [torch.zeros(2, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(got, t)
+        ms = b.max_over_ranks(times[rank], dist, "cpu")
+        out[rank] = ([tuple(int(x) for x in g) for g in got], ms, b.sharded_rate(64, ms))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_batched_workload_splits_sequences_across_two_ranks():
+    """The 16-sequence workload is data parallel: two gloo ranks take
+    disjoint contiguous slices that cover the batch once, and the job's rate
+    counts whole-batch steps over the slowest rank's time."""
+    world, times = 2, [40.0, 32.0]
+    out = tmp.Manager().dict()
+    tmp.spawn(_shard_rank, args=(world, _free_port(), times, out), nprocs=world, join=True)
+    for r in range(world):
+        slices, ms, rate = out[r]
+        assert slices == [(0, 8), (8, 8)]
+        assert ms == 40.0
+        assert rate == pytest.approx(64 / 0.040)
+
+
+def test_shard_slices_cover_the_batch():
+    b = _bench()
+    for world in (1, 2, 3, 4, 5, 8, 16):
+        covered = []
+        sizes = []
+        for r in range(world):
+            start, count = b.shard_sequences(16, world, r)
+            covered += list(range(start, start + count))
+            sizes.append(count)
+        assert covered == list(range(16))
+        assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(SystemExit):
+        b.shard_sequences(16, 17, 0)

@@ -9,7 +9,7 @@ import torch
 import decode_megakernel_interpreter_b200 as mk
 from decode_megakernel_interpreter_b200 import harness
 import synth
-from gpu_common import ATOL, RTOL, HostSetup, compare_step, kv_row_mismatch
+from gpu_common import NORM_SIGMA, HostSetup, StepCheck, kv_row_mismatch
 
 pytestmark = pytest.mark.gpu
 
@@ -20,6 +20,12 @@ def b16():
     lengths = w.lengths()
     model = synth.make_model(w.shape)
     return w, lengths, model
+
+
+@pytest.fixture(scope="module")
+def b16_norms(b16):
+    w, lengths, model = b16
+    return w, lengths, synth.with_norms(model, w.shape, NORM_SIGMA)
 
 
 def _engine(w, lengths, model, plan_kw):
@@ -43,6 +49,7 @@ def _run(w, lengths, model, steps, plan_kw, check_oracle):
     logits = torch.empty(B, w.shape.vocab, dtype=torch.float32, device="cuda")
     nxt = torch.empty(B, dtype=torch.int32, device="cuda")
     out = []
+    chk = StepCheck()
     try:
         for step in range(steps):
             tokens.copy_(torch.tensor(tok, dtype=torch.int32))
@@ -55,19 +62,11 @@ def _run(w, lengths, model, steps, plan_kw, check_oracle):
             for b in range(B):
                 assert int(gn[b]) == int(np.argmax(gl[b])), f"seq {b}: next token must be the first maximal logit"
             if check_oracle:
-                kh = harness.kv_to_host(kc)
-                vh = harness.kv_to_host(vc)
                 for b in range(B):
-                    ol = hs.orc.decode_step(hs.k, hs.v, b, tok[b], pos[b])
-                    ok, near, mabs, _ = compare_step(gl[b], ol, int(gn[b]))
-                    assert ok, f"step {step} seq {b}: logits off by up to {mabs}"
-                    if near:
-                        tol = ATOL + RTOL * abs(float(ol.max()))
-                        assert ol[gn[b]] >= ol.max() - 2 * tol, f"step {step} seq {b}: greedy id outside the tie band"
-                    else:
-                        assert int(gn[b]) == int(np.argmax(ol)), f"step {step} seq {b}: greedy id differs"
-                    mk_k = kv_row_mismatch(kh[:, b, :, pos[b]], hs.k[:, b, :, pos[b]])
-                    mk_v = kv_row_mismatch(vh[:, b, :, pos[b]], hs.v[:, b, :, pos[b]])
+                    ol, bk, bv = hs.decode(b, tok[b], pos[b])
+                    chk.check(gl[b], ol, int(gn[b]), f"step {step} seq {b}")
+                    mk_k = kv_row_mismatch(harness.kv_row_to_host(kc, b, pos[b]), hs.k[:, b, :, pos[b]], bk)
+                    mk_v = kv_row_mismatch(harness.kv_row_to_host(vc, b, pos[b]), hs.v[:, b, :, pos[b]], bv)
                     assert not mk_k, f"step {step} seq {b}: K row: {mk_k}"
                     assert not mk_v, f"step {step} seq {b}: V row: {mk_v}"
             out.append(gl.copy())
@@ -75,12 +74,26 @@ def _run(w, lengths, model, steps, plan_kw, check_oracle):
             pos = [p + 1 for p in pos]
     finally:
         eng.close()
+    if check_oracle:
+        from test_gpu_parity import log_parity
+        log_parity("batched", chk.record(), plan_kw)
+        assert chk.id_mismatches <= chk.near_ties
     return out
 
 
 def test_llama1b_batch16_matches_oracle(b16):
+    """All 16 sequences free-running for 8 greedy steps."""
     w, lengths, model = b16
-    _run(w, lengths, model, 2, dict(), check_oracle=True)
+    _run(w, lengths, model, 8, dict(), check_oracle=True)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(tensor_qkv_o=True)], ids=["default", "tensor_qkv_o"])
+def test_llama1b_batch16_norm_weights(b16_norms, kw):
+    """Seeded norm weights on both batched builds: the tensor-core operands
+    carry x * gamma as bf16 hi/lo, so a wrong gamma there shows in every
+    sequence's logits."""
+    w, lengths, model = b16_norms
+    _run(w, lengths, model, 2, kw, check_oracle=True)
 
 
 def test_llama1b_batch16_modes_agree(b16):
@@ -101,6 +114,13 @@ def test_llama1b_batch16_tensor_qkv_o_matches_oracle(b16):
     got = _run(w, lengths, model, 2, dict(tensor_qkv_o=True, exec_mode="per_op"), check_oracle=False)
     for a, b in zip(ref, got):
         np.testing.assert_array_equal(a, b)
+
+
+def test_llama1b_batch16_cuda_cores_match_oracle(b16):
+    """use_tcgen05 = -1: the same batched build with every matrix instruction
+    on CUDA cores (the comparison the tensor-core path is adopted against)."""
+    w, lengths, model = b16
+    _run(w, lengths, model, 2, dict(use_tcgen05=-1), check_oracle=True)
 
 
 def test_batched_plan_needs_a_batched_build():

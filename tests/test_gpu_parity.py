@@ -2,10 +2,14 @@
 same seeded inputs.
 
 Per step: every logit within |gpu - oracle| <= 2e-2 + 1e-2 |oracle| (the
-oracle is fed the GPU's own input token, so the two never drift apart), the
-greedy id identical unless the oracle's top-2 margin is inside the tolerance,
-next_tokens_out == argmax(logits_out) exactly, and the K/V row written at the
-step's position within one bf16 ulp of the oracle's.
+oracle is fed the GPU's own input token, so the two never drift apart); the
+greedy id identical to the oracle's unless the oracle's top-2 margin is within
+twice the step's measured logit error (then the GPU's id must be one of the
+ids that error allows); next_tokens_out == argmax(logits_out) exactly; and the
+K/V row written at the step's position within one bf16 ulp plus the fp32
+dot-product error bound of the oracle's.  Several tests use seeded norm
+weights ~N(1, 0.3) (distinct per norm and layer) so that the kernels' use of
+them is checked too; the full-size configurations run free for tens of steps.
 """
 import json
 import os
@@ -17,15 +21,24 @@ import torch
 import decode_megakernel_interpreter_b200 as mk
 from decode_megakernel_interpreter_b200 import harness
 import synth
-from gpu_common import ATOL, RTOL, HostSetup, compare_step, kv_row_mismatch
+from gpu_common import NORM_SIGMA, HostSetup, StepCheck, kv_row_mismatch
 
 pytestmark = pytest.mark.gpu
 
 
+def log_parity(name: str, rec: dict, plan_kw: dict):
+    log = os.environ.get("MK_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", name), **rec,
+                                "plan": {k: str(v) for k, v in plan_kw.items()}}) + "\n")
+
+
 def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan_kw: dict, b=0,
-               check_kv=True, engine_out=None):
+               check_kv=True, dev=None):
     s = hs.shape
-    dev = harness.upload_model(hs.model, s.tied)
+    if dev is None:
+        dev = harness.upload_model(hs.model, s.tied)
     kc, vc = harness.upload_kv(hs.k, hs.v)
     eng = harness.make_engine(s, dev, kc, vc, hs.batch, hs.max_seq)
     eng.plan(**plan_kw)
@@ -34,8 +47,8 @@ def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan
     logits = torch.empty(hs.batch, s.vocab, dtype=torch.float32, device="cuda")
     nxt = torch.empty(hs.batch, dtype=torch.int32, device="cuda")
     tok, p = first_token, first_pos
-    stats = {"near_ties": 0, "max_abs": 0.0, "max_rel": 0.0, "tokens": [], "logits": [],
-             "kernel_variant": int(eng.info.kernel_variant)}
+    chk = StepCheck()
+    stats = {"tokens": [], "logits": [], "kernel_variant": int(eng.info.kernel_variant)}
     try:
         for step in range(steps):
             tokens.fill_(tok)
@@ -46,24 +59,14 @@ def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan
             gl = logits[b].cpu().numpy()
             gn = int(nxt[b].item())
             assert gn == int(np.argmax(gl)), "next token must be the first maximal logit"
-            ol = hs.orc.decode_step(hs.k, hs.v, b, tok, p)
-            ok, near, mabs, mrel = compare_step(gl, ol, gn)
-            stats["max_abs"] = max(stats["max_abs"], mabs)
-            stats["max_rel"] = max(stats["max_rel"], mrel)
-            assert ok, f"step {step}: logits off by up to {mabs}"
-            if near:
-                # several ids are correct within the tolerance: the GPU's pick
-                # must be one of them
-                stats["near_ties"] += 1
-                tol = ATOL + RTOL * abs(float(ol.max()))
-                assert ol[gn] >= ol.max() - 2 * tol, f"step {step}: greedy id outside the tie band"
-            else:
-                assert gn == int(np.argmax(ol)), f"step {step}: greedy id differs"
             if check_kv:
-                gk = harness.kv_to_host(kc)[:, b, :, p]
-                gv = harness.kv_to_host(vc)[:, b, :, p]
-                mk_k = kv_row_mismatch(gk, hs.k[:, b, :, p])
-                mk_v = kv_row_mismatch(gv, hs.v[:, b, :, p])
+                ol, bk, bv = hs.decode(b, tok, p)
+            else:
+                ol = hs.orc.decode_step(hs.k, hs.v, b, tok, p)
+            chk.check(gl, ol, gn, f"step {step}")
+            if check_kv:
+                mk_k = kv_row_mismatch(harness.kv_row_to_host(kc, b, p), hs.k[:, b, :, p], bk)
+                mk_v = kv_row_mismatch(harness.kv_row_to_host(vc, b, p), hs.v[:, b, :, p], bv)
                 assert not mk_k, f"step {step}: K row: {mk_k}"
                 assert not mk_v, f"step {step}: V row: {mk_v}"
             stats["tokens"].append(gn)
@@ -71,12 +74,9 @@ def run_parity(hs: HostSetup, first_token: int, first_pos: int, steps: int, plan
             tok, p = gn, p + 1
     finally:
         eng.close()
-    log = os.environ.get("MK_PARITY_LOG")
-    if log:
-        with open(log, "a") as f:
-            f.write(json.dumps({"test": os.environ.get("PYTEST_CURRENT_TEST", "?"), "steps": steps,
-                                "near_ties": stats["near_ties"], "max_abs": stats["max_abs"],
-                                "max_rel": stats["max_rel"], "plan": {k: str(v) for k, v in plan_kw.items()}}) + "\n")
+    stats.update(chk.record())
+    log_parity("run_parity", chk.record(), plan_kw)
+    assert chk.id_mismatches <= chk.near_ties
     return stats
 
 
@@ -124,6 +124,17 @@ def test_schedule_independence_bitwise(tiny_model):
             np.testing.assert_array_equal(a, b)
 
 
+@pytest.mark.parametrize("kw", [dict(), dict(exec_mode="per_op"), dict(exec_mode="megakernel_generic")],
+                         ids=["mk", "per_op", "mk_generic"])
+def test_tiny_norm_weights(tiny_model, kw):
+    """Seeded norm weights ~N(1, 0.3), distinct per norm and layer: a kernel
+    that ignored them, swapped the attention and FFN norms, skipped the final
+    norm or indexed gamma in the wrong layout would fail the logits."""
+    model = synth.with_norms(tiny_model, synth.TINY, NORM_SIGMA)
+    hs, tok, pos = tiny_setup(model)
+    run_parity(hs, tok, pos, 16, kw)
+
+
 def test_tiny_from_empty_cache(tiny_model):
     """Position 0: attention over the single current key."""
     hs = HostSetup(synth.TINY, 1, 32, tiny_model)
@@ -143,16 +154,18 @@ def test_ragged_vocab_and_untied_head():
     run_parity(hs, 999, 30, 6, dict())
 
 
-def test_mha_and_head_dim_128():
+@pytest.mark.parametrize("norm_sigma", [0.0, NORM_SIGMA], ids=["unit_norms", "seeded_norms"])
+def test_mha_and_head_dim_128(norm_sigma):
     s = synth.ModelShape(2, 512, 4, 4, 128, 2048, 2048, 1e-5, 5e5, True)
-    hs = HostSetup(s, 1, 200)
+    hs = HostSetup(s, 1, 200, synth.make_model(s, norm_sigma=norm_sigma))
     hs.fill_prefix([150])
     run_parity(hs, 5, 150, 4, dict(kv_splits=6))
 
 
-def test_gqa_group_of_eight():
+@pytest.mark.parametrize("norm_sigma", [0.0, NORM_SIGMA], ids=["unit_norms", "seeded_norms"])
+def test_gqa_group_of_eight(norm_sigma):
     s = synth.ModelShape(1, 1024, 16, 2, 64, 4096, 3000, 1e-5, 1e4, True)
-    hs = HostSetup(s, 1, 300)
+    hs = HostSetup(s, 1, 300, synth.make_model(s, norm_sigma=norm_sigma))
     hs.fill_prefix([257])
     run_parity(hs, 2999, 257, 3, dict())
 
@@ -175,12 +188,13 @@ def test_next_tokens_may_alias_tokens(tiny_model):
     assert eng.status() == mk.MK_OK
     eng.close()
     # the oracle, fed the GPU's own inputs, must agree with every pick
+    # (no logits of these steps are kept: an id the oracle ranks below its
+    # maximum by more than the logit tolerance is wrong)
     inp = tok
     for i in range(6):
         ol = hs.orc.decode_step(hs.k, hs.v, 0, inp, pos + i)
         out = int(got[i].item())
-        tol = ATOL + RTOL * abs(float(ol.max()))
-        assert ol[out] >= ol.max() - 2 * tol
+        assert ol[out] >= ol.max() - 2 * (2e-2 + 1e-2 * abs(float(ol.max())))
         inp = out
 
 
@@ -234,18 +248,28 @@ def llama1b_model():
 
 
 def test_llama1b_1024_context(llama1b_model):
+    """The headline configuration, free-running for 32 greedy steps."""
     w = synth.WORKLOADS["llama1b"]
-    hs = HostSetup(w.shape, 1, w.context + 8, llama1b_model)
+    hs = HostSetup(w.shape, 1, w.context + 40, llama1b_model)
     hs.fill_prefix(w.lengths())
-    st = run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 3, dict())
-    print("llama1b max_abs", st["max_abs"], "max_rel", st["max_rel"])
+    st = run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 32, dict())
+    print("llama1b", {k: st[k] for k in ("max_abs", "max_rel", "near_ties", "id_mismatches")})
+
+
+def test_llama1b_1024_context_norm_weights(llama1b_model):
+    w = synth.WORKLOADS["llama1b"]
+    model = synth.with_norms(llama1b_model, w.shape, NORM_SIGMA)
+    hs = HostSetup(w.shape, 1, w.context + 8, model)
+    hs.fill_prefix(w.lengths())
+    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 4, dict())
 
 
 def test_llama1b_8k_context(llama1b_model):
+    """Context 8192, free-running for 16 greedy steps."""
     w = synth.WORKLOADS["llama1b_8k"]
-    hs = HostSetup(w.shape, 1, w.context + 4, llama1b_model)
+    hs = HostSetup(w.shape, 1, w.context + 20, llama1b_model)
     hs.fill_prefix(w.lengths())
-    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 2, dict())
+    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 16, dict())
 
 
 def test_llama1b_per_op_and_generic_match_megakernel(llama1b_model):
@@ -264,7 +288,16 @@ def test_llama1b_per_op_and_generic_match_megakernel(llama1b_model):
 
 
 def test_llama8b_2048_context():
+    """The 8B shape (untied head, head_dim 128): 4 free-running greedy steps
+    with the configuration's unit norm weights, then 2 with seeded ones (same
+    matrices on the device)."""
     w = synth.WORKLOADS["llama8b"]
-    hs = HostSetup(w.shape, 1, w.context + 2)
+    model = synth.make_model(w.shape)
+    dev = harness.upload_model(model, w.shape.tied)
+    hs = HostSetup(w.shape, 1, w.context + 8, model)
     hs.fill_prefix(w.lengths())
-    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 1, dict())
+    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 4, dict(), dev=dev)
+    gm = synth.with_norms(model, w.shape, NORM_SIGMA)
+    hs = HostSetup(w.shape, 1, w.context + 8, gm)
+    hs.fill_prefix(w.lengths())
+    run_parity(hs, int(synth.first_tokens(w)[0]), w.context, 2, dict(), dev=harness.replace_norms(dev, gm))

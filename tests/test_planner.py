@@ -196,6 +196,33 @@ def test_batched_plan_tensor_qkv_o_tiles():
     assert err == ""
 
 
+def test_use_tcgen05_option():
+    """use_tcgen05: automatic (tensor-core tiles at batch > 1), forced off
+    (CUDA-core pages at any batch), forced on (refused at batch 1, where every
+    product is a matrix-vector product); the tensor-core QKV / O needs it on."""
+    cfg = cfg_for("llama1b_b16", max_batch=16)
+    F = cfg.ffn
+    auto, *_ = mk.mk_host_plan(cfg, mk.plan_opts(batch=16), 148)
+    on, *_ = mk.mk_host_plan(cfg, mk.plan_opts(batch=16, use_tcgen05=1), 148)
+    off, *_ = mk.mk_host_plan(cfg, mk.plan_opts(batch=16, use_tcgen05=-1), 148)
+    gu_units = lambda ins: sum(i.b for i in ins if i.op == OP["gateup"] and i.layer == 0)
+    assert gu_units(auto) == gu_units(on) == F // 64          # 128-row tiles of 64 gate + 64 up rows
+    rows_per_page = 16384 // (2 * cfg.hidden)
+    assert gu_units(off) == F // (rows_per_page // 2)           # one page of R/2 gate + R/2 up rows each
+    assert mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=16, use_tcgen05=-1), 148, steps=1, seed=3,
+                                    timeout_ms=20000) == ""
+    cfg1 = cfg_for("llama1b")
+    for bad in (mk.plan_opts(batch=1, use_tcgen05=1), mk.plan_opts(batch=16, use_tcgen05=2),
+                mk.plan_opts(batch=16, use_tcgen05=-1, tensor_qkv_o=True)):
+        with pytest.raises(mk.MkError) as e:
+            mk.mk_host_plan(cfg1 if bad.batch == 1 else cfg, bad, 148)
+        assert e.value.code == mk.MK_ERR_INVALID_ARG
+    # off at batch 1 is the batch-1 default
+    a, *_ = mk.mk_host_plan(cfg1, mk.plan_opts(batch=1), 148)
+    b, *_ = mk.mk_host_plan(cfg1, mk.plan_opts(batch=1, use_tcgen05=-1), 148)
+    assert [bytes(x) for x in a] == [bytes(x) for x in b]
+
+
 @pytest.mark.parametrize("tqo", [False, True])
 @pytest.mark.parametrize("sched,num_ctas", [("static", 37), ("dynamic", 148), ("dynamic", 16)])
 def test_batched_plan_other_grids(tqo, sched, num_ctas):

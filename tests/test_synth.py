@@ -59,3 +59,28 @@ def test_kv_prefix_fill():
     assert np.all(k[:, 0, :, 5:] == 0) and np.any(k[:, 0, :, :5] != 0)
     assert np.all(v[:, 1, :, 9:] == 0) and np.any(v[:, 1, :, :9] != 0)
     assert not np.array_equal(k[:, 1, :, :5], v[:, 1, :, :5])
+
+
+def test_norm_weights_unit_or_seeded():
+    s = synth.TINY
+    ones = synth.bf16_bits_to_f32(synth.make_norm(s, synth.K_ATTN_NORM, 0))
+    assert np.all(ones == 1.0)
+    g0 = synth.bf16_bits_to_f32(synth.make_norm(s, synth.K_ATTN_NORM, 0, 0.3)).astype(np.float64)
+    g1 = synth.bf16_bits_to_f32(synth.make_norm(s, synth.K_ATTN_NORM, 1, 0.3)).astype(np.float64)
+    gf = synth.bf16_bits_to_f32(synth.make_norm(s, synth.K_FFN_NORM, 0, 0.3)).astype(np.float64)
+    # distinct vectors per norm and layer, around 1 with the asked spread
+    assert not np.array_equal(g0, g1) and not np.array_equal(g0, gf)
+    big = synth.bf16_bits_to_f32(synth.normal_bf16_mean((200_000,), synth.key(0, synth.K_FFN_NORM, 3), 1.0, 0.3))
+    assert abs(big.astype(np.float64).mean() - 1.0) < 0.005 and abs(big.astype(np.float64).std() - 0.3) < 0.005
+    # the offset stream is the plain stream plus the mean, rounded once
+    k = synth.key(5, 9)
+    plain = synth.normal_f32(1000, k, 0.3)
+    shifted = synth.bf16_bits_to_f32(synth.normal_bf16_mean((1000,), k, 1.0, 0.3)).astype(np.float64)
+    ref = (np.float32(1.0) + plain).astype(np.float64)
+    assert np.all(np.abs(shifted - ref) <= np.abs(ref) * 2.0 ** -8)
+    m = synth.make_model(s, norm_sigma=0.3)
+    m1 = synth.with_norms(synth.make_model(s), s, 0.3)
+    for name in ("attn_norm", "ffn_norm"):
+        np.testing.assert_array_equal(m["layers"][1][name], m1["layers"][1][name])
+    np.testing.assert_array_equal(m["final_norm"], m1["final_norm"])
+    assert np.any(synth.bf16_bits_to_f32(m["final_norm"]) != 1.0)

@@ -76,6 +76,17 @@ def test_noalloc_matches_handle_path_on_two_calls(name, context):
         p = context + call
         np.testing.assert_array_equal(harness.kv_to_host(kc_b)[:, 0, :, p], harness.kv_to_host(kc_a)[:, 0, :, p])
         np.testing.assert_array_equal(harness.kv_to_host(vc_b)[:, 0, :, p], harness.kv_to_host(vc_a)[:, 0, :, p])
+    # a further call with the same arguments takes no device memory: free
+    # memory is unchanged across it (torch's caching allocator is not involved
+    # either, since the call goes straight through the C ABI)
+    pos = torch.tensor([context + 2], dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    rc = mk.mk_decode_step_noalloc(cfg, w, kv, t_b.data_ptr(), pos.data_ptr(), logits_b.data_ptr(), t_b.data_ptr(),
+                                   stream.cuda_stream)
+    assert rc == mk.MK_OK
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
     eng.close()
 
 
