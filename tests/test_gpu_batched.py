@@ -28,8 +28,9 @@ def b16_norms(b16):
     return w, lengths, synth.with_norms(model, w.shape, NORM_SIGMA)
 
 
-def _engine(w, lengths, model, plan_kw):
-    hs = HostSetup(w.shape, w.batch, int(lengths.max()) + 4, model)
+def _engine(w, lengths, model, plan_kw, steps):
+    # room for every step's K/V row of the longest sequence
+    hs = HostSetup(w.shape, w.batch, int(lengths.max()) + steps + 2, model)
     hs.fill_prefix(lengths)
     dev = harness.upload_model(hs.model, w.shape.tied)
     kc, vc = harness.upload_kv(hs.k, hs.v)
@@ -39,7 +40,7 @@ def _engine(w, lengths, model, plan_kw):
 
 
 def _run(w, lengths, model, steps, plan_kw, check_oracle):
-    hs, eng, kc, vc = _engine(w, lengths, model, plan_kw)
+    hs, eng, kc, vc = _engine(w, lengths, model, plan_kw, steps)
     B = w.batch
     assert eng.info.kernel_variant == 1  # batched plans run a specialised build
     tok = [int(t) for t in synth.first_tokens(w)]
