@@ -83,6 +83,18 @@ class mk_instr_desc(ctypes.Structure):
                 ("sig_n", ctypes.c_uint16), ("seq", ctypes.c_uint16)]
 
 
+class mk_cost_params(ctypes.Structure):
+    _fields_ = [("sm_gbs", ctypes.c_double), ("ring_pages", ctypes.c_int32), ("exchange_us", ctypes.c_double),
+                ("page_us", ctypes.c_double), ("attn_page_us", ctypes.c_double), ("attn_fixed_us", ctypes.c_double),
+                ("merge_us", ctypes.c_double), ("instr_us", ctypes.c_double), ("launch_us", ctypes.c_double),
+                ("tc_page_us", ctypes.c_double), ("cc_page_us_seq", ctypes.c_double), ("conv_ctas", ctypes.c_int32)]
+
+
+class mk_cost_estimate(ctypes.Structure):
+    _fields_ = [("step_us", ctypes.c_double), ("per_op_us", ctypes.c_double), ("hbm_floor_us", ctypes.c_double),
+                ("savings_us", ctypes.c_double), ("stage_us", ctypes.c_double * 7)]
+
+
 _lib = None
 
 
@@ -119,6 +131,11 @@ def load(path: str = LIB_PATH):
                                P(mk_plan_info), ctypes.c_char_p, sz]
     L.mk_decode_step_noalloc.restype = i32
     L.mk_decode_step_noalloc.argtypes = [P(mk_config), P(mk_weights), P(mk_kv_cache), vp, vp, vp, vp, vp]
+    L.mk_cost_params_default.restype = None
+    L.mk_cost_params_default.argtypes = [P(mk_cost_params)]
+    L.mk_host_plan_estimate.restype = i32
+    L.mk_host_plan_estimate.argtypes = [P(mk_config), P(mk_plan_opts), i32, i32, P(mk_cost_params),
+                                        P(mk_cost_estimate), ctypes.c_char_p, sz]
     L.mk_host_plan_simulate.restype = i32
     L.mk_host_plan_simulate.argtypes = [P(mk_config), P(mk_plan_opts), i32, i32, u64, i32, ctypes.c_char_p, sz]
     _lib = L
@@ -219,6 +236,25 @@ def mk_host_plan_simulate(cfg: mk_config, opts: mk_plan_opts | None, num_ctas: i
     rc = load().mk_host_plan_simulate(ctypes.byref(cfg), ctypes.byref(opts) if opts is not None else None, num_ctas,
                                       steps, seed, timeout_ms, err, 1024)
     return "" if rc == MK_OK else (err.value.decode() or mk_status_string(rc))
+
+
+def mk_cost_params_default() -> mk_cost_params:
+    q = mk_cost_params()
+    load().mk_cost_params_default(ctypes.byref(q))
+    return q
+
+
+def mk_host_plan_estimate(cfg: mk_config, opts: mk_plan_opts | None, num_ctas: int, context: int,
+                          params: mk_cost_params | None = None) -> mk_cost_estimate:
+    """The cost model's estimate of a plan (see mk_host.h)."""
+    out = mk_cost_estimate()
+    err = ctypes.create_string_buffer(512)
+    rc = load().mk_host_plan_estimate(ctypes.byref(cfg), ctypes.byref(opts) if opts is not None else None, num_ctas,
+                                      context, ctypes.byref(params) if params is not None else None,
+                                      ctypes.byref(out), err, 512)
+    if rc != MK_OK:
+        raise MkError(rc, "mk_host_plan_estimate: " + err.value.decode())
+    return out
 
 
 # ---------------------------------------------------------------- torch wrapper

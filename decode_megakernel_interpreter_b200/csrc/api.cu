@@ -362,17 +362,7 @@ int check_cfg(const mk_config *c, std::string *why) {
 }
 
 size_t act_floats_for(const mk_config &c, const Plan &p, int nb) {
-  const int G = c.n_q_heads / c.n_kv_heads;
-  // input vector per sequence (batch 1: + the O projection's residual rows
-  // after it)
-  size_t vec = nb == 1 ? (size_t)std::max({c.hidden, c.n_q_heads * c.head_dim + c.hidden, p.KCd})
-                       : (size_t)nb * std::max({c.hidden, c.n_q_heads * c.head_dim, p.KCd});
-  // warps' partials + the current K/V rows (bf16) + the warps' merge weights
-  size_t attn = (size_t)kComputeWarps * G * (c.head_dim + 2) + (size_t)c.head_dim + (size_t)G * (kComputeWarps + 2);
-  size_t f = std::max(vec, attn);
-  // batched builds: the tensor-core epilogue exchange follows the staged vectors
-  if (nb > 1) f += kTcXchFloats;
-  return (f + 31) / 32 * 32;
+  return staging_floats(c.hidden, c.n_q_heads * c.head_dim, p.KCd, c.n_q_heads / c.n_kv_heads, c.head_dim, nb);
 }
 
 }  // namespace
@@ -506,15 +496,12 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   // batched plans run the kernel instantiated for up to kMaxBatch sequences
   const int nb = o.batch > 1 ? kMaxBatch : 1;
   const size_t act_floats = act_floats_for(h->cfg, p, nb);
-  const int fixed = shared_bytes_fixed(0, act_floats);
-  int num_pages = (h->smem_optin - fixed) / (kPageBytes + 16);
   // a multiple of the loader count (page g and the next user of its slot,
   // g + num_pages, then belong to the same loader) with 2 * num_pages a
   // multiple of the compute-warp count (page g - 2 * num_pages belongs to the
   // same warp as page g): every mbarrier parity test is then unambiguous
-  num_pages = std::min(num_pages, 16) / kLoaders * kLoaders;
-  while (num_pages > 0 && (2 * num_pages) % kComputeWarps) num_pages -= kLoaders;
-  if (num_pages < 2 * kLoaders) return MK_ERR_UNSUPPORTED_SHAPE;
+  const int num_pages = ring_pages(h->smem_optin, act_floats);
+  if (num_pages == 0) return MK_ERR_UNSUPPORTED_SHAPE;
   const int smem = shared_bytes_fixed(num_pages, act_floats);
   // the interpreter build: specialised for this shape unless asked otherwise
   KParams sel;
@@ -917,5 +904,76 @@ extern "C" int mk_host_plan_simulate(const mk_config *cfg, const mk_plan_opts *o
     set_err(err, err_len, e);
     return MK_ERR_INVALID_ARG;
   }
+  return MK_OK;
+}
+
+// ====================================================================== cost model
+
+static CostParams cost_params_from(const mk_cost_params *q) {
+  CostParams c;
+  if (!q) return c;
+  c.sm_gbs = q->sm_gbs;
+  c.ring_pages = q->ring_pages;
+  c.exchange_us = q->exchange_us;
+  c.page_us = q->page_us;
+  c.attn_page_us = q->attn_page_us;
+  c.attn_fixed_us = q->attn_fixed_us;
+  c.merge_us = q->merge_us;
+  c.instr_us = q->instr_us;
+  c.launch_us = q->launch_us;
+  c.tc_page_us = q->tc_page_us;
+  c.cc_page_us_seq = q->cc_page_us_seq;
+  c.conv_ctas = q->conv_ctas;
+  return c;
+}
+
+extern "C" void mk_cost_params_default(mk_cost_params *q) {
+  if (!q) return;
+  const CostParams c;
+  q->sm_gbs = c.sm_gbs;
+  q->ring_pages = c.ring_pages;
+  q->exchange_us = c.exchange_us;
+  q->page_us = c.page_us;
+  q->attn_page_us = c.attn_page_us;
+  q->attn_fixed_us = c.attn_fixed_us;
+  q->merge_us = c.merge_us;
+  q->instr_us = c.instr_us;
+  q->launch_us = c.launch_us;
+  q->tc_page_us = c.tc_page_us;
+  q->cc_page_us_seq = c.cc_page_us_seq;
+  q->conv_ctas = c.conv_ctas;
+}
+
+extern "C" int mk_host_plan_estimate(const mk_config *cfg, const mk_plan_opts *opts, int32_t num_ctas,
+                                     int32_t context, const mk_cost_params *params, mk_cost_estimate *out,
+                                     char *err, size_t err_len) {
+  std::string why;
+  int rc = check_cfg(cfg, &why);
+  if (rc) {
+    set_err(err, err_len, why);
+    return rc;
+  }
+  if (num_ctas < 1 || context < 0 || context >= cfg->max_seq || !out) return MK_ERR_INVALID_ARG;
+  mk_plan_opts o = opts ? *opts : default_opts(*cfg);
+  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
+  PlanRequest req = make_request(*cfg, o, num_ctas);
+  Plan p;
+  std::string e = build_plan(req, &p);
+  if (e.empty()) e = validate_plan(req, p);
+  if (!e.empty()) {
+    set_err(err, err_len, e);
+    return MK_ERR_UNSUPPORTED_SHAPE;
+  }
+  CostEstimate est;
+  e = estimate_plan(req, p, cost_params_from(params), context, &est);
+  if (!e.empty()) {
+    set_err(err, err_len, e);
+    return MK_ERR_INVALID_ARG;
+  }
+  out->step_us = est.step_us;
+  out->per_op_us = est.per_op_us;
+  out->hbm_floor_us = est.hbm_floor_us;
+  out->savings_us = est.per_op_us - est.step_us;
+  for (int i = 0; i < 7; ++i) out->stage_us[i] = est.stage_us[i];
   return MK_OK;
 }

@@ -1,5 +1,7 @@
 // The decode interpreter's host entry: kernel selection and launch.  The
 // device code is in interp_body.cuh.
+#include <algorithm>
+
 #include "interp_body.cuh"
 #include "interp_launch.h"
 
@@ -8,6 +10,26 @@ namespace mk {
 int shared_bytes_fixed(int num_pages, size_t act_floats) {
   return (int)((size_t)num_pages * kPageBytes + act_floats * 4 + (size_t)num_pages * 16 + sizeof(Shared) +
                34 * sizeof(int) + 64);
+}
+
+size_t staging_floats(int H, int qdim, int KCd, int G, int d, int nb) {
+  // input vector per sequence (batch 1: also the O projection's residual rows
+  // after the vector, or after the split-page partial table)
+  size_t vec = nb == 1 ? std::max({(size_t)H, (size_t)qdim + H, (size_t)KCd, (size_t)kSplitRedFloats + H})
+                       : (size_t)nb * std::max({H, qdim, KCd});
+  // warps' partials + the current K/V rows (bf16) + the warps' merge weights
+  size_t attn = (size_t)kComputeWarps * G * (d + 2) + (size_t)d + (size_t)G * (kComputeWarps + 2);
+  size_t f = std::max(vec, attn);
+  // batched builds: the tensor-core epilogue exchange follows the staged vectors
+  if (nb > 1) f += kTcXchFloats;
+  return (f + 31) / 32 * 32;
+}
+
+int ring_pages(int smem_optin, size_t act_floats) {
+  int n = (smem_optin - shared_bytes_fixed(0, act_floats)) / (kPageBytes + 16);
+  n = std::min(n, 16) / kLoaders * kLoaders;
+  while (n > 0 && (2 * n) % kComputeWarps) n -= kLoaders;
+  return n < 2 * kLoaders ? 0 : n;
 }
 
 namespace {

@@ -68,6 +68,20 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// packed fp32 pair FMA (two lanes of fp32 in one 64-bit register pair)
+__device__ __forceinline__ unsigned long long f2pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void ffma2(unsigned long long &acc, unsigned long long a, unsigned long long b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ float f2sum(unsigned long long v) {
+  float lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+  return lo + hi;
+}
 // Bring [src, src + bytes) into L2 (no completion to wait for).
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
@@ -200,11 +214,6 @@ __device__ __forceinline__ uint4 ld_tf4(const float *a) {
   asm volatile("ld.relaxed.gpu.global.v4.b32 {%0, %1, %2, %3}, [%4];"
                : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
                : "l"(a));
-  return u;
-}
-__device__ __forceinline__ uint2 ld_tf2(const float *a) {
-  uint2 u;
-  asm volatile("ld.relaxed.gpu.global.v2.b32 {%0, %1}, [%2];" : "=r"(u.x), "=r"(u.y) : "l"(a));
   return u;
 }
 // Named barrier over the 256 compute threads, returning the OR of `pred`
@@ -766,7 +775,23 @@ __device__ __forceinline__ bool ring_wait(const KParams &p, const Ring &r, uint3
     }
   }
   if (px::mbar_test(&r.full[slot], ph)) return true;  // fast path: already landed
-  atomicAdd(&r.sh->stat_cwait, 1);
+  if ((threadIdx.x & 31) == 0) atomicAdd(&r.sh->stat_cwait, 1);
+  if (px::ld_volatile(&r.sh->abort)) return false;
+  if (!wait_bar(p, r.sh, &r.full[slot], ph, 0)) {
+    r.sh->abort = 1;
+    return false;
+  }
+  return true;
+}
+// Split pages (every compute warp consumes every page of the instruction, in
+// order): when a warp waits for page g, page g - np has landed (this warp
+// consumed it, or -- in an earlier instruction -- its owner did before the
+// instruction's closing barrier), and page g + np cannot have been issued
+// (that needs this warp's release of page g).  So the full barrier's parity
+// test alone is unambiguous; slot and phase are tracked by the caller.
+__device__ __forceinline__ bool ring_wait_full(const KParams &p, const Ring &r, uint32_t slot, uint32_t ph) {
+  if (px::mbar_test(&r.full[slot], ph)) return true;
+  if ((threadIdx.x & 31) == 0) atomicAdd(&r.sh->stat_cwait, 1);
   if (px::ld_volatile(&r.sh->abort)) return false;
   if (!wait_bar(p, r.sh, &r.full[slot], ph, 0)) {
     r.sh->abort = 1;
@@ -1142,142 +1167,562 @@ __device__ __forceinline__ void matvec_pages(CCtx &c, const Instr &I, Epi epi) {
   c.g = g0 + (uint32_t)np;
 }
 
-template <int NB, int R>
-__device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
-  const KParams &p = c.p;
-  const int l = I.layer;
-  const int half = R / 2, pph = p.d / R, hd = p.d / 2;
-  const int pos0 = read_pos(c.sh, 0);
-  float inv[NB];
-  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].attn_norm, false, inv);
-  const int nq = p.nq, nkv = p.nkv, d = p.d, lane = c.lane, Bn = p.B, kvdim = p.kvdim;
-  const uint32_t tag = c.epoch;
-  float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
-  float *const kvc = p.kvcur + (size_t)l * Bn * 2 * kvdim;
-  uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
-  const long long kv_bs = p.kv_bs, kv_hs = p.kv_hs;
-  const int qdim = p.qdim;
-  const float2 *rope_s = c.sh->rope;
-  const float2 *rope_g = p.rope;
-  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    const int head = j / pph, jj = j % pph;
-    if (lane >= half) return;
-    const int i = jj * half + lane;  // rotation pair index inside the head
+// ---------------------------------------------------------------- split pages
+// Batch-1 matrix-vector instructions whose page rows are 2048 or 4096 columns
+// long (R = 4 or 2 rows per page: hidden, q_dim and the down-projection K
+// piece of 2048 or more) are computed with every page SPLIT across the eight
+// compute warps: warp w takes columns [w * KC / 8, (w + 1) * KC / 8) of all R
+// rows, lane l the 16-byte chunks w * 32 * CPL + 32 * j + l (j < CPL).  So
+//  - a page is finished ~8x sooner after it lands than when one warp owns it
+//    (the last page of an instruction no longer costs one warp ~1 us: the
+//    instruction's tail, which every dependent instruction waits for, shrinks);
+//  - the thread's slice of the input vector is the same for every page: it is
+//    loaded once into registers (no shared-memory staging of the vector);
+//  - each row's sum is the eight warp partials added in a fixed order, so the
+//    result stays independent of the plan.
+// Row partials go to a double-buffered shared-memory table; after every T
+// pages one compute barrier, then the epilogue of those pages' rows.
+template <int R>
+struct Split {
+  static constexpr int KC = kPageElems / R;  // columns per page row
+  static constexpr int CPL = KC / 2048;      // 16-byte chunks per lane and row
+  static constexpr int NX = 8 * CPL;         // input elements per thread
+  static constexpr int T = 16;               // pages per epilogue batch
+  static constexpr int LOG2R = R == 4 ? 2 : 1;
+  static_assert(R == 2 || R == 4, "split pages: 2 or 4 rows per page");
+};
+// Page scheme of a batch-1 matrix instruction: 1 = split pages (every warp a
+// column slice of every page) in builds that ask for it (SPL: the Llama-8B
+// shape, where it measured 3481 against 3942 us per step); 0 = one warp per
+// page otherwise (the Llama-1B shape, where split pages measured 716 and two
+// warps per page 745 against 673 us per step: with 4-row pages the per-page
+// reduction and synchronisation cost more than the shorter tails save).
+template <int NB, int R, bool SPL>
+struct Scheme {
+  static constexpr int v = NB == 1 && SPL && (R == 2 || R == 4) ? 1 : 0;
+};
+// the partial table occupies the first kSplitRedFloats floats of the staging
+// region (two buffers of T * R * 8 floats = 512 floats each at most); the O
+// projection's residual rows follow it
+static_assert(2 * Split<4>::T * 4 * 8 <= kSplitRedFloats, "partial table");
+
+template <int R>
+__device__ __forceinline__ int split_chunk(int cw, int lane, int j) {
+  return cw * 32 * Split<R>::CPL + 32 * j + lane;
+}
+
+// Sum N per-lane values over the warp's 32 lanes; lane l ends with the total
+// of value l / (32 / N) (halving exchanges, then a butterfly).
+template <int N>
+__device__ __forceinline__ float warp_sum_rows(float (&v)[N], int lane) {
+  constexpr int LOG2N = N >= 32 ? 5 : N >= 16 ? 4 : N >= 8 ? 3 : N >= 4 ? 2 : N >= 2 ? 1 : 0;
+  static_assert((1 << LOG2N) == N && N <= 32, "power of two, at most 32 values");
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      if (NB > 1 && b >= Bn) break;
-      float u = pick<R>(acc[b], lane) * inv[b], w = pick<R>(acc[b], lane + half) * inv[b];
-      const int pos = NB == 1 ? pos0 : read_pos(c.sh, b);
-      if (head < nq + nkv) {
-        const float2 cs = NB == 1 ? rope_s[i] : __ldg(rope_g + (size_t)pos * hd + i);
-        const float u2 = u * cs.x - w * cs.y, w2 = u * cs.y + w * cs.x;
-        u = u2;
-        w = w2;
+  for (int st = 0; st < LOG2N; ++st) {
+    const int n = N >> st, off = 16 >> st;
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      if (i < n / 2) {
+        const float send = up ? v[i] : v[i + n / 2];
+        const float keep = up ? v[i + n / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
       }
-      if (head < nq) {
-        float *q = qrow + (size_t)b * qdim + head * d;
-        px::st_tf(q + i, u, tag);
-        px::st_tf(q + i + hd, w, tag);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int off = 16 >> LOG2N; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+  return t;
+}
+
+// Pages a warp takes at once in the split scheme: every warp works on the
+// same pages, so one page at a time would leave each warp's loads, FMAs and
+// shuffles a serial chain; a group of four keeps four pages' work in flight.
+constexpr int kSplitGroup = 4;
+
+// dot products of this thread's slice with the R rows of the group's pages
+// (acc[k * R + r]: page k of the group, row r; zero for pages k >= qn)
+template <int R>
+__device__ __forceinline__ void split_group_dots(const uint8_t *const (&pages)[kSplitGroup], int qn, int cw, int lane,
+                                                 const float (&xa)[Split<R>::NX], float (&acc)[kSplitGroup * R]) {
+  using G = Split<R>;
+  uint4 w[kSplitGroup][R][G::CPL];
+#pragma unroll
+  for (int k = 0; k < kSplitGroup; ++k) {
+    const uint4 *pg = reinterpret_cast<const uint4 *>(pages[k]);
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < G::CPL; ++j)
+        w[k][r][j] = k < qn ? pg[r * (G::KC / 8) + split_chunk<R>(cw, lane, j)] : make_uint4(0u, 0u, 0u, 0u);
+  }
+  // packed pair FMAs: even and odd columns accumulate in the two halves of a
+  // 64-bit register pair (12 instead of 16 instructions per 8 weights)
+  unsigned long long xp[4 * G::CPL];
+#pragma unroll
+  for (int j = 0; j < 4 * G::CPL; ++j) xp[j] = px::f2pack(xa[2 * j], xa[2 * j + 1]);
+#pragma unroll
+  for (int k = 0; k < kSplitGroup; ++k)
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      unsigned long long s2 = 0ull;
+#pragma unroll
+      for (int j = 0; j < G::CPL; ++j) {
+        const uint4 q = w[k][r][j];
+        px::ffma2(s2, px::f2pack(px::bf_lo(q.x), px::bf_hi(q.x)), xp[4 * j + 0]);
+        px::ffma2(s2, px::f2pack(px::bf_lo(q.y), px::bf_hi(q.y)), xp[4 * j + 1]);
+        px::ffma2(s2, px::f2pack(px::bf_lo(q.z), px::bf_hi(q.z)), xp[4 * j + 2]);
+        px::ffma2(s2, px::f2pack(px::bf_lo(q.w), px::bf_hi(q.w)), xp[4 * j + 3]);
+      }
+      acc[k * R + r] = px::f2sum(s2);
+    }
+}
+
+// The instruction's pages, split across the warps.  PAIRED: the epilogue
+// takes rows (i, i + R/2) of a page together, epi(page, i, v_i, v_{i+R/2})
+// (RoPE pairs, gate/up); else epi(page, r, v_r).  Called by every compute
+// thread; every thread passes the same barriers even after an abort.
+template <int R, bool PAIRED, class Epi>
+__device__ __forceinline__ void matvec_split(CCtx &c, const Instr &I, const float (&xa)[Split<R>::NX], Epi epi) {
+  using G = Split<R>;
+  constexpr int NV = kSplitGroup * R;  // values reduced per group
+  constexpr int LPV = 32 / NV;         // lanes holding each reduced value
+  static_assert(G::T % kSplitGroup == 0, "epilogue batches hold whole groups");
+  const Ring rg = ring_of(c);
+  const uint32_t g0 = c.g;
+  const int np = (int)I.b, first = (int)I.a, cw = c.cw, lane = c.lane, ctid = c.ctid;
+  float *const red = c.act;  // [2][T][R][8 warps]
+  bool dead = false;
+  int buf = 0;
+  // ring slot and phase of the next page, advanced page by page (no division
+  // by the ring size per page)
+  uint32_t slot = g0 % rg.np, ph = (g0 / rg.np) & 1u;
+  for (int t0 = 0; t0 < np; t0 += G::T, buf ^= 1) {
+    const int tn = min(G::T, np - t0);
+    float *const rb = red + buf * (G::T * R * 8);
+    for (int q0 = 0; q0 < tn; q0 += kSplitGroup) {
+      const int qn = min(kSplitGroup, tn - q0);
+      const uint8_t *pages[kSplitGroup];
+      uint32_t slots[kSplitGroup];
+#pragma unroll
+      for (int k = 0; k < kSplitGroup; ++k) {
+        slots[k] = slot;
+        pages[k] = rg.pages + (size_t)slot * kPageBytes;
+        if (k < qn) {
+          if (!dead && !ring_wait_full(c.p, rg, slot, ph)) dead = true;
+          if (++slot == rg.np) {
+            slot = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (dead) continue;
+      float acc[NV];
+      split_group_dots<R>(pages, qn, cw, lane, xa, acc);
+      __syncwarp();
+      if (lane == 0)
+        for (int k = 0; k < qn; ++k) px::mbar_arrive(&rg.empty[slots[k]], 1);
+      const float v = warp_sum_rows<NV>(acc, lane);
+      const int idx = lane / LPV;  // k * R + r
+      if ((lane & (LPV - 1)) == 0 && idx / R < qn) rb[((q0 + idx / R) * R + idx % R) * 8 + cw] = v;
+    }
+    px::cbar();  // every warp's partials of this batch are in rb
+    constexpr int PER = PAIRED ? R / 2 : R;
+    if (ctid < tn * PER) {
+      const int tt = ctid / PER, i = ctid % PER;
+      const float4 *a = reinterpret_cast<const float4 *>(rb + (tt * R + i) * 8);
+      const float4 a0 = a[0], a1 = a[1];
+      const float va = ((((((a0.x + a0.y) + a0.z) + a0.w) + a1.x) + a1.y) + a1.z) + a1.w;
+      if constexpr (PAIRED) {
+        const float4 *b = reinterpret_cast<const float4 *>(rb + (tt * R + i + R / 2) * 8);
+        const float4 b0 = b[0], b1 = b[1];
+        const float vb = ((((((b0.x + b0.y) + b0.z) + b0.w) + b1.x) + b1.y) + b1.z) + b1.w;
+        epi(first + t0 + tt, i, va, vb);
       } else {
-        // the cache row (bf16) for later steps, and the rounded values for
-        // this step's attention as tagged words
-        const bool isk = head < nq + nkv;
-        const int gk = isk ? head - nq : head - nq - nkv;
-        uint16_t *dst = (isk ? kl : vl) + (size_t)b * kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
-        const uint16_t bu = px::f2bf(u), bw = px::f2bf(w);
-        dst[i] = bu;
-        dst[i + hd] = bw;
-        float *cur = kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + gk * d;
-        px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 22 significant bits
-        px::st_tf(cur + i + hd, px::bf16f(bw), tag);
+        epi(first + t0 + tt, i, va);
+      }
+    }
+    // the other buffer is rewritten by the next batch only after the next
+    // barrier, which every epilogue thread reaches after its reads
+  }
+  c.g = g0 + (uint32_t)np;
+}
+
+// This thread's slice of x_in(l) (QKV: the residual stream entering layer l;
+// gate/up: x_mid from xres[l]; LM head: l == L) times gamma, and 1 / rms(x):
+// the dot products are scaled by it afterwards.  One compute barrier.
+template <int R>
+__device__ __forceinline__ float stage_split_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only,
+                                                  float (&xa)[Split<R>::NX]) {
+  using G = Split<R>;
+  const KParams &p = c.p;
+  float4 xs[2 * G::CPL];
+  uint4 gw[G::CPL];
+  const int tok = (l == 0 && !from_xres_only) ? read_tok(c.sh, 0) : 0;
+  settle(c, 2, [&](bool &ok) {
+#pragma unroll
+    for (int j = 0; j < G::CPL; ++j) {
+      const int ch = split_chunk<R>(c.cw, c.lane, j);
+      gw[j] = __ldg(reinterpret_cast<const uint4 *>(gamma) + ch);  // with x: one round trip
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e4 = 2 * ch + h;
+        xs[2 * j + h] = from_xres_only ? ll_load4(c.epoch, p.xres + (size_t)l * p.H + e4 * 4, ok)
+                                       : layer_input4(p, c.epoch, l, 0, tok, e4, ok);
       }
     }
   });
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < G::CPL; ++j) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float4 x = xs[2 * j + h];
+      const uint32_t g01 = h ? gw[j].z : gw[j].x, g23 = h ? gw[j].w : gw[j].y;
+      ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      float *o = xa + 8 * j + 4 * h;
+      o[0] = x.x * px::bf_lo(g01);
+      o[1] = x.y * px::bf_hi(g01);
+      o[2] = x.z * px::bf_lo(g23);
+      o[3] = x.w * px::bf_hi(g23);
+    }
+  }
+  ss = px::warp_sum(ss);
+  if (c.lane == 0) c.sh->red[c.cw][0] = ss;
+  px::cbar();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kComputeWarps; ++w) t += c.sh->red[w][0];
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+  return __frsqrt_rn(t * p.inv_H + p.eps);  // one rounding; t * (1/H) == t / H for H = 2^k
+}
+
+// This thread's slice of a tagged fp32 vector (attention output, SwiGLU
+// activations); with nrows > 0 (O projection) also x_in(l) for output rows
+// row0 .. row0 + nrows into the staging region after the partial table,
+// loaded in the same round trip.
+template <int R>
+__device__ __forceinline__ void stage_split_copy(CCtx &c, const float *src, float (&xa)[Split<R>::NX], int l = 0,
+                                                 int row0 = 0, int nrows = 0) {
+  using G = Split<R>;
+  const KParams &p = c.p;
+  const bool has_row = c.ctid < nrows;
+  const int tok0 = l == 0 ? read_tok(c.sh, 0) : 0;
+  float xr = 0.f;
+  float4 xs[2 * G::CPL];
+  settle(c, 3, [&](bool &ok) {
+    if (has_row) xr = layer_input1(p, c.epoch, l, 0, tok0, row0 + c.ctid, ok);
+#pragma unroll
+    for (int j = 0; j < G::CPL; ++j) {
+      const int ch = split_chunk<R>(c.cw, c.lane, j);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) xs[2 * j + h] = ll_load4(c.epoch, src + (2 * ch + h) * 4, ok);
+    }
+  });
+#pragma unroll
+  for (int j = 0; j < G::CPL; ++j)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float4 x = xs[2 * j + h];
+      float *o = xa + 8 * j + 4 * h;
+      o[0] = x.x;
+      o[1] = x.y;
+      o[2] = x.z;
+      o[3] = x.w;
+    }
+  float *rows = c.act + kSplitRedFloats;
+  for (int r = c.ctid; r < nrows; r += kComputeThreads)
+    rows[r] = (r == c.ctid) ? xr : layer_input1_settled(p, c.sh, c.epoch, l, 0, tok0, row0 + r);
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+}
+
+// Normed input of a split-page instruction: 1 / rms(x), with x * gamma as
+// this thread's register slice.
+template <int R, int MODE>
+__device__ __forceinline__ float stage_rows_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres_only,
+                                                 float (&xa)[Split<R>::NX]) {
+  static_assert(MODE == 1, "split pages");
+  return stage_split_norm<R>(c, l, gamma, from_xres_only, xa);
+}
+template <int R, int MODE, bool PAIRED, class Epi>
+__device__ __forceinline__ void matvec_rows(CCtx &c, const Instr &I, const float (&xa)[Split<R>::NX], Epi epi) {
+  static_assert(MODE == 1, "split pages");
+  matvec_split<R, PAIRED>(c, I, xa, epi);
+}
+
+template <int R, int MODE>
+__device__ __forceinline__ uint32_t qkv_rows(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer;
+  float xa[Split<R>::NX];
+  const float inv = stage_rows_norm<R, MODE>(c, l, p.layers[l].attn_norm, false, xa);
+  const int half = R / 2, pph = p.d / R, hd = p.d / 2, pos = read_pos(c.sh, 0);
+  const int nq = p.nq, nkv = p.nkv, d = p.d, kvdim = p.kvdim;
+  const uint32_t tag = c.epoch;
+  float *const qrow = p.qbuf + (size_t)l * p.qdim;
+  float *const kvc = p.kvcur + (size_t)l * 2 * kvdim;
+  uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
+  const long long kv_hs = p.kv_hs;
+  const float2 *rope_s = c.sh->rope;
+  matvec_rows<R, MODE, true>(c, I, xa, [&](int j, int pr, float u, float w) {
+    const int head = j / pph, jj = j % pph;
+    const int i = jj * half + pr;  // rotation pair index inside the head
+    u *= inv;
+    w *= inv;
+    if (head < nq + nkv) {
+      const float2 cs = rope_s[i];
+      const float u2 = u * cs.x - w * cs.y, w2 = u * cs.y + w * cs.x;
+      u = u2;
+      w = w2;
+    }
+    if (head < nq) {
+      float *q = qrow + head * d;
+      px::st_tf(q + i, u, tag);
+      px::st_tf(q + i + hd, w, tag);
+    } else {
+      const bool isk = head < nq + nkv;
+      const int gk = isk ? head - nq : head - nq - nkv;
+      uint16_t *dst = (isk ? kl : vl) + (size_t)gk * kv_hs + (size_t)pos * d;
+      const uint16_t bu = px::f2bf(u), bw = px::f2bf(w);
+      dst[i] = bu;
+      dst[i + hd] = bw;
+      float *cur = kvc + (isk ? 0 : kvdim) + gk * d;
+      px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 22 significant bits
+      px::st_tf(cur + i + hd, px::bf16f(bw), tag);
+    }
+  });
   return c.g;
+}
+
+template <int R, int MODE>
+__device__ __forceinline__ uint32_t oproj_rows(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer;
+  const int row0 = (int)I.a * R, nrows = (int)I.b * R;
+  float xa[Split<R>::NX];
+  // the residual rows x_in(l)[row0 ..] follow the split partial table
+  stage_split_copy<R>(c, p.obuf + (size_t)l * p.qdim, xa, l, row0, nrows);
+  const uint32_t tag = c.epoch;
+  const float *xrows = c.act + kSplitRedFloats - row0;
+  float *const xout = p.xres + (size_t)l * p.H;
+  matvec_rows<R, MODE, false>(c, I, xa, [&](int j, int r, float v) {
+    const int row = j * R + r;
+    px::st_tf(xout + row, xrows[row] + v, tag);
+  });
+  return c.g;
+}
+
+template <int R, int MODE>
+__device__ __forceinline__ uint32_t gateup_rows(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer;
+  float xa[Split<R>::NX];
+  const float inv = stage_rows_norm<R, MODE>(c, l, p.layers[l].ffn_norm, true, xa);
+  const int half = R / 2;
+  const uint32_t tag = c.epoch;
+  float *const aout = p.actb + (size_t)l * p.F;
+  matvec_rows<R, MODE, true>(c, I, xa, [&](int j, int pr, float gt, float up) {
+    gt *= inv;
+    up *= inv;
+    const float silu = gt / (1.0f + expf(-gt));
+    px::st_tf(aout + j * half + pr, silu * up, tag);
+  });
+  return c.g;
+}
+
+template <int R, int MODE>
+__device__ __forceinline__ uint32_t down_rows(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, k = I.c;
+  float xa[Split<R>::NX];
+  stage_split_copy<R>(c, p.actb + (size_t)l * p.F + (size_t)k * p.KCd, xa);
+  const uint32_t tag = c.epoch;
+  float *const dout = p.dpart + ((size_t)l * p.ndp + k) * p.H;
+  matvec_rows<R, MODE, false>(c, I, xa, [&](int j, int r, float v) { px::st_tf(dout + j * R + r, v, tag); });
+  return c.g;
+}
+
+// forward declaration: the LM head's argmax merge (defined with the paged bodies)
+template <int NB>
+__device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&bv)[NB], int (&bi)[NB]);
+__device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi);
+
+template <int R, int MODE>
+__device__ __forceinline__ uint32_t lmhead_rows(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  float xa[Split<R>::NX];
+  const float inv = stage_rows_norm<R, MODE>(c, p.L, p.final_norm, false, xa);
+  float bv[1] = {-INFINITY};
+  int bi[1] = {0x7fffffff};
+  const int V = p.V;
+  float *const logits = p.logits;
+  matvec_rows<R, MODE, false>(c, I, xa, [&](int j, int r, float v) {
+    const int row = j * R + r;
+    if (row >= V) return;  // the rows past the vocabulary of a partial last page
+    v *= inv;
+    if (logits) logits[row] = v;
+    if (arg_better(v, row, bv[0], bi[0])) {
+      bv[0] = v;
+      bi[0] = row;
+    }
+  });
+  lm_argmax_tail<1>(c, I, bv, bi);
+  return c.g;
+}
+
+template <int NB, int R, bool SPL = false>
+__device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
+  if constexpr (Scheme<NB, R, SPL>::v != 0) {
+    return qkv_rows<R, Scheme<NB, R, SPL>::v>(c, I);
+  } else {
+    const KParams &p = c.p;
+    const int l = I.layer;
+    const int half = R / 2, pph = p.d / R, hd = p.d / 2;
+    const int pos0 = read_pos(c.sh, 0);
+    float inv[NB];
+    stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].attn_norm, false, inv);
+    const int nq = p.nq, nkv = p.nkv, d = p.d, lane = c.lane, Bn = p.B, kvdim = p.kvdim;
+    const uint32_t tag = c.epoch;
+    float *const qrow = p.qbuf + (size_t)l * Bn * p.qdim;
+    float *const kvc = p.kvcur + (size_t)l * Bn * 2 * kvdim;
+    uint16_t *const kl = p.kc + (size_t)l * p.kv_ls, *const vl = p.vc + (size_t)l * p.kv_ls;
+    const long long kv_bs = p.kv_bs, kv_hs = p.kv_hs;
+    const int qdim = p.qdim;
+    const float2 *rope_s = c.sh->rope;
+    const float2 *rope_g = p.rope;
+    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+      const int head = j / pph, jj = j % pph;
+      if (lane >= half) return;
+      const int i = jj * half + lane;  // rotation pair index inside the head
+  #pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (NB > 1 && b >= Bn) break;
+        float u = pick<R>(acc[b], lane) * inv[b], w = pick<R>(acc[b], lane + half) * inv[b];
+        const int pos = NB == 1 ? pos0 : read_pos(c.sh, b);
+        if (head < nq + nkv) {
+          const float2 cs = NB == 1 ? rope_s[i] : __ldg(rope_g + (size_t)pos * hd + i);
+          const float u2 = u * cs.x - w * cs.y, w2 = u * cs.y + w * cs.x;
+          u = u2;
+          w = w2;
+        }
+        if (head < nq) {
+          float *q = qrow + (size_t)b * qdim + head * d;
+          px::st_tf(q + i, u, tag);
+          px::st_tf(q + i + hd, w, tag);
+        } else {
+          // the cache row (bf16) for later steps, and the rounded values for
+          // this step's attention as tagged words
+          const bool isk = head < nq + nkv;
+          const int gk = isk ? head - nq : head - nq - nkv;
+          uint16_t *dst = (isk ? kl : vl) + (size_t)b * kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
+          const uint16_t bu = px::f2bf(u), bw = px::f2bf(w);
+          dst[i] = bu;
+          dst[i + hd] = bw;
+          float *cur = kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + gk * d;
+          px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 22 significant bits
+          px::st_tf(cur + i + hd, px::bf16f(bw), tag);
+        }
+      }
+    });
+    return c.g;
+  }
 }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_qkv(CCtx c, const Instr I) { return qkv_body<NB, R>(c, I); }
 
-template <int NB, int R>
+template <int NB, int R, bool SPL = false>
 __device__ __forceinline__ uint32_t oproj_body(CCtx c, const Instr I) {
-  const KParams &p = c.p;
-  const int l = I.layer;
-  const int row0 = (int)I.a * R, nrows = NB == 1 ? (int)I.b * R : 0;
-  stage_copy<NB, StageIt<R>::v>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim, l, row0, nrows);
-  const int lane = c.lane, Bn = p.B, H = p.H;
-  const uint32_t tag = c.epoch;
-  const float *xrows = c.act + p.qdim - row0;
-  float *const xout = p.xres + (size_t)l * Bn * H;
-  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    if (lane >= R) return;
-    const int row = j * R + lane;
-    if constexpr (NB == 1) {
-      px::st_tf(xout + row, xrows[row] + pick<R>(acc[0], lane), tag);
-    } else {
-      // the residual row of every sequence: one group of loads (retried as a whole)
-      float xin[NB];
-      for (LLRetry r;;) {
-        bool ok = true;
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-          if (b < Bn) xin[b] = layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
-        if (ok || !ll_retry(p, c.sh, r, 9)) break;
+  if constexpr (Scheme<NB, R, SPL>::v != 0) {
+    return oproj_rows<R, Scheme<NB, R, SPL>::v>(c, I);
+  } else {
+    const KParams &p = c.p;
+    const int l = I.layer;
+    const int row0 = (int)I.a * R, nrows = NB == 1 ? (int)I.b * R : 0;
+    stage_copy<NB, StageIt<R>::v>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim, l, row0, nrows);
+    const int lane = c.lane, Bn = p.B, H = p.H;
+    const uint32_t tag = c.epoch;
+    const float *xrows = c.act + p.qdim - row0;
+    float *const xout = p.xres + (size_t)l * Bn * H;
+    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+      if (lane >= R) return;
+      const int row = j * R + lane;
+      if constexpr (NB == 1) {
+        px::st_tf(xout + row, xrows[row] + pick<R>(acc[0], lane), tag);
+      } else {
+        // the residual row of every sequence: one group of loads (retried as a whole)
+        float xin[NB];
+        for (LLRetry r;;) {
+          bool ok = true;
+  #pragma unroll
+          for (int b = 0; b < NB; ++b)
+            if (b < Bn) xin[b] = layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
+          if (ok || !ll_retry(p, c.sh, r, 9)) break;
+        }
+  #pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= Bn) break;
+          px::st_tf(xout + (size_t)b * H + row, xin[b] + pick<R>(acc[b], lane), tag);
+        }
       }
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        if (b >= Bn) break;
-        px::st_tf(xout + (size_t)b * H + row, xin[b] + pick<R>(acc[b], lane), tag);
-      }
-    }
-  });
-  return c.g;
+    });
+    return c.g;
+  }
 }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_oproj(CCtx c, const Instr I) { return oproj_body<NB, R>(c, I); }
 
-template <int NB, int R>
+template <int NB, int R, bool SPL = false>
 __device__ __forceinline__ uint32_t gateup_body(CCtx c, const Instr I) {
-  const KParams &p = c.p;
-  const int l = I.layer;
-  float inv[NB];
-  stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].ffn_norm, true, inv);
-  const int half = R / 2, lane = c.lane, Bn = p.B, F = p.F;
-  const uint32_t tag = c.epoch;
-  float *const aout = p.actb + (size_t)l * Bn * F;
-  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    if (lane >= half) return;
-    const int row = j * half + lane;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      if (NB > 1 && b >= Bn) break;
-      const float gt = pick<R>(acc[b], lane) * inv[b], up = pick<R>(acc[b], lane + half) * inv[b];
-      const float silu = gt / (1.0f + expf(-gt));
-      px::st_tf(aout + (size_t)b * F + row, silu * up, tag);
-    }
-  });
-  return c.g;
+  if constexpr (Scheme<NB, R, SPL>::v != 0) {
+    return gateup_rows<R, Scheme<NB, R, SPL>::v>(c, I);
+  } else {
+    const KParams &p = c.p;
+    const int l = I.layer;
+    float inv[NB];
+    stage_norm<NB, StageIt<R>::v>(c, l, p.layers[l].ffn_norm, true, inv);
+    const int half = R / 2, lane = c.lane, Bn = p.B, F = p.F;
+    const uint32_t tag = c.epoch;
+    float *const aout = p.actb + (size_t)l * Bn * F;
+    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+      if (lane >= half) return;
+      const int row = j * half + lane;
+  #pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (NB > 1 && b >= Bn) break;
+        const float gt = pick<R>(acc[b], lane) * inv[b], up = pick<R>(acc[b], lane + half) * inv[b];
+        const float silu = gt / (1.0f + expf(-gt));
+        px::st_tf(aout + (size_t)b * F + row, silu * up, tag);
+      }
+    });
+    return c.g;
+  }
 }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_gateup(CCtx c, const Instr I) { return gateup_body<NB, R>(c, I); }
 
-template <int NB, int R>
+template <int NB, int R, bool SPL = false>
 __device__ __forceinline__ uint32_t down_body(CCtx c, const Instr I) {
-  const KParams &p = c.p;
-  const int l = I.layer, k = I.c;
-  stage_copy<NB, StageIt<R>::v>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
-  const int lane = c.lane, Bn = p.B, H = p.H;
-  const uint32_t tag = c.epoch;
-  float *const dout = p.dpart + ((size_t)l * p.ndp + k) * Bn * H;
-  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    if (lane >= R) return;
-    const int row = j * R + lane;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      if (NB > 1 && b >= Bn) break;
-      px::st_tf(dout + (size_t)b * H + row, pick<R>(acc[b], lane), tag);
-    }
-  });
-  return c.g;
+  if constexpr (Scheme<NB, R, SPL>::v != 0) {
+    return down_rows<R, Scheme<NB, R, SPL>::v>(c, I);
+  } else {
+    const KParams &p = c.p;
+    const int l = I.layer, k = I.c;
+    stage_copy<NB, StageIt<R>::v>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
+    const int lane = c.lane, Bn = p.B, H = p.H;
+    const uint32_t tag = c.epoch;
+    float *const dout = p.dpart + ((size_t)l * p.ndp + k) * Bn * H;
+    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+      if (lane >= R) return;
+      const int row = j * R + lane;
+  #pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (NB > 1 && b >= Bn) break;
+        px::st_tf(dout + (size_t)b * H + row, pick<R>(acc[b], lane), tag);
+      }
+    });
+    return c.g;
+  }
 }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_down(CCtx c, const Instr I) { return down_body<NB, R>(c, I); }
@@ -1383,38 +1828,42 @@ __device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&
   }
 }
 
-template <int NB, int R>
+template <int NB, int R, bool SPL = false>
 __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
-  const KParams &p = c.p;
-  float inv[NB];
-  stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false, inv);
-  float bv[NB];
-  int bi[NB];
-#pragma unroll
-  for (int b = 0; b < NB; ++b) {
-    bv[b] = -INFINITY;
-    bi[b] = 0x7fffffff;
-  }
-  const int lane = c.lane, Bn = p.B, V = p.V;
-  float *const logits = p.logits;
-  matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-    const int row = j * R + lane;
-    const bool valid = lane < R && row < V;
-#pragma unroll
+  if constexpr (Scheme<NB, R, SPL>::v != 0) {
+    return lmhead_rows<R, Scheme<NB, R, SPL>::v>(c, I);
+  } else {
+    const KParams &p = c.p;
+    float inv[NB];
+    stage_norm<NB, StageIt<R>::v>(c, p.L, p.final_norm, false, inv);
+    float bv[NB];
+    int bi[NB];
+  #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      if (NB > 1 && b >= Bn) break;
-      const float v = pick<R>(acc[b], lane) * inv[b];
-      if (valid) {
-        if (logits) logits[(size_t)b * V + row] = v;
-        if (arg_better(v, row, bv[b], bi[b])) {
-          bv[b] = v;
-          bi[b] = row;
+      bv[b] = -INFINITY;
+      bi[b] = 0x7fffffff;
+    }
+    const int lane = c.lane, Bn = p.B, V = p.V;
+    float *const logits = p.logits;
+    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+      const int row = j * R + lane;
+      const bool valid = lane < R && row < V;
+  #pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (NB > 1 && b >= Bn) break;
+        const float v = pick<R>(acc[b], lane) * inv[b];
+        if (valid) {
+          if (logits) logits[(size_t)b * V + row] = v;
+          if (arg_better(v, row, bv[b], bi[b])) {
+            bv[b] = v;
+            bi[b] = row;
+          }
         }
       }
-    }
-  });
-  lm_argmax_tail<NB>(c, I, bv, bi);
-  return c.g;
+    });
+    lm_argmax_tail<NB>(c, I, bv, bi);
+    return c.g;
+  }
 }
 
 // Tensor-core matrix product for batched builds: the matrix is in 128-row
@@ -1835,6 +2284,10 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   const float *kcur = p.kvcur + (((size_t)l * p.B + b) * 2) * p.kvdim + (size_t)g * D;
   const float *vcur = kcur + p.kvdim;
   const float *qb = p.qbuf + ((size_t)l * p.B + b) * p.qdim + (size_t)g * G * D;
+  // scratch in the staging region: [warp][G][D + 2] floats, then the
+  // current position's K and V rows (bf16)
+  float *scr = c.act;
+  uint16_t *cur = reinterpret_cast<uint16_t *>(c.act + kComputeWarps * G * (D + 2));
   float q[G][DPL], ck[DPL], cv[DPL];
   settle(c, 5, [&](bool &ok) {
     uint32_t wk[DPL], wv[DPL], wq[G][DPL];
@@ -1870,10 +2323,6 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
 #pragma unroll
     for (int i = 0; i < DPL; ++i) o[h][i] = 0.f;
   }
-  // scratch in the staging region: [warp][G][D + 2] floats, then the
-  // current position's K and V rows (bf16)
-  float *scr = c.act;
-  uint16_t *cur = reinterpret_cast<uint16_t *>(c.act + kComputeWarps * G * (D + 2));
   if (load_cur) {
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
@@ -1950,8 +2399,9 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
     for (int w = 0; w < kComputeWarps; ++w) O += fac[h * kComputeWarps + w] * scr[((size_t)w * G + h) * (D + 2) + dd];
     px::st_tf(p.part_o + ((hbase + h) * p.S + s) * D + dd, O, tag);
     if (dd == 0) {
-      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 0, fac[G * kComputeWarps + h], tag);
-      px::st_ll(p.part_ml + ((hbase + h) * p.S + s) * 2 + 1, fac[G * kComputeWarps + G + h], tag);
+      llw *ml = p.part_ml + ((hbase + h) * p.S + s) * 2;
+      px::st_ll(ml + 0, fac[G * kComputeWarps + h], tag);
+      px::st_ll(ml + 1, fac[G * kComputeWarps + G + h], tag);
     }
   }
   px::cbar();
@@ -2078,10 +2528,11 @@ __device__ __forceinline__ int &sh_stat(CCtx &c) { return c.sh->stat_cwait; }
 // (all zero) reaches the bodies through calls selected at run time.  TQO
 // (batched builds): QKV and the O projection may run as tensor-core tiles; a
 // build of its own, since the extra op bodies raise every body's spills.
-template <int RH_, int RO_, int RD_, int G_, int DPL_, bool TQO_ = false>
+template <int RH_, int RO_, int RD_, int G_, int DPL_, bool TQO_ = false, bool SPL_ = false>
 struct Spec {
   static constexpr bool fixed = RH_ > 0;
   static constexpr bool TQO = TQO_;
+  static constexpr bool SPL = SPL_;  // batch 1: split pages for rows of 2048 / 4096 columns
   static constexpr int RH = RH_, RO = RO_, RD = RD_, G = G_, DPL = DPL_;
 };
 using SpecGeneric = Spec<0, 0, 0, 0, 0>;
@@ -2163,7 +2614,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
             break;
           }
         }
-        if constexpr (kInline) c.g = qkv_body<NB, S::RH>(c, I);
+        if constexpr (kInline) c.g = qkv_body<NB, S::RH, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_qkv<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_qkv, NB, p.Rh, c, I);
         break;
@@ -2179,7 +2630,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
             break;
           }
         }
-        if constexpr (kInline) c.g = oproj_body<NB, S::RO>(c, I);
+        if constexpr (kInline) c.g = oproj_body<NB, S::RO, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_oproj<NB, S::RO>(c, I);
         else MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);
         break;
@@ -2190,7 +2641,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
             break;
           }
         }
-        if constexpr (kInline) c.g = gateup_body<NB, S::RH>(c, I);
+        if constexpr (kInline) c.g = gateup_body<NB, S::RH, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_gateup<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_gateup, NB, p.Rh, c, I);
         break;
@@ -2201,7 +2652,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
             break;
           }
         }
-        if constexpr (kInline) c.g = down_body<NB, S::RD>(c, I);
+        if constexpr (kInline) c.g = down_body<NB, S::RD, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_down<NB, S::RD>(c, I);
         else MK_DISPATCH_R(op_down, NB, p.Rd, c, I);
         break;
@@ -2212,7 +2663,7 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
             break;
           }
         }
-        if constexpr (kInline) c.g = lmhead_body<NB, S::RH>(c, I);
+        if constexpr (kInline) c.g = lmhead_body<NB, S::RH, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_lmhead<NB, S::RH>(c, I);
         else MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I);
         break;

@@ -12,6 +12,16 @@ namespace mk {
 // Dynamic shared memory of a CTA with `num_pages` ring pages and a staging
 // region of `act_floats` floats.
 int shared_bytes_fixed(int num_pages, size_t act_floats);
+// Floats of the staging region for a model shape and `nb` sequences per
+// instruction (1, or kMaxBatch for batched builds): input vectors or the
+// split-page partial table and the O projection's residual rows, the
+// attention scratch, and in batched builds the tensor-core exchange.
+size_t staging_floats(int H, int qdim, int KCd, int G, int d, int nb);
+// Ring pages that fit next to a staging region of `act_floats` floats in
+// `smem_optin` bytes: a multiple of the loader count with twice it a
+// multiple of the compute-warp count (unambiguous mbarrier phases), at most
+// 16; 0 if fewer than 2 * kLoaders fit.
+int ring_pages(int smem_optin, size_t act_floats);
 // The interpreter kernel for the model shape in p and `nb` sequences per
 // instruction (1, or kMaxBatch for batched plans): a shape-specialised build
 // when one exists and `specialised` is set (*variant = 1), else the

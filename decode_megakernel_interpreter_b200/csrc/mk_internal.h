@@ -22,6 +22,7 @@ constexpr int kMaxBatch = 16;
 constexpr int kMaxDownPieces = 8;             // ffn / 2048 at most
 constexpr int kDefaultInflight = 4;           // bulk-copy pages in flight per CTA
 constexpr int kTcXchFloats = 128 * 16;        // batched builds: tensor-core epilogue exchange (floats)
+constexpr int kSplitRedFloats = 1024;         // batch 1: split-page row partials (floats, staging region)
 
 // ---------------------------------------------------------------- opcodes
 // The instruction set of the decode step (the fused instructions the

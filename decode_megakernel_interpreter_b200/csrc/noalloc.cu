@@ -148,14 +148,9 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   if (lay.off > MK_NOALLOC_SCRATCH_BYTES) return MK_ERR_UNSUPPORTED_SHAPE;
 
   // shared memory geometry (as mk_plan)
-  const int G = s.nq / s.nkv;
-  size_t act = std::max(std::max((size_t)s.H, qd + (size_t)s.H), (size_t)p.KCd);
-  act = std::max(act, (size_t)kComputeWarps * G * (s.d + 2) + s.d + (size_t)G * (kComputeWarps + 2));
-  act = (act + 31) / 32 * 32;
-  int num_pages = std::min(16, (slot->smem_optin - shared_bytes_fixed(0, act)) / (kPageBytes + 16));
-  num_pages = num_pages / kLoaders * kLoaders;  // as mk_plan: unambiguous mbarrier phases
-  while (num_pages > 0 && (2 * num_pages) % kComputeWarps) num_pages -= kLoaders;
-  if (num_pages < 2 * kLoaders) return MK_ERR_UNSUPPORTED_SHAPE;
+  const size_t act = staging_floats(s.H, (int)qd, p.KCd, s.nq / s.nkv, s.d, 1);
+  const int num_pages = ring_pages(slot->smem_optin, act);  // as mk_plan
+  if (num_pages == 0) return MK_ERR_UNSUPPORTED_SHAPE;
   const int smem = shared_bytes_fixed(num_pages, act);
 
   unsigned char *base = slot->scratch;

@@ -638,3 +638,154 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
 }
 
 }  // namespace mk
+
+// ------------------------------------------------------------------ cost model
+
+namespace mk {
+
+namespace {
+
+// weight pages one instruction streams (tensor-core units are whole tiles of
+// 64-column pages), and how many of its pages are K/V (attention)
+int instr_pages(const PlanRequest &req, const Plan &p, const Instr &I, int context, bool *kv) {
+  const Shape &s = req.s;
+  *kv = false;
+  switch (I.op) {
+    case OP_QKV: return (int)I.b * (p.tensor_qkv_o ? s.H / 64 : 1);
+    case OP_OPROJ: return (int)I.b * (p.tensor_qkv_o ? s.nq * s.d / 64 : 1);
+    case OP_GATEUP: return (int)I.b * (p.tensor ? s.H / 64 : 1);
+    case OP_DOWN: return (int)I.b * (p.tensor ? p.KCd / 64 : 1);
+    case OP_LMHEAD: return (int)I.b * (p.tensor ? s.H / 64 : 1);
+    case OP_ATTN: {
+      *kv = true;
+      const int n = context + 1, chunk = (n + p.S - 1) / p.S;
+      const int start = std::min(n, (int)I.b * chunk), end = std::min(n, start + chunk);
+      const int cached = std::max(0, std::min(end, context) - start);
+      const int ppp = kPageBytes / (4 * s.d);
+      return (cached + ppp - 1) / ppp;
+    }
+    default: return 0;
+  }
+}
+
+// compute time of one weight page of an instruction
+double page_time(const PlanRequest &req, const Plan &p, const Instr &I, const CostParams &c) {
+  if (req.B == 1) return c.page_us;
+  const bool tc = (I.op == OP_GATEUP || I.op == OP_DOWN || I.op == OP_LMHEAD) ? p.tensor
+                  : (I.op == OP_QKV || I.op == OP_OPROJ)                     ? p.tensor_qkv_o
+                                                                             : false;
+  return tc ? c.tc_page_us : c.cc_page_us_seq * req.B;
+}
+
+}  // namespace
+
+std::string estimate_plan(const PlanRequest &req, const Plan &p, const CostParams &c, int context,
+                          CostEstimate *out) {
+  if (p.dynamic) return "the cost model replays static queues";
+  if (context < 0 || c.sm_gbs <= 0 || c.ring_pages < 1) return "bad cost parameters";
+  const Shape &s = req.s;
+  const int n = p.num_ctas;
+  const double t_hbm = kPageBytes / (c.sm_gbs * 1e3);  // us per 16 KiB page at one SM's bandwidth
+  std::vector<const Instr *> order(p.instrs.size());
+  std::vector<int> cta_of(p.instrs.size());
+  for (int q = 0; q < n; ++q)
+    for (int i = 0; i < p.q_len[q]; ++i) {
+      const Instr &I = p.instrs[p.q_off[q] + i];
+      order[I.seq] = &I;
+      cta_of[I.seq] = q;
+    }
+  // per-CTA state: compute warps free at, loader's last arrival, and the
+  // consumption times of the last ring_pages pages (their slots free then)
+  std::vector<double> t_cta(n, 0.0), arrive(n, 0.0);
+  std::vector<std::vector<double>> ring(n);
+  std::vector<size_t> ring_head(n, 0);
+  std::vector<double> ctr_done(p.n_counters, 0.0);
+  // ticketed attention merges: latest split finish per (layer, sequence, kv head)
+  std::vector<double> group_max((size_t)s.L * req.B * s.nkv, 0.0);
+  double sum_t[7] = {0}, cnt_t[7] = {0}, end = 0.0, hbm_bytes = 0.0;
+  for (const Instr *Ip : order) {
+    const Instr &I = *Ip;
+    const int q = cta_of[I.seq];
+    if (I.op == OP_NOP) continue;
+    double dep = 0.0;
+    if (I.wait_ctr != kNoCounter) dep = ctr_done[I.wait_ctr] + c.exchange_us;
+    const double start = std::max(t_cta[q], dep);
+    bool kv = false;
+    const int np = instr_pages(req, p, I, context, &kv);
+    const double pt = kv ? c.attn_page_us : page_time(req, p, I, c);
+    double done = start;
+    for (int k = 0; k < np; ++k) {
+      // the loader issues a page once its ring slot is free, one SM's
+      // bandwidth apart
+      std::vector<double> &rg = ring[q];
+      const double slot_free = rg.size() < (size_t)c.ring_pages ? 0.0 : rg[ring_head[q]];
+      arrive[q] = std::max(arrive[q], slot_free) + t_hbm;
+      done = std::max(done, arrive[q]) + pt;
+      if (rg.size() < (size_t)c.ring_pages) {
+        rg.push_back(done);
+      } else {
+        rg[ring_head[q]] = done;
+        ring_head[q] = (ring_head[q] + 1) % rg.size();
+      }
+    }
+    hbm_bytes += (double)np * kPageBytes;
+    double finish = done + (I.op == OP_ATTN ? c.attn_fixed_us : c.instr_us);
+    t_cta[q] = finish;
+    sum_t[I.op] += finish - start;
+    cnt_t[I.op] += 1;
+    // producers' completion
+    if (I.op == OP_ATTN) {
+      const size_t gi = ((size_t)I.layer * req.B + I.c) * s.nkv + I.a;
+      group_max[gi] = std::max(group_max[gi], finish);
+      // the last split of the group merges: the ticket and the reload of the
+      // partials are two exchanges
+      const double merged = group_max[gi] + 2 * c.exchange_us + c.merge_us;
+      for (int k = 0; k < I.sig_n; ++k) ctr_done[I.sig_ctr + k] = std::max(ctr_done[I.sig_ctr + k], merged);
+    } else if (I.sig_ctr != kNoCounter) {
+      for (int k = 0; k < I.sig_n; ++k) ctr_done[I.sig_ctr + k] = std::max(ctr_done[I.sig_ctr + k], finish);
+    }
+    end = std::max(end, finish);
+  }
+  CostEstimate e;
+  e.step_us = end + c.exchange_us;  // the argmax merge of the LM-head instructions (ticket)
+  for (int o = 0; o < 7; ++o) e.stage_us[o] = cnt_t[o] > 0 ? sum_t[o] / cnt_t[o] : 0.0;
+  e.hbm_floor_us = hbm_bytes / (c.sm_gbs * 1e3 * n);
+  // conventional path: one launch per (layer, instruction class); a launch's
+  // instructions run on the plan's CTAs (one wave when every CTA holds at most
+  // one), each from a cold ring, and the launch ends with its slowest CTA
+  const int n_stage = s.L * kStagesPerLayer + 1;
+  std::vector<std::vector<double>> per_cta(n_stage, std::vector<double>(n, 0.0));
+  std::vector<double> merge_extra(n_stage, 0.0);
+  for (const Instr *Ip : order) {
+    const Instr &I = *Ip;
+    if (I.op == OP_NOP) continue;
+    const int st = I.op == OP_LMHEAD ? s.L * kStagesPerLayer : I.layer * kStagesPerLayer + (I.op - 1);
+    bool kv = false;
+    const int np = instr_pages(req, p, I, context, &kv);
+    const double pt = kv ? c.attn_page_us : page_time(req, p, I, c);
+    // cold ring: the first page arrives one page-time after the launch, later
+    // ones overlap compute
+    const double t = np > 0 ? t_hbm + (np - 1) * std::max(t_hbm, pt) + pt : 0.0;
+    per_cta[st][cta_of[I.seq]] += t + (kv ? c.attn_fixed_us : c.instr_us);
+    if (I.op == OP_ATTN) merge_extra[st] = 2 * c.exchange_us + c.merge_us;
+  }
+  // CTA waves: a launch whose work sits on g CTAs runs in ceil(g / W) waves
+  // on W available CTAs
+  const int W = c.conv_ctas > 0 ? std::min(c.conv_ctas, n) : n;
+  double per_op = 0.0;
+  for (int st = 0; st < n_stage; ++st) {
+    double mx = 0.0;
+    int g = 0;
+    for (double t : per_cta[st]) {
+      mx = std::max(mx, t);
+      g += t > 0.0;
+    }
+    const int waves = g > 0 ? (g + W - 1) / W : 0;
+    per_op += c.launch_us + c.exchange_us + waves * mx + merge_extra[st];
+  }
+  e.per_op_us = per_op;
+  *out = e;
+  return "";
+}
+
+}  // namespace mk

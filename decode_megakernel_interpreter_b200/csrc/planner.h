@@ -74,6 +74,46 @@ std::string build_plan(const PlanRequest &req, Plan *out);
 // written exactly once.  Returns "" when the plan is valid.
 std::string validate_plan(const PlanRequest &req, const Plan &p);
 
+// ------------------------------------------------------------------ cost model
+// Time model of a plan on the device, after the "One Megakernel is Not Enough"
+// digest (section 2.2: a service table whose operator times scale with the
+// CTA waves ceil(g / W) of the CTAs they get; section 2.3: a region is worth a
+// persistent kernel when its per-step savings S(b) over conventional launches
+// exceed its fixed cost F).  The plan's instructions are replayed in their
+// global order: each CTA streams its pages at its share of the HBM bandwidth
+// into its ring, an instruction starts once its CTA is free and its
+// producers finished plus one exchange through global memory, consumes its
+// pages at the compute rate, and finishes after a fixed epilogue/signal
+// cost.  Attention items cost a per-KV-page time; the ticketed split merge
+// adds two exchanges and the merge to the last split.  The
+// conventional path is one launch per instruction class and layer whose CTAs
+// run in ceil(items / W) waves with no prefetch across launches.
+struct CostParams {
+  double sm_gbs = 49.0;        // bulk-copy bandwidth one SM sustains (GB/s)
+  int ring_pages = 12;         // 16 KiB pages per CTA ring
+  double exchange_us = 1.6;    // a producer's last store -> a consumer's loads see it (under load)
+  double page_us = 0.13;       // compute time per 16 KiB weight page per sequence group (batch 1)
+  double attn_page_us = 0.30;  // attention compute per K/V page, all warps
+  double attn_fixed_us = 0.8;  // attention: current row, warp merge, partial stores
+  double merge_us = 0.6;       // ticketed merge: the last split's own work besides its two exchanges
+  double instr_us = 0.25;      // per instruction: fetch, barriers, epilogue, signal
+  double launch_us = 1.3;      // conventional path: one kernel launch from a CUDA graph
+  double tc_page_us = 0.20;    // batched plans: tensor-core MMAs of one weight page (16 sequences)
+  double cc_page_us_seq = 0.12;// batched plans on CUDA cores: per weight page and sequence
+  int conv_ctas = 0;           // CTAs the conventional path gets (0: the plan's); fewer -> more waves
+};
+
+struct CostEstimate {
+  double step_us = 0;          // the megakernel step
+  double per_op_us = 0;        // the conventional path (one launch per stage)
+  double hbm_floor_us = 0;     // weight + K/V bytes at every SM's share of the bandwidth
+  double stage_us[7] = {0};    // per opcode: mean instruction time (start to finish)
+};
+
+// Estimate a plan (static queues) for sequences at position `context`.
+std::string estimate_plan(const PlanRequest &req, const Plan &p, const CostParams &c, int context,
+                          CostEstimate *out);
+
 // Host simulation: `threads` CPU threads play the CTAs and run the queues
 // for `steps` steps under random delays, with real atomic counters and
 // version stamps on every buffer element; any read of a stale element, any

@@ -70,6 +70,57 @@ int mk_host_plan_simulate(const mk_config *cfg, const mk_plan_opts *opts, int32_
                           int32_t steps, uint64_t seed, int32_t timeout_ms, char *err,
                           size_t err_len);
 
+/*
+ * Cost model of a plan (no GPU).  After the "One Megakernel is Not Enough"
+ * digest: section 2.2 (a service table of operator times that scale with the
+ * CTA waves ceil(g / W) of the CTAs an operator gets) and section 2.3 (a
+ * region is worth a persistent kernel when its per-step savings S(b) over
+ * conventional launches exceed its fixed cost F).  The plan's instructions
+ * are replayed in their global order: each CTA streams its 16 KiB pages at
+ * its share of the HBM bandwidth into a ring of ring_pages pages; an
+ * instruction starts when its CTA is free and its producers have finished
+ * plus one exchange through global memory, consumes its pages at the compute
+ * rate and ends after a fixed cost; a ticketed attention merge adds two
+ * exchanges and the merge itself to the last split.  The conventional path is
+ * one launch per instruction class and layer, each launch as long as its
+ * slowest CTA from a cold ring, in ceil(g / W) waves.  The default
+ * parameters are this build's measurements on a B200 (see each field).
+ */
+typedef struct {
+  double sm_gbs;          /* bulk-copy bandwidth one SM sustains, GB/s (49) */
+  int32_t ring_pages;     /* 16 KiB ring pages per CTA (12) */
+  double exchange_us;     /* producer's last store -> consumer's loads fresh, under load (1.6) */
+  double page_us;         /* batch 1: compute per 16 KiB weight page (0.13) */
+  double attn_page_us;    /* attention compute per K/V page (0.30) */
+  double attn_fixed_us;   /* attention item: current row, warp merge, stores (0.8) */
+  double merge_us;        /* ticketed merge: the last split's own merge work (0.6) */
+  double instr_us;        /* per matrix instruction: barriers, epilogue, signal (0.25) */
+  double launch_us;       /* conventional path: one launch from a CUDA graph (1.3) */
+  double tc_page_us;      /* batched plans: tensor-core MMAs per weight page (0.20) */
+  double cc_page_us_seq;  /* batched plans on CUDA cores: per weight page and sequence (0.12) */
+  int32_t conv_ctas;      /* CTAs the conventional path gets, W (0: the plan's) */
+} mk_cost_params;
+
+typedef struct {
+  double step_us;         /* the megakernel step */
+  double per_op_us;       /* the conventional path: one launch per instruction class and layer */
+  double hbm_floor_us;    /* the plan's weight and K/V pages at every SM's bandwidth */
+  double savings_us;      /* S(b) = per_op_us - step_us */
+  double stage_us[7];     /* per opcode (index = mk_instr_desc.op): mean instruction time */
+} mk_cost_estimate;
+
+/* The default parameters (host, filled in). */
+void mk_cost_params_default(mk_cost_params *params);
+
+/*
+ * mk_host_plan_estimate: the plan mk_plan would build for cfg / opts on
+ * num_ctas CTAs (static queues only), replayed with the sequences at position
+ * `context`.  params NULL = defaults.  Errors: MK_ERR_INVALID_ARG (bad
+ * arguments, dynamic queue; message in err), MK_ERR_UNSUPPORTED_SHAPE.
+ */
+int mk_host_plan_estimate(const mk_config *cfg, const mk_plan_opts *opts, int32_t num_ctas, int32_t context,
+                          const mk_cost_params *params, mk_cost_estimate *out, char *err, size_t err_len);
+
 #ifdef __cplusplus
 }
 #endif
