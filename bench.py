@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--workload", default="llama1b")
     ap.add_argument("--exec-mode", default="megakernel",
                     choices=["megakernel", "megakernel_generic", "per_op", "per_op_graph"])
-    ap.add_argument("--sched", default="static", choices=["static", "dynamic"])
+    ap.add_argument("--sched", default="static", choices=["static", "dynamic", "event"])
     ap.add_argument("--kv-splits", type=int, default=0)
     ap.add_argument("--l2-prefetch-kb", type=int, default=0)
     ap.add_argument("--inflight", type=int, default=0, help="bulk-copy pages in flight per CTA (0 = default)")
@@ -469,7 +469,8 @@ def main():
                                                                        "sched": args.sched}}}
         Kc = max(1, min(K, args.compare_steps))
         for label, over in (("per_op", dict(exec_mode="per_op")), ("per_op_graph", dict(exec_mode="per_op_graph")),
-                            ("dynamic_queue", dict(sched="dynamic", exec_mode="megakernel"))):
+                            ("dynamic_queue", dict(sched="dynamic", exec_mode="megakernel")),
+                            ("event_queue", dict(sched="event", exec_mode="megakernel"))):
             kw = {**plan_kw, **over}
             if kw == plan_kw:
                 continue

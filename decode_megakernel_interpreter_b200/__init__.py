@@ -26,7 +26,7 @@ MK_ERR_TIMEOUT = -6
 MK_ERR_DEVICE_INPUT = -7
 MK_ERR_OUT_OF_MEMORY = -8
 
-MK_SCHED_STATIC, MK_SCHED_DYNAMIC = 0, 1
+MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_SCHED_EVENT = 0, 1, 2
 MK_EXEC_MEGAKERNEL, MK_EXEC_PER_OP, MK_EXEC_PER_OP_GRAPH, MK_EXEC_MEGAKERNEL_GENERIC = 0, 1, 2, 3
 MK_TRACE_WORDS = 10
 
@@ -73,7 +73,7 @@ class mk_plan_info(ctypes.Structure):
                 ("num_pages", ctypes.c_int32), ("num_instructions", ctypes.c_int32),
                 ("num_counters", ctypes.c_int32), ("kv_splits", ctypes.c_int32), ("max_queue_len", ctypes.c_int32),
                 ("weight_bytes_per_step", ctypes.c_int64), ("kernel_variant", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("estimated_step_us", ctypes.c_int32)]
 
 
 class mk_instr_desc(ctypes.Structure):
@@ -87,7 +87,8 @@ class mk_cost_params(ctypes.Structure):
     _fields_ = [("sm_gbs", ctypes.c_double), ("ring_pages", ctypes.c_int32), ("exchange_us", ctypes.c_double),
                 ("page_us", ctypes.c_double), ("attn_page_us", ctypes.c_double), ("attn_fixed_us", ctypes.c_double),
                 ("merge_us", ctypes.c_double), ("instr_us", ctypes.c_double), ("launch_us", ctypes.c_double),
-                ("tc_page_us", ctypes.c_double), ("cc_page_us_seq", ctypes.c_double), ("conv_ctas", ctypes.c_int32)]
+                ("tc_page_us", ctypes.c_double), ("cc_page_us_seq", ctypes.c_double), ("conv_ctas", ctypes.c_int32),
+                ("merge_split_us", ctypes.c_double)]
 
 
 class mk_cost_estimate(ctypes.Structure):
@@ -272,7 +273,7 @@ def plan_opts(batch: int = 1, kv_splits: int = 0, sched: str = "static", exec_mo
               num_sms: int = 0, trace: bool = False, wait_timeout_ns: int = 0, l2_prefetch_kb: int = 0,
               debug_drop_producer: bool = False, max_inflight_pages: int = 0,
               tensor_qkv_o: bool = False, use_tcgen05: int = 0) -> mk_plan_opts:
-    return mk_plan_opts(batch, kv_splits, {"static": 0, "dynamic": 1}[sched],
+    return mk_plan_opts(batch, kv_splits, {"static": 0, "dynamic": 1, "event": 2}[sched],
                         {"megakernel": 0, "per_op": 1, "per_op_graph": 2, "megakernel_generic": 3}[exec_mode], num_sms, int(trace),
                         wait_timeout_ns, l2_prefetch_kb, int(debug_drop_producer), max_inflight_pages,
                         int(tensor_qkv_o), int(use_tcgen05))

@@ -50,6 +50,7 @@ struct mk_handle {
   int smem = 0, grid = 0, nb = 1;
   const void *kernel = nullptr;  // the interpreter build this plan launches
   int kernel_variant = 0;        // 1: specialised for this model's shape
+  int est_step_us = 0;           // the plan cost model's step estimate at max_seq (0: dynamic queue)
   int last_detail[6] = {0, 0, 0, 0, 0, 0};
   // per-op graph mode
   cudaGraphExec_t gexec = nullptr;
@@ -321,13 +322,15 @@ PlanRequest make_request(const mk_config &c, const mk_plan_opts &o, int num_ctas
   r.B = o.batch;
   r.S = o.kv_splits;
   r.num_ctas = num_ctas;
-  r.dynamic = o.sched_mode == MK_SCHED_DYNAMIC;
+  r.dynamic = o.sched_mode == MK_SCHED_DYNAMIC || o.sched_mode == MK_SCHED_EVENT;
+  r.events = o.sched_mode == MK_SCHED_EVENT;
   r.assumed_context = std::max(1, c.max_seq);
   r.drop_producer = o.debug_drop_producer != 0;
-  // batched plans run gate/up, down and the LM head on the tensor cores
-  // unless asked not to
-  r.tensor = o.batch > 1 && o.use_tcgen05 >= 0;
   r.tensor_qkv_o = o.tensor_qkv_o != 0;
+  // batched plans: gate/up, down and the LM head on the tensor cores when
+  // asked (1), or automatically (0) when the plan cost model expects them to
+  // beat the CUDA cores at this batch
+  r.tensor = o.batch > 1 && (o.use_tcgen05 > 0 || (o.use_tcgen05 == 0 && cost_prefers_tensor(r, CostParams())));
   return r;
 }
 
@@ -468,15 +471,25 @@ static void drop_plan(mk_handle *h) {
   h->planned = false;
 }
 
+// The plan cost model's estimate of a step with every sequence at max_seq,
+// rounded to whole microseconds (0 for the dynamic queue, which the model
+// does not replay).
+static int plan_estimate_us(const PlanRequest &req, const Plan &p) {
+  if (p.dynamic) return 0;
+  CostEstimate e;
+  if (!estimate_plan(req, p, CostParams(), std::max(0, req.assumed_context - 1), &e).empty()) return 0;
+  return (int)std::lround(e.step_us);
+}
+
 extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   if (!h) return MK_ERR_INVALID_ARG;
   mk_plan_opts o = opts_in ? *opts_in : default_opts(h->cfg);
   if (o.batch < 1 || o.batch > h->cfg.max_batch) return MK_ERR_INVALID_ARG;
-  if (o.sched_mode != MK_SCHED_STATIC && o.sched_mode != MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
+  if (o.sched_mode < MK_SCHED_STATIC || o.sched_mode > MK_SCHED_EVENT) return MK_ERR_INVALID_ARG;
   if (o.exec_mode < MK_EXEC_MEGAKERNEL || o.exec_mode > MK_EXEC_MEGAKERNEL_GENERIC) return MK_ERR_INVALID_ARG;
   const bool one_launch = o.exec_mode == MK_EXEC_MEGAKERNEL || o.exec_mode == MK_EXEC_MEGAKERNEL_GENERIC;
-  if (!one_launch && o.sched_mode == MK_SCHED_DYNAMIC) return MK_ERR_INVALID_ARG;
-  if (o.kv_splits < 0 || o.num_sms < 0 || o.wait_timeout_ns < 0) return MK_ERR_INVALID_ARG;
+  if (!one_launch && o.sched_mode != MK_SCHED_STATIC) return MK_ERR_INVALID_ARG;
+  if (o.kv_splits < kSplitsByCost || o.num_sms < 0 || o.wait_timeout_ns < 0) return MK_ERR_INVALID_ARG;
   if (!tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
   cudaError_t ce = cudaDeviceSynchronize();
   if (ce != cudaSuccess) {
@@ -551,6 +564,30 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   if ((rc = dalloc(h->plan_allocs, &q_off, (size_t)num_ctas, false))) return rc;
   if ((rc = dalloc(h->plan_allocs, &q_len, (size_t)num_ctas, false))) return rc;
   if (o.trace && (rc = dalloc(h->plan_allocs, &trace, p.instrs.size() * MK_TRACE_WORDS))) return rc;
+  // event-driven plans: the counters' dependent lists and the ready queue
+  // (zeroed: no slot carries a step number >= 1 until a producer fills it)
+  int *ev_off = nullptr, *ev_list = nullptr, *ev_init = nullptr;
+  unsigned *ev_cnt = nullptr;
+  unsigned long long *ev_ready = nullptr;
+  const int n_ev = (int)(p.ev_init.size() + p.ev_list.size());
+  if (p.events) {
+    if ((rc = dalloc(h->plan_allocs, &ev_off, p.ev_off.size(), false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &ev_list, std::max<size_t>(1, p.ev_list.size()), false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &ev_init, std::max<size_t>(1, p.ev_init.size()), false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &ev_cnt, p.ev_cnt.size(), false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &ev_ready, (size_t)std::max(1, n_ev)))) return rc;
+    e = cudaMemcpy(ev_off, p.ev_off.data(), sizeof(int) * p.ev_off.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !p.ev_list.empty())
+      e = cudaMemcpy(ev_list, p.ev_list.data(), sizeof(int) * p.ev_list.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !p.ev_init.empty())
+      e = cudaMemcpy(ev_init, p.ev_init.data(), sizeof(int) * p.ev_init.size(), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = cudaMemcpy(ev_cnt, p.ev_cnt.data(), sizeof(unsigned) * p.ev_cnt.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
+  }
   e = cudaMemcpy(instrs, p.instrs.data(), p.instrs.size() * sizeof(Instr), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(q_off, p.q_off.data(), sizeof(int) * num_ctas, cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemcpy(q_len, p.q_len.data(), sizeof(int) * num_ctas, cudaMemcpyHostToDevice);
@@ -674,7 +711,15 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   }
   k.timeout_ns = o.wait_timeout_ns > 0 ? o.wait_timeout_ns : 1000000000LL;
   k.trace = trace;
-  k.mode = (o.trace ? MODE_TRACE : 0u) | (o.sched_mode == MK_SCHED_DYNAMIC ? MODE_DYNAMIC : 0u);
+  k.mode = (o.trace ? MODE_TRACE : 0u) | (p.dynamic ? MODE_DYNAMIC : 0u) | (p.events ? MODE_EVENT : 0u);
+  k.ev_tail = p.ev_tail;
+  k.n_ev = n_ev;
+  k.n_ev_init = (int)p.ev_init.size();
+  k.ev_off = ev_off;
+  k.ev_list = ev_list;
+  k.ev_init = ev_init;
+  k.ev_cnt = ev_cnt;
+  k.ev_ready = ev_ready;
   k.stage_filter = -1;
   h->plan = std::move(p);
   h->opts = o;
@@ -683,6 +728,7 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   h->nb = nb;
   h->kernel = kernel;
   h->kernel_variant = variant;
+  h->est_step_us = plan_estimate_us(req, h->plan);
   h->planned = true;
   return MK_OK;
 }
@@ -823,7 +869,7 @@ extern "C" int mk_get_plan_info(const mk_handle *h, mk_plan_info *info) {
   info->max_queue_len = mx;
   info->weight_bytes_per_step = h->plan.weight_bytes;
   info->kernel_variant = h->kernel_variant;
-  info->reserved = 0;
+  info->estimated_step_us = h->est_step_us;
   return MK_OK;
 }
 
@@ -851,7 +897,9 @@ extern "C" int mk_host_plan(const mk_config *cfg, const mk_plan_opts *opts, int3
   }
   if (num_ctas < 1) return MK_ERR_INVALID_ARG;
   mk_plan_opts o = opts ? *opts : default_opts(*cfg);
-  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
+  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o) || o.kv_splits < kSplitsByCost ||
+      o.sched_mode < MK_SCHED_STATIC || o.sched_mode > MK_SCHED_EVENT)
+    return MK_ERR_INVALID_ARG;
   PlanRequest req = make_request(*cfg, o, num_ctas);
   Plan p;
   std::string e = build_plan(req, &p);
@@ -880,6 +928,7 @@ extern "C" int mk_host_plan(const mk_config *cfg, const mk_plan_opts *opts, int3
     for (int l : p.q_len) mx = std::max(mx, l);
     info->max_queue_len = mx;
     info->weight_bytes_per_step = p.weight_bytes;
+    info->estimated_step_us = plan_estimate_us(req, p);
   }
   return MK_OK;
 }
@@ -894,7 +943,9 @@ extern "C" int mk_host_plan_simulate(const mk_config *cfg, const mk_plan_opts *o
   }
   if (num_ctas < 1 || steps < 1 || timeout_ms < 1) return MK_ERR_INVALID_ARG;
   mk_plan_opts o = opts ? *opts : default_opts(*cfg);
-  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
+  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o) || o.kv_splits < kSplitsByCost ||
+      o.sched_mode < MK_SCHED_STATIC || o.sched_mode > MK_SCHED_EVENT)
+    return MK_ERR_INVALID_ARG;
   PlanRequest req = make_request(*cfg, o, num_ctas);
   Plan p;
   std::string e = build_plan(req, &p);
@@ -924,6 +975,7 @@ static CostParams cost_params_from(const mk_cost_params *q) {
   c.tc_page_us = q->tc_page_us;
   c.cc_page_us_seq = q->cc_page_us_seq;
   c.conv_ctas = q->conv_ctas;
+  c.merge_split_us = q->merge_split_us;
   return c;
 }
 
@@ -942,6 +994,7 @@ extern "C" void mk_cost_params_default(mk_cost_params *q) {
   q->tc_page_us = c.tc_page_us;
   q->cc_page_us_seq = c.cc_page_us_seq;
   q->conv_ctas = c.conv_ctas;
+  q->merge_split_us = c.merge_split_us;
 }
 
 extern "C" int mk_host_plan_estimate(const mk_config *cfg, const mk_plan_opts *opts, int32_t num_ctas,
@@ -955,7 +1008,9 @@ extern "C" int mk_host_plan_estimate(const mk_config *cfg, const mk_plan_opts *o
   }
   if (num_ctas < 1 || context < 0 || context >= cfg->max_seq || !out) return MK_ERR_INVALID_ARG;
   mk_plan_opts o = opts ? *opts : default_opts(*cfg);
-  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o)) return MK_ERR_INVALID_ARG;
+  if (o.batch < 1 || o.batch > cfg->max_batch || !tensor_opts_ok(o) || o.kv_splits < kSplitsByCost ||
+      o.sched_mode < MK_SCHED_STATIC || o.sched_mode > MK_SCHED_EVENT)
+    return MK_ERR_INVALID_ARG;
   PlanRequest req = make_request(*cfg, o, num_ctas);
   Plan p;
   std::string e = build_plan(req, &p);

@@ -182,6 +182,9 @@ __device__ __forceinline__ void st_ll(llw *a, float v, uint32_t tag) {
   const llw w = ((llw)tag << 32) | __float_as_uint(v);
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(w) : "memory");
 }
+__device__ __forceinline__ void st_u64(unsigned long long *a, unsigned long long w) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(a), "l"(w) : "memory");
+}
 __device__ __forceinline__ llw ld_ll(const llw *a) {
   llw w;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(a));
@@ -610,7 +613,9 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
   uint32_t g = 0;
   bool ok = true;
   const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
-  const unsigned dyn_base = dyn ? (epoch - 1u) * (unsigned)(p.n_instr + gridDim.x) : 0u;
+  const bool ev = dyn && (p.mode & MODE_EVENT) != 0;
+  // claims per step: every queue entry plus one past the end per CTA
+  const unsigned dyn_base = dyn ? (epoch - 1u) * (unsigned)((ev ? p.n_ev : p.n_instr) + gridDim.x) : 0u;
   int claimed = 0;
   const bool use_pf = !RAW && !dyn && p.pf_pages > 0;
   PfCursor pf;
@@ -620,6 +625,31 @@ __device__ void run_loader(const KParams &p, Shared *sh, uint8_t *pages, uint64_
     if (dyn) {
       // claim the next instruction of the global queue; publish it to the compute warps
       unsigned k = atomicAdd(p.ctr + p.dyn_head, 1u) - dyn_base;
+      if (ev) {
+        // event-driven queue: claim k is ready slot k (the first n_ev_init
+        // are the instructions that wait on nothing); a slot past those is
+        // filled by the producer that completes a dependency count
+        if (k >= (unsigned)p.n_ev) {
+          k = (unsigned)p.n_instr;  // past the end: this loader is done
+        } else if (k < (unsigned)p.n_ev_init) {
+          k = (unsigned)p.ev_init[k];
+        } else {
+          const uint64_t tw = px::gtimer();
+          unsigned long long w;
+          for (unsigned it = 1;; ++it) {
+            w = px::ld_ll(p.ev_ready + k);
+            if ((uint32_t)(w >> 32) == epoch) break;
+            if ((it & 31u) == 0 &&
+                (px::ld_volatile(&sh->abort) || global_abort(p) || px::gtimer() - tw > (uint64_t)p.timeout_ns)) {
+              if (!global_abort(p)) record_error(p, MK_ERR_TIMEOUT, -4, (int)k, (int)(w >> 32), (int)epoch);
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+          k = (unsigned)(w & 0xffffffffu);
+        }
+      }
       int slot = claimed & 31;
       const uint64_t t0 = px::gtimer();
       while (claimed - *dyn_head >= 32) {  // FIFO space (bounded)
@@ -2545,6 +2575,27 @@ using SpecGeneric = Spec<0, 0, 0, 0, 0>;
 #endif
 constexpr unsigned kSpeculativeOps = MK_SPECULATIVE_OPS;
 
+// Event-driven queue: signal counter c; the signal that completes the
+// step's count appends the instructions waiting on it to the ready queue
+// (slot = step << 32 | instruction index).  Thread 0 of the producer.
+__device__ __noinline__ void event_signal(const KParams &p, unsigned c, unsigned epoch) {
+  const unsigned old = px::atom_relaxed_add(p.ctr + c, 1u);
+  const unsigned cnt = p.ev_cnt[c];
+  if (cnt == 0 || old + 1u != epoch * cnt) return;
+  const int j0 = p.ev_off[c], n = p.ev_off[c + 1] - j0;
+  const unsigned per_step = (unsigned)(p.n_ev - p.n_ev_init);
+  const unsigned pos = px::atom_relaxed_add(p.ctr + p.ev_tail, (unsigned)n) - (epoch - 1u) * per_step +
+                       (unsigned)p.n_ev_init;
+  for (int j = 0; j < n; ++j) {
+    if (pos + (unsigned)j >= (unsigned)p.n_ev) {
+      record_error(p, MK_ERR_TIMEOUT, -5, (int)c, (int)pos, j);
+      return;
+    }
+    px::st_u64(p.ev_ready + pos + j, ((unsigned long long)epoch << 32) | (unsigned)p.ev_list[j0 + j]);
+  }
+}
+
+
 template <int NB, class S>
 __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile int *dyn_tail,
                             volatile int *dyn_head) {
@@ -2676,7 +2727,11 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
     const bool sig = I.sig_ctr != kNoCounter && (I.op != OP_ATTN || c.sh->flag);
     if (c.ctid == 0 && sig) {
       // a hint only: the data words carry this step's tag, so no fence
-      for (int k = 0; k < I.sig_n; ++k) px::red_relaxed_add(p.ctr + I.sig_ctr + k, 1u);
+      if (p.mode & MODE_EVENT) {
+        for (int k = 0; k < I.sig_n; ++k) event_signal(p, I.sig_ctr + k, c.epoch);
+      } else {
+        for (int k = 0; k < I.sig_n; ++k) px::red_relaxed_add(p.ctr + I.sig_ctr + k, 1u);
+      }
     }
     if (tr && c.ctid == 0) {
       tr[4] = px::gtimer();

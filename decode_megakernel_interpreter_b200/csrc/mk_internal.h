@@ -89,6 +89,7 @@ enum : uint32_t {
   MODE_TRACE = 2u,
   MODE_DYNAMIC = 4u,      // one global queue claimed with an atomic
   MODE_FINAL_LAUNCH = 8u, // this launch ends the step (advances the epoch)
+  MODE_EVENT = 16u,       // with MODE_DYNAMIC: the global queue holds ready instructions only
 };
 
 // Status words (device): [0] first error code, [1] abort flag, [2..7] detail.
@@ -139,6 +140,15 @@ struct KParams {
   unsigned arg_ticket0;   // index of the first argmax ticket [B]
   unsigned exit_ticket;   // index of the exit ticket
   unsigned dyn_head;      // index of the dynamic-queue head counter
+  // event-driven queue (MODE_EVENT): claims k < n_ev_init take ev_init[k];
+  // later claims wait for ready slot k, which the last producer of a counter
+  // fills (step << 32 | instruction index) with the counter's dependents
+  // ev_list[ev_off[c] .. ev_off[c+1]) once it reaches epoch * ev_cnt[c]
+  unsigned ev_tail;       // index of the ready-queue tail counter
+  int n_ev, n_ev_init;    // claimable instructions per step, of which ready at the start
+  const int *ev_off, *ev_list, *ev_init;
+  const unsigned *ev_cnt;
+  unsigned long long *ev_ready;  // [n_ev]
   // plan
   const Instr *instrs;    // all instructions; static: per-CTA contiguous queues
   const int *q_off, *q_len;

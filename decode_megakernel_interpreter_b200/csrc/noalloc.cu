@@ -118,9 +118,9 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   PlanRequest req;
   req.s = s;
   req.B = 1;
-  req.S = 0;
   req.num_ctas = slot->sm_count;
   req.assumed_context = cfg->max_seq;
+  req.S = 0;
   Plan p;
   if (!build_plan(req, &p).empty()) return MK_ERR_UNSUPPORTED_SHAPE;
 

@@ -81,6 +81,67 @@ struct Pending {
 
 }  // namespace
 
+// The fixed rule: one attention item per CTA, but at least ~32 positions per
+// split; when the sequences alone fill the CTAs (batched plans), still split
+// long contexts up to ~4 items per CTA with >= 256 positions each, so that the
+// longest sequence does not run on one CTA alone.
+int rule_kv_splits(const PlanRequest &req) {
+  const int items = req.B * req.s.nkv;
+  int S = std::max(1, req.num_ctas / items);
+  S = std::min(S, std::max(1, req.assumed_context / 32));
+  if (req.B > 1) S = std::max(S, std::min(4 * req.num_ctas / items, req.assumed_context / 256));
+  return std::max(1, std::min(S, 64));
+}
+
+// The cost model's choice: the candidate split count whose plan has the least
+// estimated step with every sequence at the assumed context (a dynamic plan is
+// estimated through its static twin).  Candidates keep >= ~32 positions per
+// split; a tie keeps the smaller count.
+int cost_kv_splits(const PlanRequest &req, const CostParams &c, double *best_us) {
+  static const int kCand[] = {1, 2, 3, 4, 6, 8, 9, 12, 16, 18, 24, 32, 36, 48, 64};
+  PlanRequest r = req;
+  r.dynamic = false;
+  const int max_s = std::max(1, std::min(64, req.assumed_context / 32));
+  const int ctx = std::max(0, req.assumed_context - 1);
+  int best = 0;
+  double best_t = 0.0;
+  for (int S : kCand) {
+    if (S > max_s) break;
+    r.S = S;
+    Plan p;
+    CostEstimate e;
+    if (!build_plan(r, &p).empty() || !estimate_plan(r, p, c, ctx, &e).empty()) continue;
+    if (best == 0 || e.step_us < best_t) {
+      best = S;
+      best_t = e.step_us;
+    }
+  }
+  if (best == 0) return rule_kv_splits(req);
+  if (best_us) *best_us = best_t;
+  return best;
+}
+
+// The cost model's choice between the tensor-core and the CUDA-core matrix
+// instructions of a batched request (each at its own split count when the
+// request leaves that open).  A request for tensor-core QKV / O tiles keeps
+// the tensor cores.
+bool cost_prefers_tensor(const PlanRequest &req, const CostParams &c) {
+  if (req.B <= 1) return false;
+  if (req.tensor_qkv_o) return true;
+  const int ctx = std::max(0, req.assumed_context - 1);
+  double t[2] = {0.0, 0.0};
+  for (int k = 0; k < 2; ++k) {
+    PlanRequest r = req;
+    r.dynamic = false;
+    r.tensor = k == 0;
+    Plan p;
+    CostEstimate e;
+    if (!build_plan(r, &p).empty() || !estimate_plan(r, p, c, ctx, &e).empty()) return k != 0;
+    t[k] = e.step_us;
+  }
+  return t[0] <= t[1];
+}
+
 std::string build_plan(const PlanRequest &req, Plan *out) {
   const Shape &s = req.s;
   std::string err = check_shape(s, req.B);
@@ -97,16 +158,10 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   const int G = s.nq / s.nkv;
   if (req.S > 0) {
     p.S = std::min(req.S, 256);
+  } else if (req.S == kSplitsByCost) {
+    p.S = cost_kv_splits(req, CostParams(), nullptr);
   } else {
-    // one attention item per CTA, but keep at least ~32 positions per split;
-    // when the sequences alone fill the CTAs (batched plans), still split
-    // long contexts up to ~4 items per CTA with >= 256 positions each, so
-    // that the longest sequence does not run on one CTA alone
-    int items = req.B * s.nkv;
-    int S = std::max(1, req.num_ctas / items);
-    S = std::min(S, std::max(1, req.assumed_context / 32));
-    if (req.B > 1) S = std::max(S, std::min(4 * req.num_ctas / items, req.assumed_context / 256));
-    p.S = std::max(1, std::min(S, 64));
+    p.S = rule_kv_splits(req);
   }
   p.P_qkv = (s.nq + 2 * s.nkv) * s.d / p.Rh;
   p.P_o = s.H / p.Ro;
@@ -121,6 +176,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   next += (unsigned)req.B;
   p.exit_ticket = next++;
   p.dyn_head = next++;
+  p.ev_tail = next++;
   p.n_counters = (int)next;
 
   const int n = req.num_ctas;
@@ -296,6 +352,31 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
     for (auto &x : all) p.instrs.push_back(x.ins);
     p.q_off.assign(n, 0);
     p.q_len.assign(n, 0);
+    if (req.events) {
+      // event tables: dependents of every counter, grouped by counter in
+      // topological order, and the instructions that wait on nothing
+      p.events = true;
+      p.ev_off.assign(p.n_counters + 1, 0);
+      p.ev_cnt.assign(p.n_counters, 0);
+      for (const Instr &I : p.instrs) {
+        if (I.op == OP_NOP) continue;
+        if (I.wait_ctr == kNoCounter) continue;
+        if (I.wait_ctr >= (unsigned)p.n_counters) return "event plan: bad counter";
+        if (p.ev_cnt[I.wait_ctr] != 0 && p.ev_cnt[I.wait_ctr] != I.wait_cnt)
+          return "event plan: dependents of one counter wait for different counts";
+        p.ev_cnt[I.wait_ctr] = I.wait_cnt;
+        p.ev_off[I.wait_ctr + 1]++;
+      }
+      for (int c = 0; c < p.n_counters; ++c) p.ev_off[c + 1] += p.ev_off[c];
+      p.ev_list.assign(p.ev_off[p.n_counters], 0);
+      std::vector<int> fill(p.ev_off.begin(), p.ev_off.end() - 1);
+      for (int k = 0; k < (int)p.instrs.size(); ++k) {
+        const Instr &I = p.instrs[k];
+        if (I.op == OP_NOP) continue;
+        if (I.wait_ctr == kNoCounter) p.ev_init.push_back(k);
+        else p.ev_list[fill[I.wait_ctr]++] = k;
+      }
+    }
   } else {
     std::vector<std::vector<Instr>> q(n);
     std::vector<int64_t> load(n, 0);
@@ -538,8 +619,19 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
     if (!failed.exchange(true)) err = m;
   };
 
+  // event-driven plans: the ready queue (instruction index and the step
+  // that appended it, per slot)
+  const int n_init = (int)p.ev_init.size();
+  const int n_ev = n_init + (int)p.ev_list.size();
+  std::unique_ptr<std::atomic<uint32_t>[]> ready_step(new std::atomic<uint32_t>[n_ev > 0 ? n_ev : 1]);
+  std::unique_ptr<std::atomic<int>[]> ready_id(new std::atomic<int>[n_ev > 0 ? n_ev : 1]);
+  for (int i = 0; i < n_ev; ++i) {
+    ready_step[i].store(0);
+    ready_id[i].store(-1);
+  }
   for (uint32_t epoch = 1; epoch <= (uint32_t)steps && !failed; ++epoch) {
     std::atomic<uint32_t> dyn_next{0};
+    std::atomic<uint32_t> ev_tail{(uint32_t)n_init};
     auto run_cta = [&](int cta) {
       std::mt19937_64 rng(seed * 1000003ull + cta * 7919ull + epoch);
       std::uniform_int_distribution<int> jitter(0, 9);
@@ -574,7 +666,37 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
       int qi = 0;
       while (!failed) {
         const Instr *I;
-        if (p.dynamic) {
+        if (p.events) {
+          // the next ready instruction: the initial ones, then the slots the
+          // producers' events append (wait until this slot is filled)
+          const uint32_t k = dyn_next.fetch_add(1);
+          if (k >= (uint32_t)n_ev) break;
+          int id;
+          if ((int)k < n_init) {
+            id = p.ev_init[k];
+          } else {
+            auto t0 = std::chrono::steady_clock::now();
+            while (ready_step[k].load(std::memory_order_acquire) != epoch) {
+              if (failed) return;
+              std::this_thread::yield();
+              if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(timeout_ms)) {
+                char b[256];
+                snprintf(b, sizeof b, "step %u: ready-queue slot %u never filled", epoch, k);
+                fail(b);
+                return;
+              }
+            }
+            id = ready_id[k].load(std::memory_order_relaxed);
+          }
+          I = &p.instrs[id];
+          if (I->wait_ctr != kNoCounter &&
+              ctr[I->wait_ctr].load(std::memory_order_acquire) < (uint64_t)epoch * I->wait_cnt) {
+            char b[256];
+            snprintf(b, sizeof b, "step %u: instruction %d became ready before its producers finished", epoch, I->seq);
+            fail(b);
+            return;
+          }
+        } else if (p.dynamic) {
           uint32_t k = dyn_next.fetch_add(1);
           if (k >= p.instrs.size()) break;
           I = &p.instrs[k];
@@ -618,7 +740,23 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
           }
         }
         if (signal && I->sig_ctr != kNoCounter)
-          for (int k = 0; k < I->sig_n; ++k) ctr[I->sig_ctr + k].fetch_add(1, std::memory_order_release);
+          for (int k = 0; k < I->sig_n; ++k) {
+            const unsigned c = I->sig_ctr + k;
+            const uint32_t old = ctr[c].fetch_add(1, std::memory_order_acq_rel);
+            if (p.events && p.ev_cnt[c] != 0 && old + 1 == epoch * p.ev_cnt[c]) {
+              // the last producer: its dependents become ready
+              const int n = p.ev_off[c + 1] - p.ev_off[c];
+              const uint32_t pos = ev_tail.fetch_add((uint32_t)n);
+              for (int j = 0; j < n; ++j) {
+                if (pos + j >= (uint32_t)n_ev) {
+                  fail("ready queue overflow");
+                  return;
+                }
+                ready_id[pos + j].store(p.ev_list[p.ev_off[c] + j], std::memory_order_relaxed);
+                ready_step[pos + j].store(epoch, std::memory_order_release);
+              }
+            }
+          }
       }
     };
     std::vector<std::thread> th;
@@ -683,6 +821,7 @@ std::string estimate_plan(const PlanRequest &req, const Plan &p, const CostParam
                           CostEstimate *out) {
   if (p.dynamic) return "the cost model replays static queues";
   if (context < 0 || c.sm_gbs <= 0 || c.ring_pages < 1) return "bad cost parameters";
+  if ((int)p.q_off.size() != p.num_ctas || (int)p.q_len.size() != p.num_ctas || p.num_ctas < 1) return "not a plan";
   const Shape &s = req.s;
   const int n = p.num_ctas;
   const double t_hbm = kPageBytes / (c.sm_gbs * 1e3);  // us per 16 KiB page at one SM's bandwidth
@@ -739,7 +878,7 @@ std::string estimate_plan(const PlanRequest &req, const Plan &p, const CostParam
       group_max[gi] = std::max(group_max[gi], finish);
       // the last split of the group merges: the ticket and the reload of the
       // partials are two exchanges
-      const double merged = group_max[gi] + 2 * c.exchange_us + c.merge_us;
+      const double merged = group_max[gi] + 2 * c.exchange_us + c.merge_us + p.S * c.merge_split_us;
       for (int k = 0; k < I.sig_n; ++k) ctr_done[I.sig_ctr + k] = std::max(ctr_done[I.sig_ctr + k], merged);
     } else if (I.sig_ctr != kNoCounter) {
       for (int k = 0; k < I.sig_n; ++k) ctr_done[I.sig_ctr + k] = std::max(ctr_done[I.sig_ctr + k], finish);
@@ -767,7 +906,7 @@ std::string estimate_plan(const PlanRequest &req, const Plan &p, const CostParam
     // ones overlap compute
     const double t = np > 0 ? t_hbm + (np - 1) * std::max(t_hbm, pt) + pt : 0.0;
     per_cta[st][cta_of[I.seq]] += t + (kv ? c.attn_fixed_us : c.instr_us);
-    if (I.op == OP_ATTN) merge_extra[st] = 2 * c.exchange_us + c.merge_us;
+    if (I.op == OP_ATTN) merge_extra[st] = 2 * c.exchange_us + c.merge_us + p.S * c.merge_split_us;
   }
   // CTA waves: a launch whose work sits on g CTAs runs in ceil(g / W) waves
   // on W available CTAs

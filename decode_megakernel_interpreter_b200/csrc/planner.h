@@ -16,13 +16,19 @@ struct Shape {
   int L, H, nq, nkv, d, F, V;
 };
 
+constexpr int kSplitsByCost = -1;
+
 struct PlanRequest {
   Shape s;
   int B = 1;          // batch
-  int S = 0;          // kv splits (0 = automatic)
+  int S = 0;          // kv splits (0: the fixed rule; kSplitsByCost: the cost model's choice)
   int num_ctas = 148;
   bool dynamic = false;
   int dyn_chunks_per_cta = 2;  // dynamic mode: instructions per CTA per matvec stage
+  // with `dynamic`: the global queue holds only ready instructions -- an
+  // instruction is appended when the last of its producers signals (the
+  // event-driven mode); without it the queue is the fixed topological order
+  bool events = false;
   int assumed_context = 1024;  // for the automatic split count
   bool drop_producer = false;  // test hook (see mk_plan_opts)
   // tensor cores (batched plans): gate/up, down and LM-head instructions
@@ -47,10 +53,17 @@ struct Plan {
   std::vector<int> q_off, q_len;
   int num_ctas = 0;
   bool dynamic = false;
+  // event-driven mode: for counter c, the instructions (indices into instrs)
+  // that wait on it are ev_list[ev_off[c] .. ev_off[c+1]) and become ready
+  // when it reaches epoch * ev_cnt[c]; ev_init lists the instructions that
+  // wait on nothing (ready at the start of every step)
+  bool events = false;
+  std::vector<int> ev_off, ev_list, ev_init;
+  std::vector<unsigned> ev_cnt;
   // counters
   int ctr_per_layer = 0;
   int n_counters = 0;
-  unsigned attn_ticket0 = 0, arg_ticket0 = 0, exit_ticket = 0, dyn_head = 0;
+  unsigned attn_ticket0 = 0, arg_ticket0 = 0, exit_ticket = 0, dyn_head = 0, ev_tail = 0;
   int n_lm = 0;
   int64_t weight_bytes = 0;  // weight bytes streamed per step
 
@@ -89,18 +102,25 @@ std::string validate_plan(const PlanRequest &req, const Plan &p);
 // conventional path is one launch per instruction class and layer whose CTAs
 // run in ceil(items / W) waves with no prefetch across launches.
 struct CostParams {
-  double sm_gbs = 49.0;        // bulk-copy bandwidth one SM sustains (GB/s)
-  int ring_pages = 12;         // 16 KiB pages per CTA ring
-  double exchange_us = 1.6;    // a producer's last store -> a consumer's loads see it (under load)
-  double page_us = 0.13;       // compute time per 16 KiB weight page per sequence group (batch 1)
-  double attn_page_us = 0.30;  // attention compute per K/V page, all warps
-  double attn_fixed_us = 0.8;  // attention: current row, warp merge, partial stores
-  double merge_us = 0.6;       // ticketed merge: the last split's own work besides its two exchanges
-  double instr_us = 0.25;      // per instruction: fetch, barriers, epilogue, signal
-  double launch_us = 1.3;      // conventional path: one kernel launch from a CUDA graph
-  double tc_page_us = 0.20;    // batched plans: tensor-core MMAs of one weight page (16 sequences)
-  double cc_page_us_seq = 0.12;// batched plans on CUDA cores: per weight page and sequence
-  int conv_ctas = 0;           // CTAs the conventional path gets (0: the plan's); fewer -> more waves
+  // Defaults: fitted (least squares on log time) to B200 measurements of this
+  // build -- the Llama-1B shape at contexts 1024 and 8192 with 6 to 72 KV
+  // splits, the Llama-8B shape with 9 to 18, the 1B shape at batch 16 with 1
+  // to 8 splits and with and without tensor cores, and the per-op path
+  // replayed as a CUDA graph (absolute times, and the ratios between the
+  // split counts of one sweep).
+  double sm_gbs = 39.4;         // bulk-copy bandwidth one SM sustains (GB/s)
+  int ring_pages = 12;          // 16 KiB pages per CTA ring
+  double exchange_us = 1.0;     // a producer's last store -> a consumer's loads see it (under load)
+  double page_us = 0.05;        // compute time per 16 KiB weight page per sequence group (batch 1)
+  double attn_page_us = 1.45;   // attention compute per K/V page, all warps
+  double attn_fixed_us = 8.6;   // attention: q loads, current row, warp merge, partial stores, ticket
+  double merge_us = 0.1;        // ticketed merge: the last split's own work besides its two exchanges
+  double instr_us = 0.46;       // per instruction: fetch, barriers, epilogue, signal
+  double launch_us = 26.6;      // conventional path: one launch (cooperative, from a CUDA graph) and its prologue
+  double tc_page_us = 3.56;     // batched plans: tensor-core MMAs of one weight page (16 sequences)
+  double cc_page_us_seq = 0.49; // batched plans on CUDA cores: per weight page and sequence
+  int conv_ctas = 0;            // CTAs the conventional path gets (0: the plan's); fewer -> more waves
+  double merge_split_us = 0.28; // ticketed merge: per split whose partial the last split reloads
 };
 
 struct CostEstimate {
@@ -113,6 +133,15 @@ struct CostEstimate {
 // Estimate a plan (static queues) for sequences at position `context`.
 std::string estimate_plan(const PlanRequest &req, const Plan &p, const CostParams &c, int context,
                           CostEstimate *out);
+
+// Split counts for a request whose S is not fixed: the fixed rule (one
+// attention item per CTA), and the cost model's choice among candidate counts
+// at the request's assumed context (*best_us: its estimate, may be NULL).
+int rule_kv_splits(const PlanRequest &req);
+int cost_kv_splits(const PlanRequest &req, const CostParams &c, double *best_us);
+// Batched requests: whether the cost model expects the tensor-core matrix
+// instructions to beat the CUDA-core ones (false at batch 1).
+bool cost_prefers_tensor(const PlanRequest &req, const CostParams &c);
 
 // Host simulation: `threads` CPU threads play the CTAs and run the queues
 // for `steps` steps under random delays, with real atomic counters and

@@ -119,7 +119,7 @@ int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv,
               mk_handle **out);
 
 /* ------------------------------------------------------------------ plan */
-enum { MK_SCHED_STATIC = 0, MK_SCHED_DYNAMIC = 1 };
+enum { MK_SCHED_STATIC = 0, MK_SCHED_DYNAMIC = 1, MK_SCHED_EVENT = 2 };
 enum {
   MK_EXEC_MEGAKERNEL = 0,        /* one persistent launch per step */
   MK_EXEC_PER_OP = 1,            /* comparison path: one launch per instruction class */
@@ -132,9 +132,18 @@ enum {
 
 typedef struct {
   int32_t batch;          /* sequences per step, 1..max_batch */
-  int32_t kv_splits;      /* split-KV factor of decode attention; 0 = automatic */
-  int32_t sched_mode;     /* MK_SCHED_STATIC (per-SM queues) or MK_SCHED_DYNAMIC
-                             (one global queue claimed with an atomic) */
+  int32_t kv_splits;      /* split-KV factor of decode attention; 0 = automatic
+                             (one attention item per CTA, at least ~32
+                             positions per split); -1 = the count the plan cost
+                             model (mk_host.h) estimates fastest at max_seq */
+  int32_t sched_mode;     /* MK_SCHED_STATIC (per-SM queues), MK_SCHED_DYNAMIC
+                             (one global queue in topological order, claimed
+                             with an atomic), or MK_SCHED_EVENT (one global
+                             queue of ready instructions: the producer whose
+                             signal completes a dependency count appends the
+                             instructions waiting on it -- the event-driven
+                             scheduling of the "Mirage Persistent Kernel"
+                             article, part 2) */
   int32_t exec_mode;      /* MK_EXEC_MEGAKERNEL, or the comparison path:
                              one launch per instruction class (PER_OP), optionally
                              replayed as a CUDA graph (PER_OP_GRAPH), or
@@ -164,8 +173,9 @@ typedef struct {
                              tensor-memory accumulators) for the matrix
                              instructions of batched plans, where a step's
                              matrix-vector products are dense contractions
-                             over the batch: 0 = automatic (on when
-                             batch > 1), 1 = on (MK_ERR_INVALID_ARG at
+                             over the batch: 0 = automatic (batch > 1: on
+                             when the plan cost model expects them to beat
+                             the CUDA cores), 1 = on (MK_ERR_INVALID_ARG at
                              batch 1, where every product is a matrix-vector
                              product and CUDA-core FMAs are used), -1 = off
                              (CUDA cores for every batch) */
@@ -244,14 +254,18 @@ typedef struct {
   int32_t kernel_variant;  /* 0: the shape-generic interpreter build, 1: a build
                               specialised for this model's shape (every op body
                               inlined into the interpreter loop) */
-  int32_t reserved;
+  int32_t estimated_step_us; /* the plan cost model's estimate of one step with
+                              every sequence at max_seq, microseconds (see
+                              mk_host_plan_estimate); 0 for the dynamic queue */
 } mk_plan_info;
 
 /*
  * mk_get_error_detail: the detail words of the last device-side error that
  * mk_get_status returned (host int32 [6]): instruction sequence number (-1:
  * a shared-memory page wait, -2: the final drain, -3: a group of tagged
- * activation loads that never saw this step's tag), counter index or wait kind,
+ * activation loads that never saw this step's tag, -4: an event-driven
+ * ready-queue slot that was never filled, -5: a ready-queue overflow),
+ * counter index or wait kind,
  * observed value, target value, CTA, and the abort flag.  All zero if none.
  */
 int mk_get_error_detail(const mk_handle *h, int32_t detail[6]);

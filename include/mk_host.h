@@ -99,6 +99,7 @@ typedef struct {
   double tc_page_us;      /* batched plans: tensor-core MMAs per weight page (0.20) */
   double cc_page_us_seq;  /* batched plans on CUDA cores: per weight page and sequence (0.12) */
   int32_t conv_ctas;      /* CTAs the conventional path gets, W (0: the plan's) */
+  double merge_split_us;  /* ticketed merge: per split whose partial the last split reloads (0) */
 } mk_cost_params;
 
 typedef struct {

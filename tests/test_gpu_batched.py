@@ -100,7 +100,7 @@ def test_llama1b_batch16_norm_weights(b16_norms, kw):
 def test_llama1b_batch16_modes_agree(b16):
     w, lengths, model = b16
     ref = _run(w, lengths, model, 2, dict(), check_oracle=False)
-    for kw in (dict(exec_mode="per_op"), dict(sched="dynamic")):
+    for kw in (dict(exec_mode="per_op"), dict(sched="dynamic"), dict(sched="event")):
         got = _run(w, lengths, model, 2, kw, check_oracle=False)
         for a, b in zip(ref, got):
             np.testing.assert_array_equal(a, b)

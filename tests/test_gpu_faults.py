@@ -14,7 +14,8 @@ from gpu_common import HostSetup
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("exec_kw", [dict(), dict(sched="dynamic")], ids=["static", "dynamic"])
+@pytest.mark.parametrize("exec_kw", [dict(), dict(sched="dynamic"), dict(sched="event")],
+                         ids=["static", "dynamic", "event"])
 def test_timeout_is_reported_and_engine_recovers(exec_kw):
     s = synth.TINY
     hs = HostSetup(s, 1, 80)

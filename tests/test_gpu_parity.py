@@ -101,10 +101,12 @@ def tiny_setup(model, max_seq=96):
     dict(exec_mode="per_op_graph"),
     dict(exec_mode="megakernel_generic"),
     dict(sched="dynamic"),
+    dict(sched="event"),
+    dict(sched="event", num_sms=3),
     dict(num_sms=3, kv_splits=7),
     dict(num_sms=1, kv_splits=1),
     dict(l2_prefetch_kb=256),
-], ids=["mk", "per_op", "per_op_graph", "mk_generic", "dynamic", "3sm", "1sm", "l2pf"])
+], ids=["mk", "per_op", "per_op_graph", "mk_generic", "dynamic", "event", "event3sm", "3sm", "1sm", "l2pf"])
 def test_tiny_16_steps(tiny_model, kw):
     hs, tok, pos = tiny_setup(tiny_model)
     run_parity(hs, tok, pos, 16, kw)
@@ -115,7 +117,7 @@ def test_schedule_independence_bitwise(tiny_model):
     placement must not change a single bit (fixed kv_splits)."""
     outs = []
     for kw in (dict(kv_splits=4), dict(kv_splits=4, exec_mode="per_op"), dict(kv_splits=4, sched="dynamic"),
-               dict(kv_splits=4, num_sms=5)):
+               dict(kv_splits=4, sched="event"), dict(kv_splits=4, num_sms=5)):
         hs, tok, pos = tiny_setup(tiny_model)
         outs.append(run_parity(hs, tok, pos, 4, kw))
     for o in outs[1:]:

@@ -108,15 +108,43 @@ def test_static_plan_balances_bytes():
         assert len(keys) == len(set(keys))
 
 
-def test_kv_splits_automatic_and_explicit():
-    cfg = cfg_for("llama1b")
-    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1), 148)
-    assert info.kv_splits == 148 // 8
-    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=1, kv_splits=5), 148)
+SPLIT_CANDIDATES = (1, 2, 3, 4, 6, 8, 9, 12, 16, 18, 24, 32, 36, 48, 64)
+
+
+@pytest.mark.parametrize("name", ["llama1b", "llama1b_8k", "llama1b_b16"])
+def test_kv_splits_rule_cost_model_and_explicit(name):
+    """0: the fixed rule (one attention item per CTA); -1: the candidate count
+    with the least cost-model estimate at max_seq (ties: the smaller); > 0:
+    as given.  mk_plan_info reports the model's estimate of the plan."""
+    w = synth.WORKLOADS[name]
+    cfg = cfg_for(name, max_batch=w.batch)
+    B = w.batch
+    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=B), 148)
+    items = B * w.shape.n_kv_heads
+    rule = max(1, min(148 // items, cfg.max_seq // 32))
+    if B > 1:
+        rule = max(rule, min(4 * 148 // items, cfg.max_seq // 256))
+    assert info.kv_splits == max(1, min(rule, 64))
+    est = lambda S: mk.mk_host_plan_estimate(cfg, mk.plan_opts(batch=B, kv_splits=S), 148, cfg.max_seq - 1).step_us
+    assert info.estimated_step_us == round(est(info.kv_splits))
+    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=B, kv_splits=-1), 148)
+    cands = [S for S in SPLIT_CANDIDATES if S <= max(1, min(64, cfg.max_seq // 32))]
+    e = {}
+    for S in cands:
+        try:
+            e[S] = est(S)
+        except mk.MkError:  # a plan too large for one step
+            pass
+    best = min(e, key=lambda S: (e[S], S))
+    assert info.kv_splits == best
+    assert info.estimated_step_us == round(e[best])
+    *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=B, kv_splits=5), 148)
     assert info.kv_splits == 5
+    with pytest.raises(mk.MkError):
+        mk.mk_host_plan(cfg, mk.plan_opts(batch=B, kv_splits=-2), 148)
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "event"])
 @pytest.mark.parametrize("num_ctas", [8, 3, 1])
 def test_simulation_tiny(sched, num_ctas):
     cfg = cfg_for("tiny")
@@ -125,7 +153,7 @@ def test_simulation_tiny(sched, num_ctas):
     assert err == ""
 
 
-@pytest.mark.parametrize("sched", ["static", "dynamic"])
+@pytest.mark.parametrize("sched", ["static", "dynamic", "event"])
 def test_simulation_llama1b_full_grid(sched):
     cfg = cfg_for("llama1b")
     err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched=sched), 148, steps=2, seed=7,
@@ -142,8 +170,30 @@ def test_simulation_detects_a_missing_producer():
     assert "waited too long" in err
 
 
+def test_simulation_event_queue_detects_a_missing_producer():
+    """In the event-driven mode a dropped producer leaves its dependents out
+    of the ready queue: the simulation reports the slot that is never filled."""
+    cfg = cfg_for("tiny")
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched="event", debug_drop_producer=True), 4, steps=1,
+                                   seed=1, timeout_ms=300)
+    assert "never filled" in err
+
+
+def test_event_plan_is_the_dynamic_order():
+    """The event-driven plan holds the same instructions in the same
+    topological order as the dynamic queue (only the claim order differs)."""
+    cfg = cfg_for("llama1b")
+    a, *_ = mk.mk_host_plan(cfg, mk.plan_opts(batch=1, sched="dynamic"), 148)
+    b, *_ = mk.mk_host_plan(cfg, mk.plan_opts(batch=1, sched="event"), 148)
+    assert [bytes(x) for x in a] == [bytes(x) for x in b]
+
+
 def test_plan_rejects_bad_options():
     cfg = cfg_for("tiny")
+    with pytest.raises(mk.MkError):
+        o = mk.plan_opts(batch=1)
+        o.sched_mode = 3
+        mk.mk_host_plan(cfg, o, 8)
     with pytest.raises(mk.MkError):
         mk.mk_host_plan(cfg, mk.plan_opts(batch=2), 8)
     with pytest.raises(mk.MkError):
@@ -224,7 +274,8 @@ def test_use_tcgen05_option():
 
 
 @pytest.mark.parametrize("tqo", [False, True])
-@pytest.mark.parametrize("sched,num_ctas", [("static", 37), ("dynamic", 148), ("dynamic", 16)])
+@pytest.mark.parametrize("sched,num_ctas", [("static", 37), ("dynamic", 148), ("dynamic", 16), ("event", 148),
+                                            ("event", 16)])
 def test_batched_plan_other_grids(tqo, sched, num_ctas):
     """Batched plans on smaller grids and with the dynamic queue: every
     matrix row of every layer is covered exactly once, and the host
@@ -291,6 +342,9 @@ def test_plan_structure_shape_grid(H, d, nq, nkv, F, V):
     err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched="dynamic"), 13, steps=2, seed=V,
                                    timeout_ms=30000)
     assert err == ""
+    err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=1, sched="event"), 13, steps=2, seed=V + 1,
+                                   timeout_ms=30000)
+    assert err == ""
 
 
 @pytest.mark.parametrize("F", [768, 1280, 3072, 18432])
@@ -305,6 +359,7 @@ def test_unsupported_ffn_widths_rejected(F):
 
 @pytest.mark.parametrize("seed", [101, 202, 303])
 @pytest.mark.parametrize("name,batch,kw", [("llama1b", 1, {}), ("llama1b", 1, {"sched": "dynamic"}),
+                                            ("llama1b", 1, {"sched": "event"}), ("llama1b_b16", 16, {"sched": "event"}),
                                             ("llama8b", 1, {}), ("llama1b_b16", 16, {}),
                                             ("llama1b_b16", 16, {"tensor_qkv_o": True})])
 def test_simulation_more_seeds(seed, name, batch, kw):
