@@ -115,6 +115,18 @@ def load(path: str = LIB_PATH):
     L.mk_plan.argtypes = [vp, P(mk_plan_opts)]
     L.mk_decode_step.restype = i32
     L.mk_decode_step.argtypes = [vp, vp, vp, vp, vp, vp]
+    L.mk_prefill.restype = i32
+    L.mk_prefill.argtypes = [vp, i32, vp, i32, i32, vp, vp, vp]
+    L.mk_tp_create.restype = i32
+    L.mk_tp_create.argtypes = [P(mk_config), P(mk_weights), P(mk_kv_cache), i32, P(vp)]
+    L.mk_tp_plan.restype = i32
+    L.mk_tp_plan.argtypes = [vp, P(mk_plan_opts)]
+    L.mk_tp_decode_step.restype = i32
+    L.mk_tp_decode_step.argtypes = [vp, vp, vp, vp, vp, vp]
+    L.mk_tp_get_status.restype = i32
+    L.mk_tp_get_status.argtypes = [vp, vp]
+    L.mk_tp_destroy.restype = None
+    L.mk_tp_destroy.argtypes = [vp]
     L.mk_get_status.restype = i32
     L.mk_get_status.argtypes = [vp, vp]
     L.mk_status_string.restype = ctypes.c_char_p
@@ -167,6 +179,12 @@ def mk_decode_step(h: int, tokens: int, positions: int, logits_out: int | None, 
                    stream: int | None) -> int:
     """Raw pointers (ints).  Returns the status code (no exception: the step is async)."""
     return load().mk_decode_step(h, tokens, positions, logits_out, next_tokens_out, stream)
+
+
+def mk_prefill(h: int, seq: int, tokens: int, n_tokens: int, pos0: int, logits_out: int | None,
+               next_token_out: int, stream: int | None) -> int:
+    """Raw pointers (ints).  Returns the status code (asynchronous)."""
+    return load().mk_prefill(h, seq, tokens, n_tokens, pos0, logits_out, next_token_out, stream)
 
 
 def mk_decode_step_noalloc(cfg: mk_config, weights: mk_weights, kv: mk_kv_cache, tokens: int, positions: int,
@@ -318,6 +336,16 @@ class Engine:
         if rc != MK_OK:
             raise MkError(rc, "mk_decode_step")
 
+    def prefill(self, seq, tokens, pos0, logits_out, next_token_out, stream=None) -> None:
+        """Prompt tokens (device int32 tensor) of sequence `seq` from position
+        pos0: their K/V rows, and the last token's logits / greedy next token."""
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream()
+        rc = mk_prefill(self.h, seq, _ptr(tokens), int(tokens.numel()), pos0,
+                        _ptr(logits_out) if logits_out is not None else None, _ptr(next_token_out), s.cuda_stream)
+        if rc != MK_OK:
+            raise MkError(rc, "mk_prefill")
+
     def status(self, stream=None) -> int:
         import torch
         s = stream if stream is not None else torch.cuda.current_stream()
@@ -345,3 +373,59 @@ def _ptr(t):
         return t
     assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
     return t.data_ptr()
+
+
+class TpEngine:
+    """A tensor-parallel group of n ranks emulated on this GPU (mk_tp_*): the
+    same weights / cache arguments as Engine (batch 1 plans)."""
+
+    def __init__(self, shape, weights: dict, kcache, vcache, max_batch: int, max_seq: int, n_ranks: int):
+        self.cfg = make_config(shape, max_batch, max_seq)
+        self._keep = (weights, kcache, vcache)
+        layers = weights["layers"]
+        self._lw = (mk_layer_weights * len(layers))()
+        for i, L in enumerate(layers):
+            for n, _ in mk_layer_weights._fields_:
+                setattr(self._lw[i], n, _ptr(L[n]))
+        lm = weights.get("lm_head")
+        self._w = mk_weights(_ptr(weights["embed"]), _ptr(lm) if lm is not None else None,
+                             _ptr(weights["final_norm"]), self._lw)
+        self._kv = mk_kv_cache(_ptr(kcache), _ptr(vcache))
+        g = ctypes.c_void_p()
+        rc = load().mk_tp_create(ctypes.byref(self.cfg), ctypes.byref(self._w), ctypes.byref(self._kv), n_ranks,
+                                 ctypes.byref(g))
+        if rc != MK_OK:
+            raise MkError(rc, "mk_tp_create")
+        self.g = g.value
+        self.n_ranks = n_ranks
+
+    def plan(self, **kw) -> None:
+        self.opts = plan_opts(**kw)
+        rc = load().mk_tp_plan(self.g, ctypes.byref(self.opts))
+        if rc != MK_OK:
+            raise MkError(rc, "mk_tp_plan")
+
+    def decode_step(self, tokens, positions, logits_out, next_tokens_out, stream=None) -> None:
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream()
+        rc = load().mk_tp_decode_step(self.g, _ptr(tokens), _ptr(positions),
+                                      _ptr(logits_out) if logits_out is not None else None, _ptr(next_tokens_out),
+                                      s.cuda_stream)
+        if rc != MK_OK:
+            raise MkError(rc, "mk_tp_decode_step")
+
+    def status(self, stream=None) -> int:
+        import torch
+        s = stream if stream is not None else torch.cuda.current_stream()
+        return load().mk_tp_get_status(self.g, s.cuda_stream)
+
+    def close(self) -> None:
+        if getattr(self, "g", None):
+            load().mk_tp_destroy(self.g)
+            self.g = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -51,6 +51,10 @@ struct mk_handle {
   const void *kernel = nullptr;  // the interpreter build this plan launches
   int kernel_variant = 0;        // 1: specialised for this model's shape
   int est_step_us = 0;           // the plan cost model's step estimate at max_seq (0: dynamic queue)
+  // mk_prefill's scratch for the logits and greedy tokens of a chunk's rows
+  // (allocated with the plan on first use)
+  float *pf_logits = nullptr;
+  int *pf_next = nullptr;
   int last_detail[6] = {0, 0, 0, 0, 0, 0};
   // per-op graph mode
   cudaGraphExec_t gexec = nullptr;
@@ -468,6 +472,8 @@ static void drop_plan(mk_handle *h) {
     h->gexec = nullptr;
   }
   free_list(h->plan_allocs);
+  h->pf_logits = nullptr;
+  h->pf_next = nullptr;
   h->planned = false;
 }
 
@@ -801,6 +807,48 @@ extern "C" int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t
   return MK_OK;
 }
 
+extern "C" int mk_prefill(mk_handle *h, int32_t seq, const int32_t *tokens, int32_t n_tokens, int32_t pos0,
+                          float *logits_out, int32_t *next_token_out, void *stream) {
+  if (!h || !tokens || !next_token_out || n_tokens < 1 || pos0 < 0) return MK_ERR_INVALID_ARG;
+  if (!h->planned) return MK_ERR_NOT_PLANNED;
+  if (seq < 0 || seq >= h->cfg.max_batch || (int64_t)pos0 + n_tokens > h->cfg.max_seq) return MK_ERR_INVALID_ARG;
+  if (h->opts.exec_mode != MK_EXEC_MEGAKERNEL && h->opts.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC)
+    return MK_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int B = h->kp.B, V = h->kp.V;
+  if (!h->pf_next) {
+    int rc;
+    if ((rc = dalloc(h->plan_allocs, &h->pf_logits, (size_t)B * V, false))) return rc;
+    if ((rc = dalloc(h->plan_allocs, &h->pf_next, (size_t)B, false))) return rc;
+  }
+  // chunks of up to B consecutive tokens, one launch each: row b of a chunk
+  // is its b-th token (batched plans), or one token per launch (batch 1)
+  int last_n = 0;
+  for (int c0 = 0; c0 < n_tokens; c0 += B) {
+    KParams k = h->kp;
+    k.chunk_n = std::min(B, n_tokens - c0);
+    k.chunk_pos0 = pos0 + c0;
+    k.kv_seq0 = seq;
+    k.tokens = tokens + c0;
+    k.positions = tokens + c0;  // unused for chunks
+    k.logits = (c0 + B >= n_tokens && logits_out) ? h->pf_logits : nullptr;
+    k.next_tokens = h->pf_next;
+    k.mode |= MODE_FINAL_LAUNCH;
+    cudaError_t e = launch_interp(h->kernel, k, h->grid, h->smem, st, true);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_code(e);
+    }
+    last_n = k.chunk_n;
+  }
+  // the last token's row: its logits and greedy next token
+  if (logits_out)
+    MK_CUDA(cudaMemcpyAsync(logits_out, h->pf_logits + (size_t)(last_n - 1) * V, sizeof(float) * V,
+                            cudaMemcpyDeviceToDevice, st));
+  MK_CUDA(cudaMemcpyAsync(next_token_out, h->pf_next + (last_n - 1), sizeof(int32_t), cudaMemcpyDeviceToDevice, st));
+  return MK_OK;
+}
+
 extern "C" int mk_get_status(mk_handle *h, void *stream) {
   if (!h) return MK_ERR_INVALID_ARG;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
@@ -1031,4 +1079,246 @@ extern "C" int mk_host_plan_estimate(const mk_config *cfg, const mk_plan_opts *o
   out->savings_us = est.per_op_us - est.step_us;
   for (int i = 0; i < 7; ++i) out->stage_us[i] = est.stage_us[i];
   return MK_OK;
+}
+
+// ====================================================================== tensor parallelism
+
+// A tensor-parallel group of n ranks emulated on this GPU: rank r is a handle
+// over its shard of the model (heads, FFN columns, vocabulary rows), and one
+// cooperative launch of n * (SMs / n) CTAs runs every rank's plan, each block
+// of SMs / n CTAs with its rank's parameters (ranks whose kernels wait on one
+// another must run in one launch on one GPU).
+struct mk_tp_group {
+  int n = 0;
+  mk_config cfg;                      // the full model's
+  std::vector<mk_handle *> ranks;
+  std::vector<void *> allocs;         // column shards of Wo and Wd
+  std::vector<void *> plan_allocs;    // per plan: partial buffers, tables, I/O
+  KParams *d_params = nullptr;        // [n]
+  int32_t *d_tok = nullptr, *d_pos = nullptr, *d_next = nullptr;  // [B]
+  float *d_logits = nullptr;          // [B][V]
+  KParams launch{};                   // rank 0's parameters + the group table
+  const void *kernel = nullptr;
+  int smem = 0, ctas = 0, B = 1;
+  bool planned = false;
+};
+
+extern "C" int mk_tp_create(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv, int32_t n_ranks,
+                            mk_tp_group **out) {
+  if (out) *out = nullptr;
+  if (!cfg || !w || !kv || !out || !w->layers) return MK_ERR_INVALID_ARG;
+  if (n_ranks != 2 && n_ranks != 4 && n_ranks != 8) return MK_ERR_INVALID_ARG;
+  std::string why;
+  int rc = check_cfg(cfg, &why);
+  if (rc) return rc;
+  const int n = n_ranks;
+  if (cfg->n_q_heads % n || cfg->n_kv_heads % n || cfg->ffn % n || cfg->vocab % n) return MK_ERR_UNSUPPORTED_SHAPE;
+  if (!w->embed || !w->final_norm || (!cfg->tied_lm_head && !w->lm_head) || !kv->k || !kv->v)
+    return MK_ERR_INVALID_ARG;
+  mk_tp_group *g = new (std::nothrow) mk_tp_group();
+  if (!g) return MK_ERR_OUT_OF_MEMORY;
+  g->n = n;
+  g->cfg = *cfg;
+  auto fail = [&](int code) {
+    cudaDeviceSynchronize();
+    for (mk_handle *h : g->ranks) mk_destroy(h);
+    free_list(g->allocs);
+    delete g;
+    return code;
+  };
+  const int H = cfg->hidden, d = cfg->head_dim, L = cfg->n_layers;
+  const int qd_r = cfg->n_q_heads / n * d, kvd_r = cfg->n_kv_heads / n * d, F_r = cfg->ffn / n,
+            V_r = cfg->vocab / n;
+  const uint16_t *lm = (const uint16_t *)(cfg->tied_lm_head ? w->embed : w->lm_head);
+  for (int r = 0; r < n; ++r) {
+    mk_config rc_cfg = *cfg;
+    rc_cfg.n_q_heads = cfg->n_q_heads / n;
+    rc_cfg.n_kv_heads = cfg->n_kv_heads / n;
+    rc_cfg.ffn = F_r;
+    rc_cfg.vocab = V_r;
+    rc_cfg.tied_lm_head = 0;
+    std::vector<mk_layer_weights> lw(L);
+    for (int l = 0; l < L; ++l) {
+      const mk_layer_weights &S = w->layers[l];
+      mk_layer_weights &D = lw[l];
+      D = S;
+      // row shards are views; column shards (Wo, Wd) are copied
+      D.wq = (const uint16_t *)S.wq + (size_t)r * qd_r * H;
+      D.wk = (const uint16_t *)S.wk + (size_t)r * kvd_r * H;
+      D.wv = (const uint16_t *)S.wv + (size_t)r * kvd_r * H;
+      D.w_gate = (const uint16_t *)S.w_gate + (size_t)r * F_r * H;
+      D.w_up = (const uint16_t *)S.w_up + (size_t)r * F_r * H;
+      uint16_t *wo = nullptr, *wd = nullptr;
+      if ((rc = dalloc(g->allocs, &wo, (size_t)H * qd_r, false))) return fail(rc);
+      if ((rc = dalloc(g->allocs, &wd, (size_t)H * F_r, false))) return fail(rc);
+      cudaError_t e = cudaMemcpy2D(wo, (size_t)qd_r * 2, (const uint16_t *)S.wo + (size_t)r * qd_r,
+                                   (size_t)cfg->n_q_heads * d * 2, (size_t)qd_r * 2, H, cudaMemcpyDeviceToDevice);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2D(wd, (size_t)F_r * 2, (const uint16_t *)S.w_down + (size_t)r * F_r, (size_t)cfg->ffn * 2,
+                         (size_t)F_r * 2, H, cudaMemcpyDeviceToDevice);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MK_ERR_CUDA);
+      }
+      D.wo = wo;
+      D.w_down = wd;
+    }
+    mk_weights rw = *w;
+    rw.lm_head = lm + (size_t)r * V_r * H;
+    rw.layers = lw.data();
+    // this rank's KV heads inside the caller's cache (strides of the full cache
+    // are set when planning)
+    mk_kv_cache rk;
+    rk.k = (uint16_t *)kv->k + (size_t)r * (cfg->n_kv_heads / n) * cfg->max_seq * d;
+    rk.v = (uint16_t *)kv->v + (size_t)r * (cfg->n_kv_heads / n) * cfg->max_seq * d;
+    mk_handle *h = nullptr;
+    if ((rc = mk_create(&rc_cfg, &rw, &rk, &h))) return fail(rc);
+    g->ranks.push_back(h);
+  }
+  *out = g;
+  return MK_OK;
+}
+
+static void tp_drop_plan(mk_tp_group *g) {
+  free_list(g->plan_allocs);
+  g->d_params = nullptr;
+  g->planned = false;
+}
+
+extern "C" int mk_tp_plan(mk_tp_group *g, const mk_plan_opts *opts_in) {
+  if (!g) return MK_ERR_INVALID_ARG;
+  mk_plan_opts o = opts_in ? *opts_in : default_opts(g->cfg);
+  // the rank build: batch 1, static per-SM queues, one launch
+  if (o.batch != 1 || o.sched_mode != MK_SCHED_STATIC || o.kv_splits < 0 ||
+      (o.exec_mode != MK_EXEC_MEGAKERNEL && o.exec_mode != MK_EXEC_MEGAKERNEL_GENERIC) || o.trace)
+    return MK_ERR_INVALID_ARG;
+  cudaDeviceSynchronize();
+  tp_drop_plan(g);
+  const int n = g->n;
+  mk_handle *h0 = g->ranks[0];
+  const int C = h0->sm_count / n;
+  if (C < 1) return MK_ERR_LAUNCH;
+  o.exec_mode = MK_EXEC_MEGAKERNEL_GENERIC;
+  o.num_sms = C;
+  int rc;
+  for (mk_handle *h : g->ranks)
+    if ((rc = mk_plan(h, &o))) return rc;
+  const mk_config &c = g->cfg;
+  const int B = 1, H = c.hidden, L = c.n_layers, V = c.vocab;
+  const int ndp_r = h0->plan.ndp, n_lm_r = h0->plan.n_lm;
+  for (mk_handle *h : g->ranks)
+    if (h->plan.ndp != ndp_r || h->plan.n_lm != n_lm_r || h->smem != h0->smem) return MK_ERR_UNSUPPORTED_SHAPE;
+  if (n * ndp_r > kMaxDownPieces) return MK_ERR_UNSUPPORTED_SHAPE;
+  TpPeer *d_peers = nullptr;
+  std::vector<TpPeer> peers(n);
+  if ((rc = dalloc(g->plan_allocs, &d_peers, (size_t)n, false))) return rc;
+  if ((rc = dalloc(g->plan_allocs, &g->d_params, (size_t)n, false))) return rc;
+  if ((rc = dalloc(g->plan_allocs, &g->d_tok, (size_t)B))) return rc;
+  if ((rc = dalloc(g->plan_allocs, &g->d_pos, (size_t)B))) return rc;
+  if ((rc = dalloc(g->plan_allocs, &g->d_next, (size_t)B))) return rc;
+  if ((rc = dalloc(g->plan_allocs, &g->d_logits, (size_t)B * V))) return rc;
+  std::vector<KParams> kp(n);
+  for (int r = 0; r < n; ++r) {
+    mk_handle *h = g->ranks[r];
+    KParams &k = kp[r];
+    k = h->kp;
+    // every rank's copies of the cross-rank buffers (zeroed: no step tag yet)
+    if ((rc = dalloc(g->plan_allocs, &k.opart, (size_t)L * n * B * H))) return rc;
+    if ((rc = dalloc(g->plan_allocs, &k.dpart, (size_t)L * n * ndp_r * B * H))) return rc;
+    if ((rc = dalloc(g->plan_allocs, &k.arg_val, (size_t)B * n * n_lm_r))) return rc;
+    if ((rc = dalloc(g->plan_allocs, &k.arg_idx, (size_t)B * n * n_lm_r))) return rc;
+    peers[r] = TpPeer{k.opart, k.dpart, k.ctr, k.arg_val, k.arg_idx};
+    k.tp_n = n;
+    k.tp_rank = r;
+    k.tp_ctas = C;
+    k.tp_peers = d_peers;
+    k.ndp_local = ndp_r;
+    k.ndp = n * ndp_r;
+    k.n_lm_local = n_lm_r;
+    k.n_lm = n * n_lm_r;
+    k.n_gu_layer = h->plan.n_gu;
+    k.V = V;
+    k.V_lm = V / n;
+    k.lm_row0 = r * (V / n);
+    // the caller's full cache: this rank's heads, full strides
+    k.kv_hs = (long long)c.max_seq * c.head_dim;
+    k.kv_bs = k.kv_hs * c.n_kv_heads;
+    k.kv_ls = k.kv_bs * c.max_batch;
+    k.tokens = g->d_tok;
+    k.positions = g->d_pos;
+    k.logits = g->d_logits;
+    k.next_tokens = g->d_next;
+    k.mode = MODE_FINAL_LAUNCH;
+    // the O and down counters count every rank's producers
+    std::vector<Instr> ins = h->plan.instrs;
+    for (Instr &I : ins)
+      if ((I.op == OP_GATEUP) || (I.op == OP_QKV && I.layer > 0) || I.op == OP_LMHEAD) I.wait_cnt *= (uint32_t)n;
+    cudaError_t e = cudaMemcpy(const_cast<Instr *>(k.instrs), ins.data(), ins.size() * sizeof(Instr),
+                               cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return MK_ERR_CUDA;
+    }
+  }
+  cudaError_t e = cudaMemcpy(d_peers, peers.data(), sizeof(TpPeer) * n, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemcpy(g->d_params, kp.data(), sizeof(KParams) * n, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  g->kernel = interp_kernel_tp();
+  g->smem = h0->smem;
+  g->ctas = C;
+  g->B = B;
+  int per_sm = 0;
+  e = interp_prepare(g->kernel, g->smem, &per_sm);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (per_sm < 1) return MK_ERR_LAUNCH;
+  g->launch = kp[0];
+  g->launch.tp_params = g->d_params;
+  g->planned = true;
+  return MK_OK;
+}
+
+extern "C" int mk_tp_decode_step(mk_tp_group *g, const int32_t *tokens, const int32_t *positions, float *logits_out,
+                                 int32_t *next_tokens_out, void *stream) {
+  if (!g || !tokens || !positions || !next_tokens_out) return MK_ERR_INVALID_ARG;
+  if (!g->planned) return MK_ERR_NOT_PLANNED;
+  cudaStream_t st = (cudaStream_t)stream;
+  MK_CUDA(cudaMemcpyAsync(g->d_tok, tokens, sizeof(int32_t) * g->B, cudaMemcpyDeviceToDevice, st));
+  MK_CUDA(cudaMemcpyAsync(g->d_pos, positions, sizeof(int32_t) * g->B, cudaMemcpyDeviceToDevice, st));
+  cudaError_t e = launch_interp(g->kernel, g->launch, g->n * g->ctas, g->smem, st, true);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_code(e);
+  }
+  if (logits_out)
+    MK_CUDA(cudaMemcpyAsync(logits_out, g->d_logits, sizeof(float) * g->B * g->cfg.vocab, cudaMemcpyDeviceToDevice,
+                            st));
+  MK_CUDA(cudaMemcpyAsync(next_tokens_out, g->d_next, sizeof(int32_t) * g->B, cudaMemcpyDeviceToDevice, st));
+  return MK_OK;
+}
+
+extern "C" int mk_tp_get_status(mk_tp_group *g, void *stream) {
+  if (!g) return MK_ERR_INVALID_ARG;
+  int first = MK_OK;
+  for (mk_handle *h : g->ranks) {
+    const int rc = mk_get_status(h, stream);
+    if (rc != MK_OK && first == MK_OK) first = rc;
+  }
+  // a failed step leaves the ranks' counters and step numbers apart: plan again
+  if (first != MK_OK) tp_drop_plan(g);
+  return first;
+}
+
+extern "C" void mk_tp_destroy(mk_tp_group *g) {
+  if (!g) return;
+  cudaDeviceSynchronize();
+  tp_drop_plan(g);
+  for (mk_handle *h : g->ranks) mk_destroy(h);
+  free_list(g->allocs);
+  delete g;
 }

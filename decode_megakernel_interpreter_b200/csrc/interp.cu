@@ -18,7 +18,9 @@ size_t staging_floats(int H, int qdim, int KCd, int G, int d, int nb) {
   size_t vec = nb == 1 ? std::max({(size_t)H, (size_t)qdim + H, (size_t)KCd, (size_t)kSplitRedFloats + H})
                        : (size_t)nb * std::max({H, qdim, KCd});
   // warps' partials + the current K/V rows (bf16) + the warps' merge weights
-  size_t attn = (size_t)kComputeWarps * G * (d + 2) + (size_t)d + (size_t)G * (kComputeWarps + 2);
+  // (+ batched builds: two K and two V rows of a prompt chunk per warp, bf16)
+  size_t attn = (size_t)kComputeWarps * G * (d + 2) + (size_t)d + (((size_t)G * (kComputeWarps + 2) + 3) & ~(size_t)3) +
+                (nb > 1 ? (size_t)kComputeWarps * 2 * d : 0);
   size_t f = std::max(vec, attn);
   // batched builds: the tensor-core epilogue exchange follows the staged vectors
   if (nb > 1) f += kTcXchFloats;
@@ -64,6 +66,8 @@ const void *interp_kernel_for(const KParams &p, bool specialised, int nb, bool t
 }
 
 const void *interp_kernel_raw() { return (const void *)interp_kernel<1, true, SpecGeneric>; }
+
+const void *interp_kernel_tp() { return (const void *)interp_kernel<1, false, SpecGenericTP>; }
 
 cudaError_t interp_prepare(const void *fn, int smem, int *blocks_per_sm) {
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -299,6 +299,11 @@ __device__ __forceinline__ bool global_abort(const KParams &p) { return px::ld_v
 // positions and token ids are read once per launch into shared memory
 __device__ __forceinline__ int read_pos(const Shared *sh, int b) { return sh->pos[b]; }
 __device__ __forceinline__ int read_tok(const Shared *sh, int b) { return sh->tok[b]; }
+// KV-cache sequence of row b: b in decode steps (kv_seq0 = 0), the prompt's
+// sequence kv_seq0 for every row of a prompt chunk
+__device__ __forceinline__ int kv_seq(const KParams &p, int b) { return p.kv_seq0 + (p.chunk_n > 0 ? 0 : b); }
+// rows of a prompt chunk past its last token: computed, never stored
+__device__ __forceinline__ bool chunk_pad(const KParams &p, int b) { return p.chunk_n > 0 && b >= p.chunk_n; }
 
 // Tagged loads are consumed in groups: every word of a group is loaded, the
 // values are used as loaded, and `ok` collects whether each word carried this
@@ -403,6 +408,17 @@ struct SplitRange {
 __device__ __forceinline__ SplitRange split_range(const KParams &p, const Shared *sh, int b, int s) {
   SplitRange r;
   r.pos = read_pos(sh, b);
+  if (p.chunk_n > 1) {
+    // a prompt chunk of several tokens: the S splits share the positions
+    // cached before the chunk; the last split also takes the chunk's own
+    // rows up to this row's position (this step's K/V exchange, not the cache)
+    const int n = p.chunk_pos0, chunk = (n + p.S - 1) / p.S;
+    r.start = min(n, s * chunk);
+    r.end = min(n, r.start + chunk);
+    r.pref_end = r.end;
+    r.has_cur = s == p.S - 1;
+    return r;
+  }
   int n = r.pos + 1;
   int chunk = (n + p.S - 1) / p.S;
   r.start = min(n, s * chunk);
@@ -548,7 +564,8 @@ __device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, 
       const SplitRange r = split_range(p, sh, I.c, I.b);
       const int ppp = attn_ppp(p), n = r.pref_end - r.start;
       s.npg = n > 0 ? (n + ppp - 1) / ppp : 0;
-      const size_t off = (size_t)I.layer * p.kv_ls + (size_t)I.c * p.kv_bs + (size_t)I.a * p.kv_hs + (size_t)r.start * p.d;
+      const size_t off = (size_t)I.layer * p.kv_ls + (size_t)kv_seq(p, I.c) * p.kv_bs + (size_t)I.a * p.kv_hs +
+                         (size_t)r.start * p.d;
       s.a = p.kc + off;
       s.b = p.vc + off;
       s.stride = (size_t)ppp * p.d;
@@ -1513,7 +1530,7 @@ __device__ __forceinline__ uint32_t qkv_rows(CCtx c, const Instr I) {
     } else {
       const bool isk = head < nq + nkv;
       const int gk = isk ? head - nq : head - nq - nkv;
-      uint16_t *dst = (isk ? kl : vl) + (size_t)gk * kv_hs + (size_t)pos * d;
+      uint16_t *dst = (isk ? kl : vl) + (size_t)kv_seq(p, 0) * p.kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
       const uint16_t bu = px::f2bf(u), bw = px::f2bf(w);
       dst[i] = bu;
       dst[i + hd] = bw;
@@ -1574,7 +1591,7 @@ __device__ __forceinline__ uint32_t down_rows(CCtx c, const Instr I) {
 }
 
 // forward declaration: the LM head's argmax merge (defined with the paged bodies)
-template <int NB>
+template <int NB, bool TP = false>
 __device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&bv)[NB], int (&bi)[NB]);
 __device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi);
 
@@ -1645,10 +1662,12 @@ __device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
           // this step's attention as tagged words
           const bool isk = head < nq + nkv;
           const int gk = isk ? head - nq : head - nq - nkv;
-          uint16_t *dst = (isk ? kl : vl) + (size_t)b * kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
+          uint16_t *dst = (isk ? kl : vl) + (size_t)kv_seq(p, b) * kv_bs + (size_t)gk * kv_hs + (size_t)pos * d;
           const uint16_t bu = px::f2bf(u), bw = px::f2bf(w);
-          dst[i] = bu;
-          dst[i + hd] = bw;
+          if (!chunk_pad(p, b)) {
+            dst[i] = bu;
+            dst[i + hd] = bw;
+          }
           float *cur = kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + gk * d;
           px::st_tf(cur + i, px::bf16f(bu), tag);  // bf16 values: exact in 22 significant bits
           px::st_tf(cur + i + hd, px::bf16f(bw), tag);
@@ -1764,7 +1783,7 @@ __device__ __forceinline__ bool arg_better(float v, int i, float bv, int bi) {
 // The LM-head instruction's argmax: per thread (bv, bi) of each sequence ->
 // per warp -> per CTA (the instruction's tagged slot); the last LM instruction
 // to finish merges every slot and writes the next tokens.
-template <int NB>
+template <int NB, bool TP>
 __device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&bv)[NB], int (&bi)[NB]) {
   const KParams &p = c.p;
   // CTA-wide argmax of this instruction
@@ -1797,8 +1816,17 @@ __device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&
         v = c.sh->argv[w][b];
         i = c.sh->argi[w][b];
       }
-    px::st_ll(p.arg_val + (size_t)b * p.n_lm + I.c, v, c.epoch);
-    px::st_ll(p.arg_idx + (size_t)b * p.n_lm + I.c, __int_as_float(i), c.epoch);
+    if constexpr (TP) {
+      // this rank's slot in every rank's table
+      const size_t slot = (size_t)b * p.n_lm + (size_t)p.tp_rank * p.n_lm_local + I.c;
+      for (int rr = 0; rr < p.tp_n; ++rr) {
+        px::st_ll(p.tp_peers[rr].arg_val + slot, v, c.epoch);
+        px::st_ll(p.tp_peers[rr].arg_idx + slot, __int_as_float(i), c.epoch);
+      }
+    } else {
+      px::st_ll(p.arg_val + (size_t)b * p.n_lm + I.c, v, c.epoch);
+      px::st_ll(p.arg_idx + (size_t)b * p.n_lm + I.c, __int_as_float(i), c.epoch);
+    }
   }
   px::cbar();
   // the last LM instruction to finish merges every slot (all compute threads
@@ -1806,7 +1834,9 @@ __device__ __forceinline__ void lm_argmax_tail(CCtx &c, const Instr &I, float (&
   // tagged words, so the ticket needs no fence
   if (c.ctid == 0) {
     const unsigned old = px::atom_relaxed_add(p.ctr + p.arg_ticket0, 1u);
-    c.sh->flag = (old == c.epoch * (unsigned)p.n_lm - 1u);
+    // (tensor parallelism: the rank's own LM instructions; the other ranks'
+    // slots are tagged, and the merge below waits for them)
+    c.sh->flag = (old == c.epoch * (unsigned)(TP ? p.n_lm_local : p.n_lm) - 1u);
   }
   px::cbar();
   if (c.sh->flag) {  // uniform: every compute thread reads the same flag
@@ -1883,7 +1913,7 @@ __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
         if (NB > 1 && b >= Bn) break;
         const float v = pick<R>(acc[b], lane) * inv[b];
         if (valid) {
-          if (logits) logits[(size_t)b * V + row] = v;
+          if (logits && !chunk_pad(p, b)) logits[(size_t)b * V + row] = v;
           if (arg_better(v, row, bv[b], bi[b])) {
             bv[b] = v;
             bi[b] = row;
@@ -1984,7 +2014,7 @@ __device__ __forceinline__ uint32_t lmhead_tc_body(CCtx c, const Instr I) {
     for (int b = 0; b < NB; ++b) {
       if (b >= Bn) break;
       const float x = v[b] * inv[b];
-      if (p.logits) p.logits[(size_t)b * V + row] = x;
+      if (p.logits && !chunk_pad(p, b)) p.logits[(size_t)b * V + row] = x;
       if (arg_better(x, row, bv[b], bi[b])) {
         bv[b] = x;
         bi[b] = row;
@@ -2127,8 +2157,8 @@ __device__ __forceinline__ uint32_t qkv_tc_body(CCtx c, const Instr I) {
         const bool isk = head < nq + nkv;
         const int gk = isk ? head - nq : head - nq - nkv;
         const uint16_t bo = px::f2bf(out);
-        uint16_t *dst = (isk ? kl : vl) + (size_t)b * p.kv_bs + (size_t)gk * p.kv_hs + (size_t)pos * d;
-        dst[i] = bo;
+        uint16_t *dst = (isk ? kl : vl) + (size_t)kv_seq(p, b) * p.kv_bs + (size_t)gk * p.kv_hs + (size_t)pos * d;
+        if (!chunk_pad(p, b)) dst[i] = bo;
         px::st_tf(kvc + ((size_t)b * 2 + (isk ? 0 : 1)) * kvdim + (size_t)gk * d + i, px::bf16f(bo), tag);
       }
     }
@@ -2177,6 +2207,162 @@ template <int NB, int R>
 __device__ __noinline__ uint32_t op_lmhead_tc(CCtx c, const Instr I) { return lmhead_tc_body<NB, R>(c, I); }
 template <int NB, int R>
 __device__ __noinline__ uint32_t op_lmhead(CCtx c, const Instr I) { return lmhead_body<NB, R>(c, I); }
+
+// ---------------------------------------------------------------- tensor parallelism
+// One rank of a tensor-parallel group (batch 1, one page per warp; the
+// "Mirage Persistent Kernel" article, part 1: a collective split into chunks,
+// each depending only on the tile that produces it).  The rank holds the
+// heads, FFN columns and vocabulary rows of its shard: the O projection (row
+// split: its heads' columns of Wo) and the down projection (its FFN columns)
+// produce partial sums of every output row, which each producing page stores
+// into every rank's copy of the partial buffers (peer stores; tagged words,
+// so a consumer needs no flag beyond the counters it already polls); the
+// consumers sum the ranks' partials in rank order -- an all-reduce whose
+// chunks are single pages.
+
+// x_mid(l) * gamma staged (x_mid = x_in(l) + the ranks' O partials), 1/rms
+// returned; this instruction also stores rows [row_lo, row_hi) of x_mid as the
+// rank's residual copy xres[l] (the next layer's input starts from it).
+template <int IT>
+__device__ float stage_norm_tp_mid(CCtx &c, int l, const uint16_t *gamma, int row_lo, int row_hi) {
+  const KParams &p = c.p;
+  const int H = p.H, n4 = H / 4;
+  const uint32_t tag = c.epoch;
+  float4 xs[IT];
+  uint2 gws[IT];
+  const int tok = l == 0 ? read_tok(c.sh, 0) : 0;
+  settle(c, 2, [&](bool &ok) {
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int e4 = c.ctid + it * kComputeThreads;
+      if (e4 < n4) {
+        gws[it] = __ldg(reinterpret_cast<const uint2 *>(gamma) + e4);
+        float4 x = layer_input4(p, tag, l, 0, tok, e4, ok);
+        for (int r = 0; r < p.tp_n; ++r) {
+          const float4 v = tf_chk4(px::ld_tf4(p.opart + ((size_t)l * p.tp_n + r) * p.B * H + e4 * 4), tag, ok);
+          x.x += v.x;
+          x.y += v.y;
+          x.z += v.z;
+          x.w += v.w;
+        }
+        xs[it] = x;
+      }
+    }
+  });
+  float ss = 0.f;
+  float4 *dst = reinterpret_cast<float4 *>(c.act);
+  float *const xres = p.xres + (size_t)l * p.B * H;
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int e4 = c.ctid + it * kComputeThreads;
+    if (e4 < n4) {
+      const float4 x = xs[it];
+      const uint2 gw = gws[it];
+      ss += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+      dst[stage_slot4(e4, H)] =
+          make_float4(x.x * px::bf_lo(gw.x), x.y * px::bf_hi(gw.x), x.z * px::bf_lo(gw.y), x.w * px::bf_hi(gw.y));
+      if (e4 * 4 >= row_lo && e4 * 4 < row_hi) {
+        px::st_tf(xres + e4 * 4 + 0, x.x, tag);
+        px::st_tf(xres + e4 * 4 + 1, x.y, tag);
+        px::st_tf(xres + e4 * 4 + 2, x.z, tag);
+        px::st_tf(xres + e4 * 4 + 3, x.w, tag);
+      }
+    }
+  }
+  ss = px::warp_sum(ss);
+  if (c.lane == 0) c.sh->red[c.cw][0] = ss;
+  px::cbar();
+  float t = 0.f;
+#pragma unroll
+  for (int w = 0; w < kComputeWarps; ++w) t += c.sh->red[w][0];
+  if (c.tr && c.ctid == 0) c.tr[2] = px::gtimer();
+  return __frsqrt_rn(t * p.inv_H + p.eps);
+}
+
+// O projection, row split: this rank's heads' columns; the partial of every
+// output row goes to slot tp_rank of every rank's opart[l]
+template <int R>
+__device__ __noinline__ uint32_t op_oproj_tp(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, lane = c.lane;
+  stage_copy<1, StageIt<R>::v>(c, p.obuf + (size_t)l * p.B * p.qdim, p.qdim, p.qdim);
+  const uint32_t tag = c.epoch;
+  const size_t off = ((size_t)l * p.tp_n + p.tp_rank) * p.B * p.H;
+  matvec_pages<1, R>(c, I, [&](int j, float (&acc)[1][R]) {
+    if (lane >= R) return;
+    const int row = j * R + lane;
+    const float v = pick<R>(acc[0], lane);
+    for (int rr = 0; rr < p.tp_n; ++rr) px::st_tf(p.tp_peers[rr].opart + off + row, v, tag);
+  });
+  return c.g;
+}
+
+// gate/up + SiLU * up for this rank's FFN columns; the instruction's slice of
+// x_mid becomes the rank's residual copy
+template <int R>
+__device__ __noinline__ uint32_t op_gateup_tp(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, half = R / 2, lane = c.lane, F = p.F;
+  const int n4 = p.H / 4, per = (n4 + p.n_gu_layer - 1) / p.n_gu_layer;
+  const int row_lo = min(n4, (int)I.c * per) * 4, row_hi = min(n4, ((int)I.c + 1) * per) * 4;
+  const float inv = stage_norm_tp_mid<StageIt<R>::v>(c, l, p.layers[l].ffn_norm, row_lo, row_hi);
+  const uint32_t tag = c.epoch;
+  float *const aout = p.actb + (size_t)l * p.B * F;
+  matvec_pages<1, R>(c, I, [&](int j, float (&acc)[1][R]) {
+    if (lane >= half) return;
+    const int row = j * half + lane;
+    const float gt = pick<R>(acc[0], lane) * inv, up = pick<R>(acc[0], lane + half) * inv;
+    const float silu = gt / (1.0f + expf(-gt));
+    px::st_tf(aout + row, silu * up, tag);
+  });
+  return c.g;
+}
+
+// down projection of this rank's FFN columns, K piece I.c: the partial goes
+// to piece tp_rank * ndp_local + I.c of every rank's dpart[l]
+template <int R>
+__device__ __noinline__ uint32_t op_down_tp(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  const int l = I.layer, k = I.c, lane = c.lane, H = p.H;
+  stage_copy<1, StageIt<R>::v>(c, p.actb + (size_t)l * p.B * p.F + (size_t)k * p.KCd, p.F, p.KCd);
+  const uint32_t tag = c.epoch;
+  const size_t off = ((size_t)l * p.ndp + (size_t)p.tp_rank * p.ndp_local + k) * p.B * H;
+  matvec_pages<1, R>(c, I, [&](int j, float (&acc)[1][R]) {
+    if (lane >= R) return;
+    const int row = j * R + lane;
+    const float v = pick<R>(acc[0], lane);
+    for (int rr = 0; rr < p.tp_n; ++rr) px::st_tf(p.tp_peers[rr].dpart + off + row, v, tag);
+  });
+  return c.g;
+}
+
+// LM head of this rank's vocabulary rows: their logits, and the rank's
+// argmax candidates in every rank's slots; the rank's last LM instruction
+// merges all ranks' slots
+template <int R>
+__device__ __noinline__ uint32_t op_lmhead_tp(CCtx c, const Instr I) {
+  const KParams &p = c.p;
+  float inv[1];
+  stage_norm<1, StageIt<R>::v>(c, p.L, p.final_norm, false, inv);
+  float bv[1] = {-INFINITY};
+  int bi[1] = {0x7fffffff};
+  const int lane = c.lane;
+  float *const logits = p.logits;
+  matvec_pages<1, R>(c, I, [&](int j, float (&acc)[1][R]) {
+    const int row = j * R + lane;
+    if (lane < R && row < p.V_lm) {
+      const float v = pick<R>(acc[0], lane) * inv[0];
+      const int gi = p.lm_row0 + row;
+      if (logits) logits[gi] = v;
+      if (arg_better(v, gi, bv[0], bi[0])) {
+        bv[0] = v;
+        bi[0] = gi;
+      }
+    }
+  });
+  lm_argmax_tail<1, true>(c, I, bv, bi);
+  return c.g;
+}
 
 // ---------------------------------------------------------------- attention
 // One (sequence b, kv head g, split s) item: online softmax over the split's
@@ -2292,7 +2478,7 @@ __device__ void attn_block(const float (&q)[G][DPL], const uint16_t *kb, const u
   }
 }
 
-template <int G, int DPL>
+template <int G, int DPL, bool CHUNK>
 __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   const KParams &p = c.p;
   constexpr int D = DPL * 32;
@@ -2310,7 +2496,13 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   // share of the last cached page (often none), not to an already loaded warp
   const int last_cnt = npg > 0 ? (r.pref_end - r.start) - (npg - 1) * PPP : 0;
   const int cur_warp = min(kComputeWarps - 1, last_cnt / PW);
-  const bool load_cur = r.has_cur && c.cw == cur_warp;
+  // a prompt chunk of several tokens (batched builds): the last split takes
+  // the chunk's rows 0 .. cb instead of one current row -- row j is token j's
+  // K/V row of this step's exchange; warp w takes rows w and w + 8
+  const bool chunk_rows = CHUNK && p.chunk_n > 1 && r.has_cur;
+  const int cb = chunk_rows ? r.pos - p.chunk_pos0 : -1;
+  const int nmine = chunk_rows ? (c.cw <= cb) + (c.cw + kComputeWarps <= cb) : 0;
+  const bool load_cur = !chunk_rows && r.has_cur && c.cw == cur_warp;
   const float *kcur = p.kvcur + (((size_t)l * p.B + b) * 2) * p.kvdim + (size_t)g * D;
   const float *vcur = kcur + p.kvdim;
   const float *qb = p.qbuf + ((size_t)l * p.B + b) * p.qdim + (size_t)g * G * D;
@@ -2318,9 +2510,37 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   // current position's K and V rows (bf16)
   float *scr = c.act;
   uint16_t *cur = reinterpret_cast<uint16_t *>(c.act + kComputeWarps * G * (D + 2));
+  // after the merge weights (below): this warp's chunk rows, K [2][D] then V [2][D]
+  uint16_t *mine = reinterpret_cast<uint16_t *>(c.act + kComputeWarps * G * (D + 2) + D +
+                                                ((G * (kComputeWarps + 2) + 3) & ~3)) +
+                   (size_t)c.cw * 4 * D;
   float q[G][DPL], ck[DPL], cv[DPL];
   settle(c, 5, [&](bool &ok) {
     uint32_t wk[DPL], wv[DPL], wq[G][DPL];
+    if constexpr (CHUNK) {
+      if (nmine > 0) {
+        uint32_t rk[2][DPL], rv[2][DPL];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (j >= nmine) break;
+          const float *kr = p.kvcur + (((size_t)l * p.B + c.cw + j * kComputeWarps) * 2) * p.kvdim + (size_t)g * D;
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) {
+            rk[j][i] = px::ld_tf(kr + c.lane * DPL + i);
+            rv[j][i] = px::ld_tf(kr + p.kvdim + c.lane * DPL + i);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (j >= nmine) break;
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) {
+            mine[j * D + c.lane * DPL + i] = px::f2bf(tf_chk(rk[j][i], tag, ok));
+            mine[2 * D + j * D + c.lane * DPL + i] = px::f2bf(tf_chk(rv[j][i], tag, ok));
+          }
+        }
+      }
+    }
     if (load_cur) {
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
@@ -2385,6 +2605,9 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   if (load_cur && !c.sh->abort) {
     // one valid position; the block reads PW rows, rows past the first are masked
     attn_block<G, DPL, PB>(q, cur, cur + D, 1, c.lane, m, lsum, o);
+  }
+  if constexpr (CHUNK) {
+    if (nmine > 0 && !c.sh->abort) attn_block<G, DPL, PB>(q, mine, mine + 2 * D, nmine, c.lane, m, lsum, o);
   }
   // merge the warps
 #pragma unroll
@@ -2517,24 +2740,25 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   }
   return c.g;
 }
-template <int G, int DPL>
-__device__ __noinline__ uint32_t op_attn_t(CCtx c, const Instr I) { return attn_body<G, DPL>(c, I); }
+template <int G, int DPL, bool CHUNK>
+__device__ __noinline__ uint32_t op_attn_t(CCtx c, const Instr I) { return attn_body<G, DPL, CHUNK>(c, I); }
 
+template <bool CHUNK>
 __device__ __forceinline__ uint32_t op_attn(const CCtx &c, const Instr &I) {
   const int G = c.p.nq / c.p.nkv;
   if (c.p.d == 64) {
     switch (G) {
-      case 1: return op_attn_t<1, 2>(c, I);
-      case 2: return op_attn_t<2, 2>(c, I);
-      case 4: return op_attn_t<4, 2>(c, I);
-      default: return op_attn_t<8, 2>(c, I);
+      case 1: return op_attn_t<1, 2, CHUNK>(c, I);
+      case 2: return op_attn_t<2, 2, CHUNK>(c, I);
+      case 4: return op_attn_t<4, 2, CHUNK>(c, I);
+      default: return op_attn_t<8, 2, CHUNK>(c, I);
     }
   }
   switch (G) {
-    case 1: return op_attn_t<1, 4>(c, I);
-    case 2: return op_attn_t<2, 4>(c, I);
-    case 4: return op_attn_t<4, 4>(c, I);
-    default: return op_attn_t<8, 4>(c, I);
+    case 1: return op_attn_t<1, 4, CHUNK>(c, I);
+    case 2: return op_attn_t<2, 4, CHUNK>(c, I);
+    case 4: return op_attn_t<4, 4, CHUNK>(c, I);
+    default: return op_attn_t<8, 4, CHUNK>(c, I);
   }
 }
 
@@ -2547,6 +2771,14 @@ __device__ __forceinline__ uint32_t op_attn(const CCtx &c, const Instr &I) {
     case 16: c.g = fn<NB, 16>(c, I); break;       \
     default: c.g = fn<NB, 32>(c, I); break;       \
   }
+#define MK_DISPATCH_R1(fn, R, c, I)               \
+  switch (R) {                                    \
+    case 2: c.g = fn<2>(c, I); break;             \
+    case 4: c.g = fn<4>(c, I); break;             \
+    case 8: c.g = fn<8>(c, I); break;             \
+    case 16: c.g = fn<16>(c, I); break;           \
+    default: c.g = fn<32>(c, I); break;           \
+  }
 
 __device__ __forceinline__ int &sh_stat(CCtx &c) { return c.sh->stat_cwait; }
 
@@ -2558,14 +2790,16 @@ __device__ __forceinline__ int &sh_stat(CCtx &c) { return c.sh->stat_cwait; }
 // (all zero) reaches the bodies through calls selected at run time.  TQO
 // (batched builds): QKV and the O projection may run as tensor-core tiles; a
 // build of its own, since the extra op bodies raise every body's spills.
-template <int RH_, int RO_, int RD_, int G_, int DPL_, bool TQO_ = false, bool SPL_ = false>
+template <int RH_, int RO_, int RD_, int G_, int DPL_, bool TQO_ = false, bool SPL_ = false, bool TP_ = false>
 struct Spec {
   static constexpr bool fixed = RH_ > 0;
   static constexpr bool TQO = TQO_;
   static constexpr bool SPL = SPL_;  // batch 1: split pages for rows of 2048 / 4096 columns
+  static constexpr bool TP = TP_;    // the tensor-parallel rank build (shape-generic, batch 1)
   static constexpr int RH = RH_, RO = RO_, RD = RD_, G = G_, DPL = DPL_;
 };
 using SpecGeneric = Spec<0, 0, 0, 0, 0>;
+using SpecGenericTP = Spec<0, 0, 0, 0, 0, false, false, true>;
 
 // Ops that start before their producers are known to be done (bit op): all
 // of them (measured: 682 us/step, against 697 with attention and the output
@@ -2670,9 +2904,9 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         else MK_DISPATCH_R(op_qkv, NB, p.Rh, c, I);
         break;
       case OP_ATTN:
-        if constexpr (kInline) c.g = attn_body<S::G, S::DPL>(c, I);
-        else if constexpr (S::fixed) c.g = op_attn_t<S::G, S::DPL>(c, I);
-        else c.g = op_attn(c, I);
+        if constexpr (kInline) c.g = attn_body<S::G, S::DPL, false>(c, I);
+        else if constexpr (S::fixed) c.g = op_attn_t<S::G, S::DPL, (NB > 1)>(c, I);
+        else c.g = op_attn<(NB > 1)>(c, I);
         break;
       case OP_OPROJ:
         if constexpr (NB > 1 && S::fixed && S::TQO) {
@@ -2683,7 +2917,11 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         }
         if constexpr (kInline) c.g = oproj_body<NB, S::RO, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_oproj<NB, S::RO>(c, I);
-        else MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);
+        else if constexpr (S::TP) {
+          MK_DISPATCH_R1(op_oproj_tp, p.Ro, c, I);
+        } else {
+          MK_DISPATCH_R(op_oproj, NB, p.Ro, c, I);
+        }
         break;
       case OP_GATEUP:
         if constexpr (NB > 1 && S::fixed) {
@@ -2694,7 +2932,11 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         }
         if constexpr (kInline) c.g = gateup_body<NB, S::RH, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_gateup<NB, S::RH>(c, I);
-        else MK_DISPATCH_R(op_gateup, NB, p.Rh, c, I);
+        else if constexpr (S::TP) {
+          MK_DISPATCH_R1(op_gateup_tp, p.Rh, c, I);
+        } else {
+          MK_DISPATCH_R(op_gateup, NB, p.Rh, c, I);
+        }
         break;
       case OP_DOWN:
         if constexpr (NB > 1 && S::fixed) {
@@ -2705,7 +2947,11 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         }
         if constexpr (kInline) c.g = down_body<NB, S::RD, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_down<NB, S::RD>(c, I);
-        else MK_DISPATCH_R(op_down, NB, p.Rd, c, I);
+        else if constexpr (S::TP) {
+          MK_DISPATCH_R1(op_down_tp, p.Rd, c, I);
+        } else {
+          MK_DISPATCH_R(op_down, NB, p.Rd, c, I);
+        }
         break;
       case OP_LMHEAD:
         if constexpr (NB > 1 && S::fixed) {
@@ -2716,7 +2962,11 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         }
         if constexpr (kInline) c.g = lmhead_body<NB, S::RH, S::SPL>(c, I);
         else if constexpr (S::fixed) c.g = op_lmhead<NB, S::RH>(c, I);
-        else MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I);
+        else if constexpr (S::TP) {
+          MK_DISPATCH_R1(op_lmhead_tp, p.Rh, c, I);
+        } else {
+          MK_DISPATCH_R(op_lmhead, NB, p.Rh, c, I);
+        }
         break;
       default: break;
     }
@@ -2730,7 +2980,16 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
       if (p.mode & MODE_EVENT) {
         for (int k = 0; k < I.sig_n; ++k) event_signal(p, I.sig_ctr + k, c.epoch);
       } else {
-        for (int k = 0; k < I.sig_n; ++k) px::red_relaxed_add(p.ctr + I.sig_ctr + k, 1u);
+        if constexpr (S::TP) {
+          // the O and down partials feed every rank: count them on every rank
+          const bool all = I.op == OP_OPROJ || I.op == OP_DOWN;
+          for (int rr = 0; rr < (all ? p.tp_n : 1); ++rr) {
+            unsigned *ctr = all ? p.tp_peers[rr].ctr : p.ctr;
+            for (int k = 0; k < I.sig_n; ++k) px::red_relaxed_add(ctr + I.sig_ctr + k, 1u);
+          }
+        } else {
+          for (int k = 0; k < I.sig_n; ++k) px::red_relaxed_add(p.ctr + I.sig_ctr + k, 1u);
+        }
       }
     }
     if (tr && c.ctid == 0) {
@@ -2745,7 +3004,12 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
 
 // ============================================================== kernel
 template <int NB, bool RAW, class S>
-__global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_constant__ KParams p) {
+__global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_constant__ KParams pk) {
+  // the tensor-parallel build runs an emulated group in one launch: CTA
+  // blocks of tp_ctas each run one rank, with that rank's parameters
+  const KParams &p = S::TP ? pk.tp_params[blockIdx.x / pk.tp_ctas] : pk;
+  const unsigned cta = S::TP ? blockIdx.x % (unsigned)pk.tp_ctas : blockIdx.x;
+  const unsigned ncta = S::TP ? (unsigned)pk.tp_ctas : gridDim.x;
   extern __shared__ __align__(128) uint8_t smem[];
   const int NP = p.num_pages;
   uint8_t *pages = smem;
@@ -2781,7 +3045,15 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   if (threadIdx.x < (unsigned)p.B) {
     // this step's inputs, clamped once (out-of-range values are reported)
     const int b = threadIdx.x;
-    const int t = __ldcg(p.tokens + b), pos = __ldcg(p.positions + b);  // tokens may alias next_tokens
+    int t, pos;
+    if (p.chunk_n > 0) {  // prompt chunk: consecutive tokens of one sequence
+      const int j = min(b, p.chunk_n - 1);
+      t = __ldcg(p.tokens + j);
+      pos = p.chunk_pos0 + j;
+    } else {
+      t = __ldcg(p.tokens + b);  // tokens may alias next_tokens
+      pos = __ldcg(p.positions + b);
+    }
     if (t < 0 || t >= p.V || pos < 0 || pos >= p.max_seq) record_error(p, MK_ERR_DEVICE_INPUT, b, t, pos, 0);
     sh->tok[b] = (t < 0 || t >= p.V) ? 0 : t;
     sh->pos[b] = pos < 0 ? 0 : (pos >= p.max_seq ? p.max_seq - 1 : pos);
@@ -2801,8 +3073,8 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   if constexpr (NB > 1) px::tc_fence_after();
   const unsigned epoch = *reinterpret_cast<volatile unsigned *>(p.epoch);
   Queue q;
-  q.base = p.instrs + p.q_off[blockIdx.x];
-  q.len = p.q_len[blockIdx.x];
+  q.base = p.instrs + p.q_off[cta];
+  q.len = p.q_len[cta];
   if (warp < kLoaders) {
     // the dynamic queue is claimed by one loader only
     const bool dyn = (p.mode & MODE_DYNAMIC) != 0;
@@ -2839,7 +3111,7 @@ __global__ void __launch_bounds__(kThreads, 1) interp_kernel(const __grid_consta
   if (threadIdx.x == 0 && (p.mode & MODE_FINAL_LAUNCH)) {
     __threadfence();
     const unsigned old = px::atom_add_acq_rel(p.ctr + p.exit_ticket, 1u);
-    if (old == epoch * gridDim.x - 1u) {
+    if (old == epoch * ncta - 1u) {
       // every CTA of the step has finished: advance the step number
       atomicExch(p.epoch, epoch + 1u);
     }

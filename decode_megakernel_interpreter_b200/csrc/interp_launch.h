@@ -31,6 +31,8 @@ int ring_pages(int smem_optin, size_t act_floats);
 const void *interp_kernel_for(const KParams &p, bool specialised, int nb, bool tqo, int *variant);
 // The raw-layout variant (weights read in the caller's layout).
 const void *interp_kernel_raw();
+// the tensor-parallel rank build (shape-generic, batch 1, static queues)
+const void *interp_kernel_tp();
 // Allow `smem` bytes of dynamic shared memory for fn and report how many of
 // its CTAs fit on one SM.
 cudaError_t interp_prepare(const void *fn, int smem, int *blocks_per_sm);

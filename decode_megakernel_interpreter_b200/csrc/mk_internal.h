@@ -92,6 +92,17 @@ enum : uint32_t {
   MODE_EVENT = 16u,       // with MODE_DYNAMIC: the global queue holds ready instructions only
 };
 
+// Tensor parallelism: where the outputs of one rank that the other ranks read
+// go -- every rank's own copies of these buffers (device pointers; on one GPU
+// for an emulated group, peer pointers over NVLink for a group of GPUs).
+struct TpPeer {
+  float *opart;                  // [L][tp_n][B][H] O-projection partials, by producing rank
+  float *dpart;                  // [L][ndp][B][H] down-projection pieces (rank r: pieces r*ndp_local ..)
+  unsigned *ctr;                 // counters (the O and down counters count every rank's producers)
+  unsigned long long *arg_val;   // [B][n_lm] argmax slots (rank r: slots r*n_lm_local ..)
+  unsigned long long *arg_idx;
+};
+
 // Status words (device): [0] first error code, [1] abort flag, [2..7] detail.
 constexpr int kStatusWords = 8;
 
@@ -161,6 +172,24 @@ struct KParams {
   unsigned long long *trace;  // [n_instr][5]
   uint32_t mode;
   int stage_filter;       // per-op path: run only this (layer*5 + stage), -1 = all
+  // tensor parallelism (tp_n > 1, the TP interpreter build only): this rank
+  // computes the heads, FFN columns and vocabulary rows of its shard; the O
+  // projection and the down projection write partial sums into every rank's
+  // opart / dpart (summed by the consumers in a fixed order), the gate/up
+  // instructions materialise x_mid as this rank's residual copy, and the LM
+  // head writes its rows' logits and argmax slots.  Unused otherwise.
+  int tp_n, tp_rank, tp_ctas;     // ranks, this rank, CTAs per rank
+  const KParams *tp_params;       // emulated group (one launch): every rank's parameters, by CTA
+  const TpPeer *tp_peers;         // [tp_n]
+  float *opart;                   // this rank's copy [L][tp_n][B][H]
+  int ndp_local, n_lm_local;      // this rank's down pieces per layer and LM-head instructions
+  int n_gu_layer;                 // gate/up instructions per layer (each stores a slice of x_mid)
+  int lm_row0, V_lm;              // this rank's LM-head rows [lm_row0, lm_row0 + V_lm)
+  // prompt chunks (chunk_n > 0; see mk_prefill): row b of the step is prompt
+  // token j = min(b, chunk_n - 1) at position chunk_pos0 + j, and every row
+  // uses KV sequence kv_seq0; rows past chunk_n - 1 repeat the last token and
+  // write neither the cache nor logits.  0 for decode steps.
+  int chunk_n, chunk_pos0, kv_seq0;
   // io
   const int *tokens, *positions;
   float *logits;

@@ -264,6 +264,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       Instr I = mk_instr(OP_GATEUP, l);
       I.a = cg[i].first;
       I.b = cg[i].count;
+      I.c = (uint32_t)i;  // its index in the layer (tensor parallelism: its slice of x_mid)
       I.wait_ctr = p.ctr_o(l);
       I.wait_cnt = n_o[l];
       int row0 = cg[i].first * half, row1 = (cg[i].first + cg[i].count) * half;  // act rows
@@ -273,6 +274,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
       for (int k = k0; k <= k1; ++k) gu_per_piece[k]++;
       all.push_back({I, (int64_t)cg[i].count * gu_unit_bytes, l * 8 + ST_GATEUP, (int)i});
     }
+    p.n_gu = (int)cg.size();
     // down projection, K-split into pieces; each piece waits only for the
     // gate/up instructions that produce its K range
     int total = p.ndp * p.P_dp;

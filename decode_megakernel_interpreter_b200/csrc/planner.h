@@ -65,6 +65,7 @@ struct Plan {
   int n_counters = 0;
   unsigned attn_ticket0 = 0, arg_ticket0 = 0, exit_ticket = 0, dyn_head = 0, ev_tail = 0;
   int n_lm = 0;
+  int n_gu = 0;  // gate/up instructions per layer
   int64_t weight_bytes = 0;  // weight bytes streamed per step
 
   unsigned ctr_qkv(int l) const { return l * ctr_per_layer + 0; }

@@ -224,6 +224,36 @@ int mk_decode_step(mk_handle *h, const int32_t *tokens, const int32_t *positions
                    float *logits_out, int32_t *next_tokens_out, void *stream);
 
 /*
+ * mk_prefill ("One Megakernel is Not Enough" digest, 首次出现的概念: prefill,
+ * which processes a prompt's tokens together, against decode, one token per
+ * step; the digest notes that prefill is usually left to conventional
+ * execution -- here it runs in the same persistent interpreter): write the K
+ * and V rows of prompt tokens pos0 .. pos0+n_tokens-1 of KV sequence `seq`
+ * and return the logits and greedy next token of the last one.
+ *  - seq             0 <= seq < max_batch: the cache sequence to fill.
+ *  - tokens          device int32 [n_tokens]: the prompt tokens, in order.
+ *  - n_tokens, pos0  n_tokens >= 1, pos0 >= 0, pos0 + n_tokens <= max_seq;
+ *                    rows 0 .. pos0-1 of the sequence must already hold its
+ *                    earlier keys and values (e.g. an earlier mk_prefill).
+ *  - logits_out      device float [vocab]: the last token's logits, or NULL.
+ *  - next_token_out  device int32 [1]: their argmax (lowest index on ties).
+ *  - stream          cudaStream_t (as void*).
+ * With a batched plan (batch B > 1, a shape with a batched build) the prompt
+ * runs in chunks of up to B consecutive tokens, one launch per chunk: the
+ * chunk's tokens are the B rows of the tensor-core matrix instructions, and
+ * token j of a chunk attends over the cache rows before the chunk and the
+ * chunk's rows 0..j (this launch's K/V exchange).  With a batch-1 plan, one
+ * token per launch (any shape).  Needs a plan with a one-launch exec_mode;
+ * each launch counts as a step of the plan (like mk_decode_step).
+ * Asynchronous and stream-ordered.  Errors: MK_ERR_INVALID_ARG,
+ * MK_ERR_NOT_PLANNED, MK_ERR_OUT_OF_MEMORY (its scratch, allocated with the
+ * plan on first use), MK_ERR_LAUNCH, MK_ERR_CUDA; device-side ones at the
+ * next mk_get_status.
+ */
+int mk_prefill(mk_handle *h, int32_t seq, const int32_t *tokens, int32_t n_tokens, int32_t pos0,
+               float *logits_out, int32_t *next_token_out, void *stream);
+
+/*
  * mk_get_status ("Hazy megakernel summary", section 四(二) 同步: the counters
  * in global memory that replace kernel boundaries; every wait on them is
  * bounded here, and a wait that gives up is reported by this call):
@@ -239,6 +269,46 @@ const char *mk_status_string(int code);
 /* Free everything the handle owns (synchronises the device first).  Borrowed
    weights and KV are untouched.  NULL is allowed. */
 void mk_destroy(mk_handle *h);
+
+/* ------------------------------------------------------------------ tensor parallelism */
+/*
+ * A tensor-parallel group ("Mirage Persistent Kernel" article, part 1: the
+ * matrix products split across GPUs, with each chunk of the collective that
+ * follows depending only on the tile that produces it).  Rank r of n holds
+ * query heads [r nq/n, (r+1) nq/n) and their KV heads, FFN columns
+ * [r F/n, (r+1) F/n) and vocabulary rows [r V/n, (r+1) V/n): QKV and gate/up
+ * are split by output rows (no exchange), the O and down projections by
+ * input columns -- each of their pages stores its partial sums into every
+ * rank's partial buffers (the all-reduce, chunked by page; consumers sum the
+ * ranks' partials in rank order) -- and the LM head by vocabulary rows, with
+ * the argmax merged over every rank's candidates.  This build emulates the
+ * group on one GPU: one cooperative launch of n * (SMs / n) CTAs runs every
+ * rank's plan with its own parameters and buffers (ranks whose kernels wait
+ * on one another must share a launch on one GPU); the stores into the other
+ * ranks' buffers are the ones a group of GPUs makes over NVLink.
+ */
+typedef struct mk_tp_group mk_tp_group;
+
+/*
+ * mk_tp_create: n_ranks in {2, 4, 8}, dividing n_q_heads, n_kv_heads, ffn and
+ * vocab.  Weights and the KV cache as for mk_create (borrowed; each rank
+ * reads its heads' rows of the caller's cache in place, and copies its column
+ * shards of Wo and W_down).  Errors: MK_ERR_INVALID_ARG,
+ * MK_ERR_UNSUPPORTED_SHAPE, MK_ERR_OUT_OF_MEMORY, MK_ERR_CUDA.
+ */
+int mk_tp_create(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv, int32_t n_ranks,
+                 mk_tp_group **out);
+/* Plan every rank (opts: batch 1, static queues, a one-launch exec_mode; the
+   ranks run the shape-generic build on SMs / n CTAs each). */
+int mk_tp_plan(mk_tp_group *g, const mk_plan_opts *opts);
+/* One decode step of the group (arguments as mk_decode_step, batch 1);
+   asynchronous, stream-ordered.  logits_out receives every rank's rows. */
+int mk_tp_decode_step(mk_tp_group *g, const int32_t *tokens, const int32_t *positions, float *logits_out,
+                      int32_t *next_tokens_out, void *stream);
+/* Synchronise and return the first device-side error of any rank (then the
+   group must be planned again), or MK_OK. */
+int mk_tp_get_status(mk_tp_group *g, void *stream);
+void mk_tp_destroy(mk_tp_group *g);
 
 /* ------------------------------------------------------------------ introspection */
 typedef struct {
