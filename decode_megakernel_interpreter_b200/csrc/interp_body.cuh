@@ -557,7 +557,8 @@ __device__ __forceinline__ PageSrc page_src(const KParams &p, const Shared *sh, 
       }
       s.a = p.lm_head + (size_t)I.a * p.Rh * p.H;
       const int r_last = (int)(I.a + I.b - 1) * p.Rh;
-      s.last = (uint32_t)min(p.Rh, p.V - r_last) * p.H * 2;
+      const int rows = p.tp_n > 1 ? p.V_lm : p.V;  // a tensor-parallel rank: its vocabulary rows
+      s.last = (uint32_t)min(p.Rh, rows - r_last) * p.H * 2;
       break;
     }
     case OP_ATTN: {
