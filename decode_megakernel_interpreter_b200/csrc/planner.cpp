@@ -707,6 +707,24 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
           I = &p.instrs[p.q_off[cta] + qi++];
         }
         if (I->op == OP_NOP) continue;
+        std::vector<Range> rd, wr, mrd, mwr;
+        rw_sets(req, p, *I, rd, wr, mrd, mwr);
+        // the kernel starts every instruction at once and loads its inputs
+        // before it knows its producers are done, telling this step's words
+        // from stale ones by a 2-bit step tag: that is sound only if a word
+        // it can meet was written this step or the step before (never two
+        // or more steps back, whose tag could alias)
+        for (auto &r : rd)
+          for (int64_t e = r.lo; e < r.hi; ++e) {
+            const uint32_t st = stamp[L.base[r.buf] + e].load(std::memory_order_relaxed);
+            if (st != epoch && st + 1 != epoch) {
+              char b[256];
+              snprintf(b, sizeof b, "step %u: instruction %d (op %d layer %d) could meet an element of buffer %d "
+                       "last written at step %u (its tag would alias)", epoch, I->seq, I->op, I->layer, r.buf, st);
+              fail(b);
+              return;
+            }
+          }
         if (I->wait_ctr != kNoCounter) {
           uint64_t target = (uint64_t)epoch * I->wait_cnt;
           auto t0 = std::chrono::steady_clock::now();
@@ -723,8 +741,6 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
           }
         }
         pause();
-        std::vector<Range> rd, wr, mrd, mwr;
-        rw_sets(req, p, *I, rd, wr, mrd, mwr);
         if (!check_reads(rd, *I)) return;
         pause();
         do_writes(wr, *I);
