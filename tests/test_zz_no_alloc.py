@@ -90,6 +90,52 @@ def test_noalloc_matches_handle_path_on_two_calls(name, context):
     eng.close()
 
 
+def test_noalloc_call_replays_from_a_cuda_graph():
+    """After a first call (which uploads the plan and tables and
+    synchronises), a call with the same arguments only enqueues device work:
+    captured once in a CUDA graph, its replays at later positions (updated in
+    place in the captured position buffer) give the handle path's results."""
+    shape = synth.TINY
+    context, max_seq = 64, 80
+    model, dev, k, v = _setup(shape, max_seq, context)
+    kc_a, vc_a = harness.upload_kv(k, v)
+    kc_b, vc_b = harness.upload_kv(k, v)
+    eng = harness.make_engine(shape, dev, kc_a, vc_a, 1, max_seq)
+    eng.plan()
+    cfg, w, kv, _keep = _abi_structs(shape, dev, kc_b, vc_b, max_seq)
+    t_a = torch.tensor([7], dtype=torch.int32, device="cuda")
+    t_b = t_a.clone()
+    pos_a = torch.tensor([context], dtype=torch.int32, device="cuda")
+    pos_b = pos_a.clone()
+    logits_a = torch.empty(1, shape.vocab, device="cuda")
+    logits_b = torch.empty(1, shape.vocab, device="cuda")
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):  # the first call: uploads, synchronises
+        rc = mk.mk_decode_step_noalloc(cfg, w, kv, t_b.data_ptr(), pos_b.data_ptr(), logits_b.data_ptr(),
+                                       t_b.data_ptr(), side.cuda_stream)
+        assert rc == mk.MK_OK
+    side.synchronize()
+    eng.decode_step(t_a, pos_a, logits_a, t_a)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(logits_b.cpu().numpy(), logits_a.cpu().numpy())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        rc = mk.mk_decode_step_noalloc(cfg, w, kv, t_b.data_ptr(), pos_b.data_ptr(), logits_b.data_ptr(),
+                                       t_b.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == mk.MK_OK
+    for step in range(1, 4):
+        pos_a.fill_(context + step)
+        pos_b.fill_(context + step)
+        graph.replay()
+        eng.decode_step(t_a, pos_a, logits_a, t_a)
+        torch.cuda.synchronize()
+        assert eng.status() == mk.MK_OK
+        np.testing.assert_array_equal(logits_b.cpu().numpy(), logits_a.cpu().numpy())
+        assert int(t_b.item()) == int(t_a.item())
+    del graph
+    eng.close()
+
+
 def test_noalloc_rejects_oversized_and_bad_arguments():
     shape = synth.TINY
     model, dev, k, v = _setup(shape, 16, 8)
