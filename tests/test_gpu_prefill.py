@@ -63,9 +63,10 @@ def continue_decode(eng, hs, kc, vc, b, tok, pos, steps, chk):
         tok, pos = gn, pos + 1
 
 
-def test_tiny_prompt_one_token_per_launch():
+@pytest.mark.parametrize("sched", ["static", "dynamic", "event"])
+def test_tiny_prompt_one_token_per_launch(sched):
     """The tiny configuration's 64-token prompt on an empty cache, batch-1
-    plan (one launch per token), then 8 decode steps."""
+    plan (one launch per token; each scheduling mode), then 8 decode steps."""
     s = synth.TINY
     w = synth.WORKLOADS["tiny"]
     prompt = [int(t) for t in synth.prompt_tokens(w)]
@@ -74,7 +75,7 @@ def test_tiny_prompt_one_token_per_launch():
     kc, vc = harness.upload_kv(hs.k, hs.v)
     eng = harness.make_engine(s, dev, kc, vc, 1, 96)
     try:
-        eng.plan(batch=1)
+        eng.plan(batch=1, sched=sched)
         toks = torch.tensor(prompt, dtype=torch.int32, device="cuda")
         logits = torch.empty(s.vocab, dtype=torch.float32, device="cuda")
         nxt = torch.empty(1, dtype=torch.int32, device="cuda")

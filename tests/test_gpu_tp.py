@@ -19,7 +19,7 @@ import torch
 import decode_megakernel_interpreter_b200 as mk
 from decode_megakernel_interpreter_b200 import harness
 import synth
-from gpu_common import HostSetup, StepCheck, kv_row_mismatch
+from gpu_common import NORM_SIGMA, HostSetup, StepCheck, kv_row_mismatch
 
 
 def llama1b_2layer():
@@ -27,11 +27,12 @@ def llama1b_2layer():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("n_ranks", [2, 4, 8])
-def test_llama1b_shape_tp_group(n_ranks):
+@pytest.mark.parametrize("n_ranks,norm_sigma", [(2, 0.0), (4, 0.0), (8, 0.0), (2, NORM_SIGMA)],
+                         ids=["tp2", "tp4", "tp8", "tp2_seeded_norms"])
+def test_llama1b_shape_tp_group(n_ranks, norm_sigma):
     s = llama1b_2layer()
     max_seq = 160
-    hs = HostSetup(s, 1, max_seq)
+    hs = HostSetup(s, 1, max_seq, synth.make_model(s, norm_sigma=norm_sigma))
     hs.fill_prefix([100])
     dev = harness.upload_model(hs.model, s.tied)
     kc, vc = harness.upload_kv(hs.k, hs.v)
