@@ -688,6 +688,13 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   k.part_ml = part_ml;
   k.obuf = h->obuf;
   k.xres = h->xres;
+  // batched tensor-core plans: the next layer's input, summed once per down tile
+  if (p.tensor) {
+    float *xin = nullptr;
+    if ((rc = dalloc(h->plan_allocs, &xin, (size_t)s.L * B * s.H))) return rc;
+    k.xin = xin;
+    k.dn_ticket0 = p.dn_ticket0;
+  }
   k.actb = h->actb;
   k.dpart = h->dpart;
   k.arg_val = arg_val;
@@ -879,6 +886,7 @@ extern "C" int mk_get_status(mk_handle *h, void *stream) {
     if (e == cudaSuccess) e = cudaMemset(h->kp.part_ml, 0, 8 * L * B * nq * S * 2);
     if (e == cudaSuccess) e = cudaMemset(h->kp.arg_val, 0, 8 * B * h->plan.n_lm);
     if (e == cudaSuccess) e = cudaMemset(h->kp.arg_idx, 0, 8 * B * h->plan.n_lm);
+    if (e == cudaSuccess && h->kp.xin) e = cudaMemset(h->kp.xin, 0, sizeof(float) * L * B * h->shape.H);
     if (e == cudaSuccess) e = cudaMemcpy(h->ctr_epoch, &one, sizeof one, cudaMemcpyHostToDevice);
   }
   if (e != cudaSuccess) {

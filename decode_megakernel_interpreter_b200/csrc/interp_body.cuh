@@ -993,8 +993,12 @@ __device__ void stage_norm(CCtx &c, int l, const uint16_t *gamma, bool from_xres
           const int e4 = c.ctid + it * kComputeThreads;
           if (e4 < n4) {
             if (b == 0) gws[it] = __ldg(reinterpret_cast<const uint2 *>(gamma) + e4);  // with x: one round trip
-            xs[i][it] = from_xres_only ? ll_load4(c.epoch, p.xres + ((size_t)l * p.B + b) * H + e4 * 4, ok)
-                                       : layer_input4(p, c.epoch, l, b, tok, e4, ok);
+            if (from_xres_only)
+              xs[i][it] = ll_load4(c.epoch, p.xres + ((size_t)l * p.B + b) * H + e4 * 4, ok);
+            else if (NB > 1 && p.xin && l > 0)  // summed once by the down tiles
+              xs[i][it] = ll_load4(c.epoch, p.xin + ((size_t)(l - 1) * p.B + b) * H + e4 * 4, ok);
+            else
+              xs[i][it] = layer_input4(p, c.epoch, l, b, tok, e4, ok);
           }
         }
       }
@@ -1706,7 +1710,9 @@ __device__ __forceinline__ uint32_t oproj_body(CCtx c, const Instr I) {
           bool ok = true;
   #pragma unroll
           for (int b = 0; b < NB; ++b)
-            if (b < Bn) xin[b] = layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
+            if (b < Bn)
+              xin[b] = (p.xin && l > 0) ? tf_chk(px::ld_tf(p.xin + ((size_t)(l - 1) * Bn + b) * H + row), tag, ok)
+                                        : layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
           if (ok || !ll_retry(p, c.sh, r, 9)) break;
         }
   #pragma unroll
@@ -2115,6 +2121,47 @@ __device__ __forceinline__ uint32_t down_tc_body(CCtx c, const Instr I) {
       px::st_tf(dout + (size_t)b * H + row, v[b], tag);
     }
   });
+  if (!p.xin) return c.g;
+  // the last of the tile's K pieces to finish (a ticket; the pieces are
+  // tagged words, so no fence) sums the tile's rows once: x_in(l + 1) =
+  // x_mid + piece 0 + piece 1 + ... (the order every consumer used), so the
+  // next layer's consumers load one word per element instead of 1 + ndp
+  px::cbar();
+  if (c.ctid == 0) {
+    const unsigned t = p.dn_ticket0 + (unsigned)l * (unsigned)(H / 128) + I.a;
+    const unsigned old = px::atom_relaxed_add(p.ctr + t, 1u);
+    c.sh->flag = (old == c.epoch * (unsigned)p.ndp - 1u);
+  }
+  px::cbar();
+  if (c.sh->flag) {
+    const int r0 = (int)I.a * 128;
+    // 32 float4 per sequence in the tile's rows
+    for (int idx = c.ctid; idx < Bn * 32; idx += kComputeThreads) {
+      const int b = idx / 32, e = r0 + (idx % 32) * 4;
+      const size_t off = (size_t)b * H + e;
+      float4 x;
+      for (LLRetry rr;;) {
+        bool ok = true;
+        uint4 w[1 + kMaxDownPieces];
+        w[0] = px::ld_tf4(p.xres + (size_t)l * Bn * H + off);
+        for (int kk = 0; kk < p.ndp; ++kk) w[1 + kk] = px::ld_tf4(p.dpart + ((size_t)l * p.ndp + kk) * Bn * H + off);
+        x = tf_chk4(w[0], tag, ok);
+        for (int kk = 0; kk < p.ndp; ++kk) {
+          const float4 v = tf_chk4(w[1 + kk], tag, ok);
+          x.x += v.x;
+          x.y += v.y;
+          x.z += v.z;
+          x.w += v.w;
+        }
+        if (ok || !ll_retry(p, c.sh, rr, 10)) break;
+      }
+      float *dst = p.xin + (size_t)l * Bn * H + off;
+      px::st_tf(dst + 0, x.x, tag);
+      px::st_tf(dst + 1, x.y, tag);
+      px::st_tf(dst + 2, x.z, tag);
+      px::st_tf(dst + 3, x.w, tag);
+    }
+  }
   return c.g;
 }
 
@@ -2184,7 +2231,9 @@ __device__ __forceinline__ uint32_t oproj_tc_body(CCtx c, const Instr I) {
       bool ok = true;
 #pragma unroll
       for (int b = 0; b < NB; ++b)
-        if (b < Bn) xin[b] = layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
+        if (b < Bn)
+          xin[b] = (p.xin && l > 0) ? tf_chk(px::ld_tf(p.xin + ((size_t)(l - 1) * Bn + b) * H + row), tag, ok)
+                                    : layer_input1(p, tag, l, b, l == 0 ? read_tok(c.sh, b) : 0, row, ok);
       if (ok || !ll_retry(p, c.sh, r, 9)) break;
     }
 #pragma unroll
@@ -2975,7 +3024,10 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
     const bool abort_now = px::cbar_or(px::ld_volatile(&c.sh->abort) != 0);
     if (abort_now) break;
     // all of this CTA's outputs of the instruction are written: publish
-    const bool sig = I.sig_ctr != kNoCounter && (I.op != OP_ATTN || c.sh->flag);
+    // (merging instructions signal only when they merged: the last split of
+    // an attention group, the last piece of a tensor-core down tile)
+    const bool merging = I.op == OP_ATTN || (NB > 1 && I.op == OP_DOWN && p.xin);
+    const bool sig = I.sig_ctr != kNoCounter && (!merging || c.sh->flag);
     if (c.ctid == 0 && sig) {
       // a hint only: the data words carry this step's tag, so no fence
       if (p.mode & MODE_EVENT) {

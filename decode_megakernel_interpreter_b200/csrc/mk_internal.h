@@ -137,6 +137,12 @@ struct KParams {
   float *xres;                  // [L][B][H]
   float *actb;                  // [L][B][F]
   float *dpart;                 // [L][ndp][B][H]
+  // batched tensor-core plans: x_in of the next layer, [L][B][H], summed once
+  // per 128-row tile by the last of the tile's down pieces (ticket
+  // dn_ticket0 + l * (H / 128) + tile); null otherwise (consumers then sum
+  // the residual and the pieces themselves)
+  float *xin;
+  unsigned dn_ticket0;
   // tagged 64-bit words (step number << 32 | 32-bit value): values that may
   // be -inf, and indices
   unsigned long long *part_ml;  // [L][B][nq][S][2]

@@ -177,6 +177,9 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   p.exit_ticket = next++;
   p.dyn_head = next++;
   p.ev_tail = next++;
+  // tensor cores: one ticket per (layer, 128-row tile) of the down projection
+  p.dn_ticket0 = next;
+  if (req.tensor) next += (unsigned)(s.L * (s.H / 128));
   p.n_counters = (int)next;
 
   const int n = req.num_ctas;
@@ -281,7 +284,9 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
     int ord2 = 0;
     for (int k = 0; k < p.ndp; ++k) {
       int ck = (int)((int64_t)parts * (k + 1) / p.ndp - (int64_t)parts * k / p.ndp);
-      auto cd = split_even(dn_units, std::max(1, ck));
+      // tensor cores: one 128-row tile per instruction (the last piece of a
+      // tile to finish sums the tile's pieces: one signal per tile)
+      auto cd = split_even(dn_units, p.tensor ? dn_units : std::max(1, ck));
       for (auto &c : cd) {
         Instr I = mk_instr(OP_DOWN, l);
         I.a = c.first;
@@ -291,7 +296,7 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
         I.wait_cnt = gu_per_piece[k];
         I.sig_ctr = p.ctr_dn(l);
         I.sig_n = 1;
-        n_down[l]++;
+        if (!p.tensor || k == 0) n_down[l]++;
         all.push_back({I, (int64_t)c.count * dn_unit_bytes, l * 8 + ST_DOWN, ord2++});
       }
     }
@@ -421,7 +426,7 @@ namespace {
 
 // Element sets read and written by one instruction, as (buffer id, begin,
 // end) ranges over flattened per-step buffers.
-enum Buf { B_QKV, B_PART, B_O, B_XRES, B_ACT, B_DPART, B_ARG, B_NBUF };
+enum Buf { B_QKV, B_PART, B_O, B_XRES, B_ACT, B_DPART, B_ARG, B_XIN, B_NBUF };
 
 struct Range {
   int buf;
@@ -443,6 +448,7 @@ Layout make_layout(const PlanRequest &req, const Plan &p) {
   L.size[B_ACT] = (int64_t)s.L * s.F;
   L.size[B_DPART] = (int64_t)s.L * p.ndp * s.H;
   L.size[B_ARG] = p.n_lm;
+  L.size[B_XIN] = p.tensor ? (int64_t)s.L * s.H : 0;  // tensor cores: x_in of the next layer, summed once
   int64_t at = 0;
   for (int b = 0; b < B_NBUF; ++b) {
     L.base[b] = at;
@@ -455,6 +461,10 @@ void layer_input_reads(const PlanRequest &req, const Plan &p, int l, int64_t r0,
                        std::vector<Range> &rd) {
   if (l <= 0) return;  // embedding rows
   const Shape &s = req.s;
+  if (p.tensor) {  // summed once by the down tiles' last pieces
+    rd.push_back({B_XIN, (int64_t)(l - 1) * s.H + r0, (int64_t)(l - 1) * s.H + r1});
+    return;
+  }
   rd.push_back({B_XRES, (int64_t)(l - 1) * s.H + r0, (int64_t)(l - 1) * s.H + r1});
   for (int k = 0; k < p.ndp; ++k)
     rd.push_back({B_DPART, ((int64_t)(l - 1) * p.ndp + k) * s.H + r0,
@@ -507,7 +517,15 @@ void rw_sets(const PlanRequest &req, const Plan &p, const Instr &I, std::vector<
       rd.push_back({B_ACT, (int64_t)l * s.F + (int64_t)I.c * p.KCd,
                     (int64_t)l * s.F + (int64_t)(I.c + 1) * p.KCd});
       int64_t base = ((int64_t)l * p.ndp + I.c) * s.H;
-      wr.push_back({B_DPART, base + (int64_t)I.a * p.dn_rows_unit, base + (int64_t)(I.a + I.b) * p.dn_rows_unit});
+      const int64_t r0 = (int64_t)I.a * p.dn_rows_unit, r1 = (int64_t)(I.a + I.b) * p.dn_rows_unit;
+      wr.push_back({B_DPART, base + r0, base + r1});
+      if (p.tensor) {
+        // the tile's last piece: x_mid + every piece of the tile's rows -> x_in(l + 1)
+        merge_rd.push_back({B_XRES, (int64_t)l * s.H + r0, (int64_t)l * s.H + r1});
+        for (int k = 0; k < p.ndp; ++k)
+          merge_rd.push_back({B_DPART, ((int64_t)l * p.ndp + k) * s.H + r0, ((int64_t)l * p.ndp + k) * s.H + r1});
+        merge_wr.push_back({B_XIN, (int64_t)l * s.H + r0, (int64_t)l * s.H + r1});
+      }
       break;
     }
     case OP_LMHEAD:
@@ -559,6 +577,9 @@ std::string validate_plan(const PlanRequest &req, const Plan &p) {
       if (I->op == OP_ATTN) {
         // one signal per (sequence, kv head): counted once, by split 0's slot
         if (I->b == 0) n_prod[c]++;
+      } else if (I->op == OP_DOWN && p.tensor) {
+        // one signal per tile (the last of its pieces): counted by piece 0's slot
+        if (I->c == 0) n_prod[c]++;
       } else {
         n_prod[c]++;
       }
@@ -587,7 +608,8 @@ std::string validate_plan(const PlanRequest &req, const Plan &p) {
   for (auto *I : order) {
     std::vector<Range> rd, wr, mrd, mwr;
     rw_sets(req, p, *I, rd, wr, mrd, mwr);
-    if (I->op == OP_ATTN && I->b == 0) wr.insert(wr.end(), mwr.begin(), mwr.end());
+    if ((I->op == OP_ATTN && I->b == 0) || (I->op == OP_DOWN && p.tensor && I->c == 0))
+      wr.insert(wr.end(), mwr.begin(), mwr.end());
     for (auto &r : wr)
       for (int64_t e = r.lo; e < r.hi; ++e) wcount[L.base[r.buf] + e]++;
   }
@@ -745,16 +767,19 @@ std::string simulate_plan(const PlanRequest &req, const Plan &p, int steps, uint
         pause();
         do_writes(wr, *I);
         bool signal = true;
-        if (I->op == OP_ATTN || I->op == OP_LMHEAD) {
-          unsigned t = I->op == OP_ATTN ? p.attn_ticket0 + (I->layer * req.B + I->c) * req.s.nkv + I->a
-                                        : p.arg_ticket0;
-          uint32_t per = I->op == OP_ATTN ? (uint32_t)p.S : (uint32_t)p.n_lm;
+        if (I->op == OP_ATTN || I->op == OP_LMHEAD || (I->op == OP_DOWN && p.tensor)) {
+          // tickets: the last split (attention), LM-head instruction or piece
+          // of a down tile (tensor cores) merges
+          unsigned t = I->op == OP_ATTN   ? p.attn_ticket0 + (I->layer * req.B + I->c) * req.s.nkv + I->a
+                       : I->op == OP_DOWN ? p.dn_ticket0 + (unsigned)(I->layer * (req.s.H / 128) + I->a)
+                                          : p.arg_ticket0;
+          uint32_t per = I->op == OP_ATTN ? (uint32_t)p.S : I->op == OP_DOWN ? (uint32_t)p.ndp : (uint32_t)p.n_lm;
           uint32_t old = ctr[t].fetch_add(1, std::memory_order_acq_rel);
           signal = false;
           if (old == epoch * per - 1) {  // the last one merges
             if (!check_reads(mrd, *I)) return;
             do_writes(mwr, *I);
-            signal = I->op == OP_ATTN;
+            signal = I->op != OP_LMHEAD;
           }
         }
         if (signal && I->sig_ctr != kNoCounter)

@@ -64,6 +64,7 @@ struct Plan {
   int ctr_per_layer = 0;
   int n_counters = 0;
   unsigned attn_ticket0 = 0, arg_ticket0 = 0, exit_ticket = 0, dyn_head = 0, ev_tail = 0;
+  unsigned dn_ticket0 = 0;  // tensor cores: [L][H / 128] tickets of the down tiles' merges
   int n_lm = 0;
   int n_gu = 0;  // gate/up instructions per layer
   int64_t weight_bytes = 0;  // weight bytes streamed per step
