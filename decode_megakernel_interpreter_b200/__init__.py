@@ -142,6 +142,8 @@ def load(path: str = LIB_PATH):
     L.mk_host_plan.restype = i32
     L.mk_host_plan.argtypes = [P(mk_config), P(mk_plan_opts), i32, P(mk_instr_desc), i32, P(i32), P(i32), P(i32),
                                P(mk_plan_info), ctypes.c_char_p, sz]
+    L.mk_noalloc_get_status.restype = i32
+    L.mk_noalloc_get_status.argtypes = [vp, vp]
     L.mk_decode_step_noalloc.restype = i32
     L.mk_decode_step_noalloc.argtypes = [P(mk_config), P(mk_weights), P(mk_kv_cache), vp, vp, vp, vp, vp]
     L.mk_cost_params_default.restype = None
@@ -193,6 +195,13 @@ def mk_decode_step_noalloc(cfg: mk_config, weights: mk_weights, kv: mk_kv_cache,
     Raw pointers (ints); returns the status code."""
     return load().mk_decode_step_noalloc(ctypes.byref(cfg), ctypes.byref(weights), ctypes.byref(kv), tokens,
                                          positions, logits_out, next_tokens_out, stream)
+
+
+def mk_noalloc_get_status(stream: int | None) -> tuple:
+    """(status code, detail words) of the last allocation-free call on the current device."""
+    d = (ctypes.c_int32 * 6)()
+    rc = load().mk_noalloc_get_status(stream, d)
+    return rc, list(d)
 
 
 def mk_get_status(h: int, stream: int | None) -> int:

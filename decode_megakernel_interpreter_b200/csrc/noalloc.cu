@@ -71,6 +71,10 @@ int device_setup(int dev, DeviceSlot **out) {
   return MK_OK;
 }
 
+// the status words sit at this offset of the scratch (right after the step
+// number), where mk_noalloc_get_status reads them
+constexpr size_t kStatusAt = 256;
+
 struct Layout {
   size_t off = 0;
   size_t take(size_t bytes) {
@@ -128,6 +132,7 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
   const int B = 1, hd = s.d / 2;
   Layout lay;
   const size_t o_epoch = lay.take(4), o_status = lay.take(sizeof(int) * kStatusWords);
+  if (o_status != kStatusAt) return MK_ERR_CUDA;
   const size_t o_ctr = lay.take(sizeof(unsigned) * (size_t)p.n_counters);
   const size_t sync_end = lay.off;
   const size_t o_instr = lay.take(sizeof(Instr) * p.instrs.size());
@@ -304,4 +309,25 @@ extern "C" int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w,
                                                                                               : MK_ERR_CUDA;
   }
   return MK_OK;
+}
+
+extern "C" int mk_noalloc_get_status(void *stream, int32_t *detail) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  const DeviceSlot &slot = g_slots[dev];
+  if (!slot.ready) return MK_OK;  // no call on this device yet
+  int st[kStatusWords];
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaMemcpy(st, slot.scratch + kStatusAt, sizeof st, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MK_ERR_CUDA;
+  }
+  if (detail)
+    for (int i = 0; i < 6; ++i) detail[i] = st[0] ? st[i < 5 ? 2 + i : 1] : 0;
+  return st[0];
 }

@@ -396,12 +396,22 @@ int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
  *    scratch this shape needs exceeds MK_NOALLOC_SCRATCH_BYTES -- roughly the
  *    Llama-1B shape up to ~8K positions fits, the 8B shape does not),
  *    MK_ERR_LAUNCH, MK_ERR_CUDA.  Device-side errors of the step (timeout,
- *    clamped input) are not reported by this call.
+ *    clamped input) are reported by mk_noalloc_get_status until the next call
+ *    clears them.
  */
 #define MK_NOALLOC_SCRATCH_BYTES (16u << 20)
 int mk_decode_step_noalloc(const mk_config *cfg, const mk_weights *w, const mk_kv_cache *kv,
                            const int32_t *tokens, const int32_t *positions, float *logits_out,
                            int32_t *next_tokens_out, void *stream);
+
+/*
+ * mk_noalloc_get_status: synchronise `stream` and return the device-side
+ * error of the last mk_decode_step_noalloc on the current device
+ * (MK_ERR_TIMEOUT, MK_ERR_DEVICE_INPUT), MK_OK, or MK_ERR_CUDA; `detail`
+ * (host int32 [6] or NULL) as for mk_get_error_detail.  The next call clears
+ * the status.  MK_OK before any call on the device.
+ */
+int mk_noalloc_get_status(void *stream, int32_t *detail);
 
 #ifdef __cplusplus
 }

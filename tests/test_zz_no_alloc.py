@@ -136,6 +136,28 @@ def test_noalloc_call_replays_from_a_cuda_graph():
     eng.close()
 
 
+def test_noalloc_reports_device_side_errors():
+    """A token id outside the vocabulary is clamped and reported by
+    mk_noalloc_get_status; the next call clears it."""
+    shape = synth.TINY
+    context, max_seq = 40, 48
+    model, dev, k, v = _setup(shape, max_seq, context)
+    kc, vc = harness.upload_kv(k, v)
+    cfg, w, kv, _keep = _abi_structs(shape, dev, kc, vc, max_seq)
+    stream = torch.cuda.current_stream()
+    pos = torch.tensor([context], dtype=torch.int32, device="cuda")
+    nxt = torch.empty(1, dtype=torch.int32, device="cuda")
+    bad = torch.tensor([shape.vocab + 5], dtype=torch.int32, device="cuda")
+    rc = mk.mk_decode_step_noalloc(cfg, w, kv, bad.data_ptr(), pos.data_ptr(), None, nxt.data_ptr(), stream.cuda_stream)
+    assert rc == mk.MK_OK
+    code, detail = mk.mk_noalloc_get_status(stream.cuda_stream)
+    assert code == mk.MK_ERR_DEVICE_INPUT, (code, detail)
+    good = torch.tensor([3], dtype=torch.int32, device="cuda")
+    rc = mk.mk_decode_step_noalloc(cfg, w, kv, good.data_ptr(), pos.data_ptr(), None, nxt.data_ptr(), stream.cuda_stream)
+    assert rc == mk.MK_OK
+    assert mk.mk_noalloc_get_status(stream.cuda_stream)[0] == mk.MK_OK
+
+
 def test_noalloc_rejects_oversized_and_bad_arguments():
     shape = synth.TINY
     model, dev, k, v = _setup(shape, 16, 8)
