@@ -306,6 +306,19 @@ def plan_opts(batch: int = 1, kv_splits: int = 0, sched: str = "static", exec_mo
                         int(tensor_qkv_o), int(use_tcgen05))
 
 
+def _abi_model(weights: dict, kcache, vcache):
+    """The C structs (layer array, mk_weights, mk_kv_cache) over torch tensors;
+    the layer array must stay referenced while the structs are used."""
+    layers = weights["layers"]
+    lw = (mk_layer_weights * len(layers))()
+    for i, L in enumerate(layers):
+        for n, _ in mk_layer_weights._fields_:
+            setattr(lw[i], n, _ptr(L[n]))
+    lm = weights.get("lm_head")
+    w = mk_weights(_ptr(weights["embed"]), _ptr(lm) if lm is not None else None, _ptr(weights["final_norm"]), lw)
+    return lw, w, mk_kv_cache(_ptr(kcache), _ptr(vcache))
+
+
 class Engine:
     """Owns an mk handle over torch CUDA tensors.
 
@@ -319,15 +332,7 @@ class Engine:
     def __init__(self, shape, weights: dict, kcache, vcache, max_batch: int, max_seq: int):
         self.cfg = make_config(shape, max_batch, max_seq)
         self._keep = (weights, kcache, vcache)
-        layers = weights["layers"]
-        self._lw = (mk_layer_weights * len(layers))()
-        for i, L in enumerate(layers):
-            for n, _ in mk_layer_weights._fields_:
-                setattr(self._lw[i], n, _ptr(L[n]))
-        lm = weights.get("lm_head")
-        self._w = mk_weights(_ptr(weights["embed"]), _ptr(lm) if lm is not None else None,
-                             _ptr(weights["final_norm"]), self._lw)
-        self._kv = mk_kv_cache(_ptr(kcache), _ptr(vcache))
+        self._lw, self._w, self._kv = _abi_model(weights, kcache, vcache)
         self.h = mk_create(self.cfg, self._w, self._kv)
         self.info = None
 
@@ -391,15 +396,7 @@ class TpEngine:
     def __init__(self, shape, weights: dict, kcache, vcache, max_batch: int, max_seq: int, n_ranks: int):
         self.cfg = make_config(shape, max_batch, max_seq)
         self._keep = (weights, kcache, vcache)
-        layers = weights["layers"]
-        self._lw = (mk_layer_weights * len(layers))()
-        for i, L in enumerate(layers):
-            for n, _ in mk_layer_weights._fields_:
-                setattr(self._lw[i], n, _ptr(L[n]))
-        lm = weights.get("lm_head")
-        self._w = mk_weights(_ptr(weights["embed"]), _ptr(lm) if lm is not None else None,
-                             _ptr(weights["final_norm"]), self._lw)
-        self._kv = mk_kv_cache(_ptr(kcache), _ptr(vcache))
+        self._lw, self._w, self._kv = _abi_model(weights, kcache, vcache)
         g = ctypes.c_void_p()
         rc = load().mk_tp_create(ctypes.byref(self.cfg), ctypes.byref(self._w), ctypes.byref(self._kv), n_ranks,
                                  ctypes.byref(g))
