@@ -132,6 +132,41 @@ def test_llama1b_shape_chunked_prompt(n_prompt, pos0):
         eng.close()
 
 
+def test_llama8b_shape_prompt_second_sequence():
+    """The Llama-8B shape (2 layers; the split-page build, head_dim 128) with a
+    batch-1 plan on a two-sequence cache: an 8-token prompt of sequence 1,
+    one token per launch; sequence 0's rows untouched."""
+    base = synth.WORKLOADS["llama8b"].shape
+    s = dataclasses.replace(base, n_layers=2)
+    max_seq = 48
+    hs = HostSetup(s, 2, max_seq)
+    hs.fill_prefix([20, 12])
+    rng = np.random.default_rng(88)
+    prompt = [int(t) for t in rng.integers(0, s.vocab, 8)]
+    dev = harness.upload_model(hs.model, s.tied)
+    kc, vc = harness.upload_kv(hs.k, hs.v)
+    eng = harness.make_engine(s, dev, kc, vc, 2, max_seq)
+    try:
+        eng.plan(batch=1)
+        assert eng.info.kernel_variant == 1  # the shape-specialised (split-page) build
+        before = [harness.kv_row_to_host(kc, 0, p).copy() for p in range(12, 20)]
+        toks = torch.tensor(prompt, dtype=torch.int32, device="cuda")
+        logits = torch.empty(s.vocab, dtype=torch.float32, device="cuda")
+        nxt = torch.empty(1, dtype=torch.int32, device="cuda")
+        eng.prefill(1, toks, 12, logits, nxt)
+        assert eng.status() == mk.MK_OK, mk.mk_get_error_detail(eng.h)
+        for p, row in zip(range(12, 20), before):
+            np.testing.assert_array_equal(harness.kv_row_to_host(kc, 0, p), row)
+        gl = logits.cpu().numpy()
+        gn = int(nxt.item())
+        assert gn == int(np.argmax(gl))
+        chk = StepCheck()
+        check_prompt(hs, kc, vc, 1, prompt, 12, gl, gn, chk)
+        assert chk.id_mismatches <= chk.near_ties
+    finally:
+        eng.close()
+
+
 def test_prefill_rejects_bad_arguments():
     s = synth.TINY
     hs = HostSetup(s, 1, 40)
