@@ -366,9 +366,13 @@ def breakdown(eng, mk, info, tokens, pos0, logits, nxt):
                                      "mean_stage_us": float(stage.mean()), "mean_pages_us": float(pages.mean()),
                                      "mean_signal_us": float(sig.mean()),
                                      "mean_body_us": float((tr[m, 3] - tr[m, 1]).mean() / 1e3),
+                                     "mean_pages_per_instr": float(tr[m, 11].mean()),
                                      "consumer_page_waits": int((tr[m, 8] & 0xffffffff).sum()),
                                      "tagged_load_retries": int((tr[m, 8] >> 32).sum()),
                                      "loader_ring_full": int(tr[m, 9].sum())}
+        if (tr[m, 10] > 0).all():  # attention: the page loop and the merges after it
+            out[mk.OP_NAMES[int(op)]]["mean_page_loop_us"] = float(((tr[m, 10] - tr[m, 2]) / 1e3).mean())
+            out[mk.OP_NAMES[int(op)]]["mean_merge_us"] = float(((tr[m, 3] - tr[m, 10]) / 1e3).mean())
     return out
 
 

@@ -28,7 +28,7 @@ MK_ERR_OUT_OF_MEMORY = -8
 
 MK_SCHED_STATIC, MK_SCHED_DYNAMIC, MK_SCHED_EVENT = 0, 1, 2
 MK_EXEC_MEGAKERNEL, MK_EXEC_PER_OP, MK_EXEC_PER_OP_GRAPH, MK_EXEC_MEGAKERNEL_GENERIC = 0, 1, 2, 3
-MK_TRACE_WORDS = 10
+MK_TRACE_WORDS = 12
 
 OP_NAMES = {0: "nop", 1: "qkv", 2: "attn", 3: "oproj", 4: "gateup", 5: "down", 6: "lmhead"}
 

@@ -1090,10 +1090,12 @@ __device__ void stage_copy(CCtx &c, const float *src, size_t src_stride, int K, 
 }
 
 // acc[b][r] = dot(page row r, staged vector b) for R rows of KC = 8192/R
-// columns; every lane ends with every result.
+// columns; every lane ends with every result (up to 4 sequences; more use
+// mv_page_t).
 template <int NB, int R>
 __device__ __forceinline__ void mv_page(const uint8_t *page, const float *act, int act_stride, int B, int lane,
                                         float (&acc)[NB][R]) {
+  static_assert(NB <= 4, "more sequences: mv_page_t");
   constexpr int KC = kPageElems / R;
   constexpr int CH = KC / 8;  // 16-byte chunks per row
   const uint4 *pg = reinterpret_cast<const uint4 *>(page);
@@ -1101,51 +1103,6 @@ __device__ __forceinline__ void mv_page(const uint8_t *page, const float *act, i
   for (int b = 0; b < NB; ++b)
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[b][r] = 0.f;
-  if constexpr (NB > 4) {
-    // many sequences: one pass over the page per group of 4 sequences, so
-    // that the running sums of a pass stay in registers (the page is read
-    // from shared memory once per group)
-#pragma unroll
-    for (int b0 = 0; b0 < NB; b0 += 4) {
-      if (b0 >= B) break;
-      float part[4][R];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int r = 0; r < R; ++r) part[i][r] = 0.f;
-#pragma unroll 1
-      for (int j = 0; j < CH / 32; ++j) {
-        const int ch = lane + 32 * j;
-        uint4 w[R];
-#pragma unroll
-        for (int r = 0; r < R; ++r) w[r] = pg[r * CH + ch];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (b0 + i >= B) break;
-          const float4 *a = reinterpret_cast<const float4 *>(act + (size_t)(b0 + i) * act_stride);
-          const float4 a0 = a[ch], a1 = a[CH + ch];
-#pragma unroll
-          for (int r = 0; r < R; ++r) {
-            float t = part[i][r];
-            t = fmaf(px::bf_lo(w[r].x), a0.x, t);
-            t = fmaf(px::bf_hi(w[r].x), a0.y, t);
-            t = fmaf(px::bf_lo(w[r].y), a0.z, t);
-            t = fmaf(px::bf_hi(w[r].y), a0.w, t);
-            t = fmaf(px::bf_lo(w[r].z), a1.x, t);
-            t = fmaf(px::bf_hi(w[r].z), a1.y, t);
-            t = fmaf(px::bf_lo(w[r].w), a1.z, t);
-            t = fmaf(px::bf_hi(w[r].w), a1.w, t);
-            part[i][r] = t;
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int r = 0; r < R; ++r) acc[b0 + i][r] = px::warp_sum(part[i][r]);
-    }
-    return;
-  }
 #pragma unroll(CH / 32 > 2 ? 2 : CH / 32)
   for (int j = 0; j < CH / 32; ++j) {
     const int ch = lane + 32 * j;
@@ -1190,6 +1147,104 @@ __device__ __forceinline__ float pick(const float (&v)[R], int idx) {
   return out;
 }
 
+// Butterfly reduction of NV partial sums per lane over the warp, transposed:
+// afterwards v[0] of lane L holds the full sum of value index L >> (5 - log2 NV)
+// (each sum in 32 / NV lanes), after NV - 1 + log2(32 / NV) shuffles instead of
+// 5 per value.
+template <int NV>
+__device__ __forceinline__ void warp_sum_transposed(float (&v)[NV], int lane) {
+  static_assert(NV >= 1 && NV <= 32 && (NV & (NV - 1)) == 0, "power of two up to 32");
+  int n = NV;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    if (n > 1) {
+      const int hn = n / 2;
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < (NV > 1 ? NV / 2 : 1); ++i) {
+        if (i < hn) {
+          const float send = up ? v[i] : v[i + hn];
+          const float keep = up ? v[i + hn] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      n = hn;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+    }
+  }
+}
+constexpr int log2_pow2(int n) { return n <= 1 ? 0 : 1 + log2_pow2(n / 2); }
+
+// Row sums of a page for more than 4 sequences, kept transposed: v[grp] of
+// lane L is the sum of (sequence 4 * grp + i, row r) with i * R + r = L >> SH.
+// acc_row() fetches one by a shuffle, so a lane holds NB / 4 sums instead of
+// NB * R copies of all of them.
+template <int NB, int R>
+struct AccT {
+  static_assert(NB % 4 == 0 && 4 * R <= 32, "groups of 4 sequences, 4 * R sums per group");
+  static constexpr int SH = 5 - log2_pow2(4 * R);
+  float v[NB / 4];
+};
+template <int R, int NB>
+__device__ __forceinline__ float acc_row(const float (&acc)[NB][R], int b, int r) {
+  return pick<R>(acc[b], r);
+}
+// every lane of the warp must call this (a shuffle); r is taken modulo R
+template <int R, int NB>
+__device__ __forceinline__ float acc_row(const AccT<NB, R> &acc, int b, int r) {
+  return __shfl_sync(0xffffffffu, acc.v[b >> 2], (((b & 3) * R + (r & (R - 1))) << AccT<NB, R>::SH));
+}
+
+// mv_page for more than 4 sequences: one pass over the page per group of 4
+// sequences, so that the running sums of a pass stay in registers (the page
+// is read from shared memory once per group), then one transposed reduction
+// of the group's 4 * R sums
+template <int NB, int R>
+__device__ __forceinline__ void mv_page_t(const uint8_t *page, const float *act, int act_stride, int B, int lane,
+                                          AccT<NB, R> &acc) {
+  constexpr int KC = kPageElems / R;
+  constexpr int CH = KC / 8;  // 16-byte chunks per row
+  const uint4 *pg = reinterpret_cast<const uint4 *>(page);
+#pragma unroll
+  for (int b0 = 0; b0 < NB; b0 += 4) {
+    acc.v[b0 / 4] = 0.f;
+    if (b0 >= B) continue;
+    float part[4 * R];
+#pragma unroll
+    for (int i = 0; i < 4 * R; ++i) part[i] = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < CH / 32; ++j) {
+      const int ch = lane + 32 * j;
+      uint4 w[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) w[r] = pg[r * CH + ch];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (b0 + i >= B) break;
+        const float4 *a = reinterpret_cast<const float4 *>(act + (size_t)(b0 + i) * act_stride);
+        const float4 a0 = a[ch], a1 = a[CH + ch];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float t = part[i * R + r];
+          t = fmaf(px::bf_lo(w[r].x), a0.x, t);
+          t = fmaf(px::bf_hi(w[r].x), a0.y, t);
+          t = fmaf(px::bf_lo(w[r].y), a0.z, t);
+          t = fmaf(px::bf_hi(w[r].y), a0.w, t);
+          t = fmaf(px::bf_lo(w[r].z), a1.x, t);
+          t = fmaf(px::bf_hi(w[r].z), a1.y, t);
+          t = fmaf(px::bf_lo(w[r].w), a1.z, t);
+          t = fmaf(px::bf_hi(w[r].w), a1.w, t);
+          part[i * R + r] = t;
+        }
+      }
+    }
+    warp_sum_transposed<4 * R>(part, lane);
+    acc.v[b0 / 4] = part[0];
+  }
+}
+
+
 // float4 loads per compute thread to stage a K = 8192 / R vector
 template <int R>
 struct StageIt {
@@ -1210,11 +1265,19 @@ __device__ __forceinline__ void matvec_pages(CCtx &c, const Instr &I, Epi epi) {
   for (; t < np; t += kComputeWarps) {
     const uint32_t g = g0 + (uint32_t)t;
     if (!ring_wait(p, rg, g)) break;
-    float acc[NB][R];
-    mv_page<NB, R>(ring_page(rg, g), act, stride, B, lane, acc);
-    __syncwarp();
-    if (lane == 0) ring_release(rg, g, kComputeWarps);
-    epi(first + t, acc);
+    if constexpr (NB > 4) {
+      AccT<NB, R> acc;
+      mv_page_t<NB, R>(ring_page(rg, g), act, stride, B, lane, acc);
+      __syncwarp();
+      if (lane == 0) ring_release(rg, g, kComputeWarps);
+      epi(first + t, acc);
+    } else {
+      float acc[NB][R];
+      mv_page<NB, R>(ring_page(rg, g), act, stride, B, lane, acc);
+      __syncwarp();
+      if (lane == 0) ring_release(rg, g, kComputeWarps);
+      epi(first + t, acc);
+    }
   }
   c.g = g0 + (uint32_t)np;
 }
@@ -1643,14 +1706,16 @@ __device__ __forceinline__ uint32_t qkv_body(CCtx c, const Instr I) {
     const int qdim = p.qdim;
     const float2 *rope_s = c.sh->rope;
     const float2 *rope_g = p.rope;
-    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    matvec_pages<NB, R>(c, I, [&](int j, auto &acc) {
+      constexpr bool kT = NB > 4;  // transposed sums: every lane takes part in the shuffles
       const int head = j / pph, jj = j % pph;
-      if (lane >= half) return;
+      if (!kT && lane >= half) return;
       const int i = jj * half + lane;  // rotation pair index inside the head
   #pragma unroll
       for (int b = 0; b < NB; ++b) {
         if (NB > 1 && b >= Bn) break;
-        float u = pick<R>(acc[b], lane) * inv[b], w = pick<R>(acc[b], lane + half) * inv[b];
+        float u = acc_row<R>(acc, b, lane) * inv[b], w = acc_row<R>(acc, b, lane + half) * inv[b];
+        if (kT && lane >= half) continue;
         const int pos = NB == 1 ? pos0 : read_pos(c.sh, b);
         if (head < nq + nkv) {
           const float2 cs = NB == 1 ? rope_s[i] : __ldg(rope_g + (size_t)pos * hd + i);
@@ -1698,12 +1763,17 @@ __device__ __forceinline__ uint32_t oproj_body(CCtx c, const Instr I) {
     const uint32_t tag = c.epoch;
     const float *xrows = c.act + p.qdim - row0;
     float *const xout = p.xres + (size_t)l * Bn * H;
-    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-      if (lane >= R) return;
+    matvec_pages<NB, R>(c, I, [&](int j, auto &acc) {
+      constexpr bool kT = NB > 4;
+      if (!kT && lane >= R) return;
       const int row = j * R + lane;
       if constexpr (NB == 1) {
-        px::st_tf(xout + row, xrows[row] + pick<R>(acc[0], lane), tag);
+        px::st_tf(xout + row, xrows[row] + acc_row<R>(acc, 0, lane), tag);
       } else {
+        float av[NB];
+  #pragma unroll
+        for (int b = 0; b < NB; ++b) av[b] = (b < Bn) ? acc_row<R>(acc, b, lane) : 0.f;
+        if (kT && lane >= R) return;
         // the residual row of every sequence: one group of loads (retried as a whole)
         float xin[NB];
         for (LLRetry r;;) {
@@ -1718,7 +1788,7 @@ __device__ __forceinline__ uint32_t oproj_body(CCtx c, const Instr I) {
   #pragma unroll
         for (int b = 0; b < NB; ++b) {
           if (b >= Bn) break;
-          px::st_tf(xout + (size_t)b * H + row, xin[b] + pick<R>(acc[b], lane), tag);
+          px::st_tf(xout + (size_t)b * H + row, xin[b] + av[b], tag);
         }
       }
     });
@@ -1740,13 +1810,15 @@ __device__ __forceinline__ uint32_t gateup_body(CCtx c, const Instr I) {
     const int half = R / 2, lane = c.lane, Bn = p.B, F = p.F;
     const uint32_t tag = c.epoch;
     float *const aout = p.actb + (size_t)l * Bn * F;
-    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-      if (lane >= half) return;
+    matvec_pages<NB, R>(c, I, [&](int j, auto &acc) {
+      constexpr bool kT = NB > 4;
+      if (!kT && lane >= half) return;
       const int row = j * half + lane;
   #pragma unroll
       for (int b = 0; b < NB; ++b) {
         if (NB > 1 && b >= Bn) break;
-        const float gt = pick<R>(acc[b], lane) * inv[b], up = pick<R>(acc[b], lane + half) * inv[b];
+        const float gt = acc_row<R>(acc, b, lane) * inv[b], up = acc_row<R>(acc, b, lane + half) * inv[b];
+        if (kT && lane >= half) continue;
         const float silu = gt / (1.0f + expf(-gt));
         px::st_tf(aout + (size_t)b * F + row, silu * up, tag);
       }
@@ -1768,13 +1840,16 @@ __device__ __forceinline__ uint32_t down_body(CCtx c, const Instr I) {
     const int lane = c.lane, Bn = p.B, H = p.H;
     const uint32_t tag = c.epoch;
     float *const dout = p.dpart + ((size_t)l * p.ndp + k) * Bn * H;
-    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
-      if (lane >= R) return;
+    matvec_pages<NB, R>(c, I, [&](int j, auto &acc) {
+      constexpr bool kT = NB > 4;
+      if (!kT && lane >= R) return;
       const int row = j * R + lane;
   #pragma unroll
       for (int b = 0; b < NB; ++b) {
         if (NB > 1 && b >= Bn) break;
-        px::st_tf(dout + (size_t)b * H + row, pick<R>(acc[b], lane), tag);
+        const float v = acc_row<R>(acc, b, lane);
+        if (kT && lane >= R) continue;
+        px::st_tf(dout + (size_t)b * H + row, v, tag);
       }
     });
     return c.g;
@@ -1912,13 +1987,13 @@ __device__ __forceinline__ uint32_t lmhead_body(CCtx c, const Instr I) {
     }
     const int lane = c.lane, Bn = p.B, V = p.V;
     float *const logits = p.logits;
-    matvec_pages<NB, R>(c, I, [&](int j, float (&acc)[NB][R]) {
+    matvec_pages<NB, R>(c, I, [&](int j, auto &acc) {
       const int row = j * R + lane;
       const bool valid = lane < R && row < V;
   #pragma unroll
       for (int b = 0; b < NB; ++b) {
         if (NB > 1 && b >= Bn) break;
-        const float v = pick<R>(acc[b], lane) * inv[b];
+        const float v = acc_row<R>(acc, b, lane) * inv[b];
         if (valid) {
           if (logits && !chunk_pad(p, b)) logits[(size_t)b * V + row] = v;
           if (arg_better(v, row, bv[b], bi[b])) {
@@ -2659,6 +2734,7 @@ __device__ __forceinline__ uint32_t attn_body(CCtx c, const Instr I) {
   if constexpr (CHUNK) {
     if (nmine > 0 && !c.sh->abort) attn_block<G, DPL, PB>(q, mine, mine + 2 * D, nmine, c.lane, m, lsum, o);
   }
+  if (c.tr && c.ctid == 0) c.tr[10] = px::gtimer();
   // merge the warps
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -2939,7 +3015,11 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
       }
     }
     if (px::cbar_or(px::ld_volatile(&c.sh->abort))) break;
-    if (tr && c.ctid == 0) tr[1] = px::gtimer();
+    if (tr && c.ctid == 0) {
+      tr[1] = px::gtimer();
+      tr[10] = 0;
+      tr[11] = c.g;  // pages consumed: replaced by the difference below
+    }
     c.tr = tr;
     switch (I.op) {
       case OP_QKV:
@@ -3020,7 +3100,10 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         break;
       default: break;
     }
-    if (tr && c.ctid == 0) tr[3] = px::gtimer();
+    if (tr && c.ctid == 0) {
+      tr[3] = px::gtimer();
+      tr[11] = (uint64_t)(c.g - (uint32_t)tr[11]);
+    }
     const bool abort_now = px::cbar_or(px::ld_volatile(&c.sh->abort) != 0);
     if (abort_now) break;
     // all of this CTA's outputs of the instruction are written: publish

@@ -354,9 +354,11 @@ int mk_get_plan_info(const mk_handle *h, mk_plan_info *info);
  * 7 = (opcode | layer << 8 | cta << 16), 8 = pages the compute warps found
  * not yet landed (low 32 bits) | groups of tagged activation loads re-issued
  * because a word was not yet this step's (high 32 bits), 9 = pages the loader
- * found no free ring slot for.
+ * found no free ring slot for, 10 = attention: the first compute warp left
+ * the page loop (before the warps' merge and the split merge; 0 for other
+ * instructions), 11 = pages the instruction consumed.
  */
-#define MK_TRACE_WORDS 10
+#define MK_TRACE_WORDS 12
 int mk_trace_read(mk_handle *h, uint64_t *out, size_t n_words);
 
 /* ------------------------------------------------------------------ allocation-free step */
