@@ -3035,8 +3035,14 @@ __device__ void run_compute(CCtx &c, Queue q, volatile int *dyn_fifo, volatile i
         break;
       case OP_ATTN:
         if constexpr (kInline) c.g = attn_body<S::G, S::DPL, false>(c, I);
-        else if constexpr (S::fixed) c.g = op_attn_t<S::G, S::DPL, (NB > 1)>(c, I);
-        else c.g = op_attn<(NB > 1)>(c, I);
+        else if constexpr (S::fixed) {
+          // the prompt-chunk rows only in prompt launches: decode steps run
+          // the instantiation without them (fewer live registers)
+          if (NB > 1 && p.chunk_n > 1) c.g = op_attn_t<S::G, S::DPL, (NB > 1)>(c, I);
+          else c.g = op_attn_t<S::G, S::DPL, false>(c, I);
+        } else {
+          c.g = op_attn<(NB > 1)>(c, I);
+        }
         break;
       case OP_OPROJ:
         if constexpr (NB > 1 && S::fixed && S::TQO) {
