@@ -37,6 +37,7 @@ struct mk_handle {
   // tagged fp32 activation words (the step number mod 4 in the two low
   // mantissa bits)
   float *qbuf = nullptr, *obuf = nullptr, *xres = nullptr, *actb = nullptr, *dpart = nullptr, *kvcur = nullptr;
+  int dpart_pieces = 0;  // down-projection K pieces dpart holds per layer and sequence
   unsigned *ctr_epoch = nullptr;  // [0] = epoch
   // every tagged buffer (pointer, bytes): zeroed whenever the step number restarts
   std::vector<std::pair<void *, size_t>> tagged;
@@ -434,9 +435,12 @@ extern "C" int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_
     cudaGetLastError();
     return fail(MK_ERR_CUDA);
   }
-  // geometry (independent of batch and CTA count)
+  // geometry of the CUDA-core page layouts (independent of batch and CTA
+  // count; a tensor-core plan's down pieces are its own)
   PlanRequest req = make_request(*cfg, default_opts(*cfg), 1);
   req.B = 1;
+  req.tensor = false;
+  req.tensor_qkv_o = false;
   Plan geo;
   std::string err = build_plan(req, &geo);
   if (!err.empty()) return fail(MK_ERR_UNSUPPORTED_SHAPE);
@@ -453,7 +457,11 @@ extern "C" int mk_create(const mk_config *cfg, const mk_weights *w, const mk_kv_
   if ((rc = tagged(&h->obuf, (size_t)s.L * Bm * s.nq * s.d))) return fail(rc);
   if ((rc = tagged(&h->xres, (size_t)s.L * Bm * s.H))) return fail(rc);
   if ((rc = tagged(&h->actb, (size_t)s.L * Bm * s.F))) return fail(rc);
-  if ((rc = tagged(&h->dpart, (size_t)s.L * geo.ndp * Bm * s.H))) return fail(rc);
+  // the partial sums of every K piece of the down projection, for the plan
+  // with the most pieces (tensor-core plans split K finer than the CUDA-core
+  // layout)
+  h->dpart_pieces = down_pieces_max(s);
+  if ((rc = tagged(&h->dpart, (size_t)s.L * h->dpart_pieces * Bm * s.H))) return fail(rc);
   if ((rc = tagged(&h->kvcur, (size_t)s.L * Bm * 2 * s.nkv * s.d))) return fail(rc);
   if ((rc = dalloc(h->allocs, &h->ctr_epoch, 4))) return fail(rc);
   if ((rc = dalloc(h->allocs, &h->status, kStatusWords))) return fail(rc);
@@ -508,6 +516,7 @@ extern "C" int mk_plan(mk_handle *h, const mk_plan_opts *opts_in) {
   Plan p;
   std::string err = build_plan(req, &p);
   if (err.empty()) err = validate_plan(req, p);
+  if (err.empty() && p.ndp > h->dpart_pieces) err = "more down-projection pieces than the partial-sum buffer holds";
   if (!err.empty()) {
     fprintf(stderr, "mk_plan: %s\n", err.c_str());
     return MK_ERR_UNSUPPORTED_SHAPE;

@@ -19,7 +19,7 @@ constexpr int kThreads = 32 * (kLoaders + kComputeWarps);
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kMaxKc = 4096;                  // largest K staged in one page row
 constexpr int kMaxBatch = 16;
-constexpr int kMaxDownPieces = 8;             // ffn / 2048 at most
+constexpr int kMaxDownPieces = 8;             // down-projection K pieces at most
 constexpr int kDefaultInflight = 4;           // bulk-copy pages in flight per CTA
 constexpr int kTcXchFloats = 128 * 16;        // batched builds: tensor-core epilogue exchange (floats)
 constexpr int kSplitRedFloats = 1024;         // batch 1: split-page row partials (floats, staging region)

@@ -30,6 +30,13 @@ static bool pow2_in(int x, int lo, int hi) {
 }
 
 static int down_kc(int F) { return F <= 2048 ? F : 2048; }
+// Tensor-core plans split the down projection's K into pieces of 1024 when the
+// piece count allows: one 128-row tile per instruction, so at hidden 2048 and
+// ffn 8192 that is 128 instructions of 16 pages instead of 64 of 32 (64 of
+// the 148 SMs busy), at the price of 1 + 8 instead of 1 + 4 loads per element
+// in the tile's sum.  The CUDA-core layout (rows per page) keeps down_kc.
+static int down_kc_tensor(int F) { return (F % 1024 == 0 && F / 1024 <= kMaxDownPieces) ? 1024 : down_kc(F); }
+int down_pieces_max(const Shape &s) { return std::max(s.F / down_kc(s.F), s.F / down_kc_tensor(s.F)); }
 
 std::string check_shape(const Shape &s, int B) {
   char buf[256];
@@ -153,7 +160,8 @@ std::string build_plan(const PlanRequest &req, Plan *out) {
   p.Rh = kPageElems / s.H;
   p.Ro = kPageElems / (s.nq * s.d);
   p.KCd = down_kc(s.F);
-  p.Rd = kPageElems / p.KCd;
+  p.Rd = kPageElems / p.KCd;  // rows per page of the CUDA-core down layout
+  if (req.tensor) p.KCd = down_kc_tensor(s.F);
   p.ndp = s.F / p.KCd;
   const int G = s.nq / s.nkv;
   if (req.S > 0) {

@@ -82,6 +82,9 @@ std::string check_shape(const Shape &s, int B);
 
 // Build a plan.  Returns "" on success, else an error message.
 std::string build_plan(const PlanRequest &req, Plan *out);
+// The most down-projection K pieces any plan of this shape uses (buffers of
+// per-piece partial sums are sized for it).
+int down_pieces_max(const Shape &s);
 
 // Structural validation: every dependency is produced by instructions that
 // come earlier in the global order, every queue is a subsequence of that

@@ -214,9 +214,11 @@ def test_batched_plan_uses_tensor_core_tiles():
         gu = [i for i in instrs if i.op == OP["gateup"] and i.layer == l]
         assert sorted((i.a, i.a + i.b) for i in gu)[0][0] == 0
         assert sum(i.b for i in gu) == F // 64
-        for k in range(F // 2048):
-            dn = [i for i in instrs if i.op == OP["down"] and i.layer == l and i.c == k]
-            assert sum(i.b for i in dn) == H // 128
+        # the down projection in K pieces of 1024 columns, one 128-row tile per
+        # instruction: every (piece, tile) once
+        dn = [i for i in instrs if i.op == OP["down"] and i.layer == l]
+        assert all(i.b == 1 for i in dn)
+        assert sorted((i.c, i.a) for i in dn) == [(k, t) for k in range(F // 1024) for t in range(H // 128)]
     lm = [i for i in instrs if i.op == OP["lmhead"]]
     assert sum(i.b for i in lm) == -(-V // 128)
     err = mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=16), 148, steps=1, seed=5, timeout_ms=20000)
@@ -259,6 +261,9 @@ def test_use_tcgen05_option():
     assert gu_units(auto) == gu_units(on) == F // 64          # 128-row tiles of 64 gate + 64 up rows
     rows_per_page = 16384 // (2 * cfg.hidden)
     assert gu_units(off) == F // (rows_per_page // 2)           # one page of R/2 gate + R/2 up rows each
+    # down K pieces: 1024 columns on the tensor cores, 2048 (the page rows' width) on CUDA cores
+    pieces = lambda ins: sorted({i.c for i in ins if i.op == OP["down"] and i.layer == 0})
+    assert pieces(on) == list(range(F // 1024)) and pieces(off) == list(range(F // 2048))
     assert mk.mk_host_plan_simulate(cfg, mk.plan_opts(batch=16, use_tcgen05=-1), 148, steps=1, seed=3,
                                     timeout_ms=20000) == ""
     cfg1 = cfg_for("llama1b")
