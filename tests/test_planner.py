@@ -123,8 +123,11 @@ def test_kv_splits_rule_cost_model_and_explicit(name):
     items = B * w.shape.n_kv_heads
     rule = max(1, min(148 // items, cfg.max_seq // 32))
     if B > 1:
-        rule = max(rule, min(4 * 148 // items, cfg.max_seq // 256))
+        rule = max(rule, min(3 * 148 // items, cfg.max_seq // 256))
     assert info.kv_splits == max(1, min(rule, 64))
+    if B > 1:  # at the contexts the batched bench decodes (up to 4096 + its steps): 3 splits
+        *_, info16 = mk.mk_host_plan(cfg_for(name, max_batch=B, max_seq=4200), mk.plan_opts(batch=B), 148)
+        assert info16.kv_splits == 3
     est = lambda S: mk.mk_host_plan_estimate(cfg, mk.plan_opts(batch=B, kv_splits=S), 148, cfg.max_seq - 1).step_us
     assert info.estimated_step_us == round(est(info.kv_splits))
     *_, info = mk.mk_host_plan(cfg, mk.plan_opts(batch=B, kv_splits=-1), 148)
